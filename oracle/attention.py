@@ -1,0 +1,270 @@
+"""fp64 reference for scaled-dot-product attention (bf16 path and decode).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): the tests, the smoke
+check and the benchmark's CPU baseline call this; the product never does.
+
+Everything is float64 numpy.  Inputs may be any real dtype; bf16 tensors are
+converted exactly (every bf16 value is a float64 value).  Shapes are
+[B][H][N][d] as in [FA-trading] "Integration in eight lines" (q, k, v shaped
+(batch, heads, seq, head_dim)).
+
+Causal alignment (the pages only say "the model must not look at the future",
+[FA-trading] "Causal masking"): key j is visible to query i iff
+j <= i + (Nkv - Nq), i.e. the last query sees every key.  For Nq == Nkv this is
+the usual lower-triangular mask of the explicit-score code in "Integration in
+eight lines".  A query row that sees no key gets O = 0 and LSE = -inf.
+
+LSE is the natural-log log-sum-exp of the scaled scores,
+LSE_i = log sum_j exp(scale * q_i . k_j): the per-row softmax statistics that
+[FA-trading] "Backward: recompute instead of store" keeps instead of P.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+LOG2E = 1.0 / math.log(2.0)
+LN2 = math.log(2.0)
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion of a numpy array or a torch tensor to float64 numpy."""
+    if hasattr(x, "detach"):  # torch tensor, any dtype; .double() is exact
+        return x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def visible_mask(Nq: int, Nkv: int, causal: bool, rows=None) -> np.ndarray:
+    """Boolean [rows][Nkv]: True where key j is visible to query i."""
+    i = np.arange(Nq) if rows is None else np.asarray(rows)
+    j = np.arange(Nkv)
+    if not causal:
+        return np.ones((i.size, Nkv), dtype=bool)
+    return j[None, :] <= (i[:, None] + (Nkv - Nq))
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None,
+              rows=None, row_chunk: int = 1024):
+    """O = softmax(scale * Q K^T, masked) V and LSE, the plain definition.
+
+    [FA-trading] "Why attention is memory-bound": softmax(Q K^T / sqrt(d_k)) V,
+    with the N x N score matrix S = Q K^T / sqrt(d_k) materialised;
+    "Integration in eight lines": scores, masked_fill(-inf), softmax, matmul.
+
+    ``rows`` optionally restricts the computation to a subset of query rows
+    (same rows for every (b, h)); the result then has len(rows) query rows.
+    Rows are processed ``row_chunk`` at a time (rows are independent, so this is
+    the same definition, only with less memory).
+
+    Returns (O [B,H,R,d] float64, LSE [B,H,R] float64).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    row_idx = np.arange(Nq) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = row_idx.size
+    O = np.zeros((B, H, R, v.shape[3]), dtype=np.float64)
+    LSE = np.full((B, H, R), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, R, row_chunk):
+                ri = row_idx[r0:r0 + row_chunk]
+                S = (q[b, h, ri] @ k[b, h].T) * scale           # [r, Nkv]
+                S = np.where(visible_mask(Nq, Nkv, causal, ri), S, -np.inf)
+                m = S.max(axis=1)
+                alive = np.isfinite(m)
+                m_safe = np.where(alive, m, 0.0)
+                P = np.exp(S - m_safe[:, None])                  # exp(-inf) = 0
+                l = P.sum(axis=1)
+                l_safe = np.where(alive, l, 1.0)
+                P = P / l_safe[:, None]
+                O[b, h, r0:r0 + ri.size] = np.where(alive[:, None], P @ v[b, h], 0.0)
+                LSE[b, h, r0:r0 + ri.size] = np.where(alive, m_safe + np.log(l_safe),
+                                                       -np.inf)
+    return O, LSE
+
+
+def softmax_rows(q, k, causal: bool = False, scale: float | None = None):
+    """The normalised probability matrix P [B,H,Nq,Nkv] (small inputs only)."""
+    q, k = _f64(q), _f64(k)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = np.einsum("bhid,bhjd->bhij", q, k) * scale
+    S = np.where(visible_mask(Nq, Nkv, causal)[None, None], S, -np.inf)
+    m = S.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    P = np.exp(S - m)
+    l = P.sum(axis=-1, keepdims=True)
+    return P / np.where(l > 0, l, 1.0)
+
+
+def _exp_shift(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """exp(a - b) with the convention exp(-inf - (-inf)) = 0 (nothing seen yet)."""
+    out = np.zeros(np.broadcast(a, b).shape)
+    ok = np.isfinite(a) & np.isfinite(b)
+    np.exp(np.where(ok, a - np.where(np.isfinite(b), b, 0.0), 0.0), out=out, where=ok)
+    return out
+
+
+def attention_blockwise(q, k, v, causal: bool = False, scale: float | None = None,
+                        Br: int = 128, Bc: int = 128):
+    """The tiled forward as [FA-trading] "The Flash Attention algorithm" states
+    it: Q in T_r = ceil(N/B_r) row blocks, K/V in T_c = ceil(N/B_c) column
+    blocks; per KV block a local row max m_ij, P_ij = exp(S_ij - m_ij), local
+    sum l_ij, then the running (m, l) and the normalised output O_i updated with
+    the factors l_i e^{m_i - m_new} / l_new and e^{m_ij - m_new} / l_new.
+
+    A second, independent route to the same numbers as ``attention``; used by
+    the oracle's self-tests.  Returns (O, LSE) with LSE = m + log l.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((B, H, Nq, v.shape[3]))
+    LSE = np.full((B, H, Nq), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, Nq, Br):
+                rows = np.arange(i0, min(Nq, i0 + Br))
+                Oi = np.zeros((rows.size, v.shape[3]))
+                mi = np.full(rows.size, -np.inf)
+                li = np.zeros(rows.size)
+                vis = visible_mask(Nq, Nkv, causal, rows)
+                for j0 in range(0, Nkv, Bc):
+                    cols = slice(j0, min(Nkv, j0 + Bc))
+                    Sij = (q[b, h, rows] @ k[b, h, cols].T) * scale
+                    Sij = np.where(vis[:, cols], Sij, -np.inf)
+                    mij = Sij.max(axis=1)
+                    Pij = _exp_shift(Sij, mij[:, None])
+                    lij = Pij.sum(axis=1)
+                    m_new = np.maximum(mi, mij)
+                    a_old = li * _exp_shift(mi, m_new)
+                    a_new = _exp_shift(mij, m_new)
+                    l_new = a_old + lij * a_new
+                    ok = l_new > 0
+                    inv = np.where(ok, 1.0 / np.where(ok, l_new, 1.0), 0.0)
+                    Oi = Oi * (a_old * inv)[:, None] + (Pij @ v[b, h, cols]) * (a_new * inv)[:, None]
+                    mi, li = m_new, l_new
+                O[b, h, rows] = Oi
+                LSE[b, h, rows] = np.where(li > 0, mi + np.log(np.where(li > 0, li, 1.0)),
+                                           -np.inf)
+    return O, LSE
+
+
+def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = None,
+                           Bc: int = 128, tau: float = 8.0, count_rescales: bool = False):
+    """The deferred-normalisation form with lazy rescaling, base 2.
+
+    [FA-trading] "FA2" item 1: the output accumulator stays unnormalised and is
+    divided by l once after the inner loop.  [FA4-overview] "Smarter online
+    softmax rescaling": the reference maximum only moves (and O, l are only
+    rescaled) when the new block maximum exceeds it by a significant amount;
+    the pages give no constant, ``tau`` is that amount in log2 units (tau = 0
+    rescales on every increase, the classic recurrence of "Online softmax
+    recurrence").  Scores are handled as base-2 logits x = scale * S * log2(e)
+    ([FA4-overview] "Software exponent on CUDA cores": the kernel evaluates
+    exp2).  Exact in exact arithmetic for every tau, because O and l share the
+    same stale reference.
+
+    Returns (O, LSE) and, if ``count_rescales``, the number of (row, block)
+    pairs in which the reference moved after the first block.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((B, H, Nq, v.shape[3]))
+    LSE = np.full((B, H, Nq), -np.inf)
+    vis = visible_mask(Nq, Nkv, causal)
+    rescales = 0
+    for b in range(B):
+        for h in range(H):
+            acc = np.zeros((Nq, v.shape[3]))
+            l = np.zeros(Nq)
+            m = np.full(Nq, -np.inf)
+            for jb, j0 in enumerate(range(0, Nkv, Bc)):
+                cols = slice(j0, min(Nkv, j0 + Bc))
+                x = (q[b, h] @ k[b, h, cols].T) * (scale * LOG2E)
+                x = np.where(vis[:, cols], x, -np.inf)
+                m_blk = x.max(axis=1)
+                m_new = np.maximum(m, m_blk)
+                move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
+                if jb > 0:
+                    rescales += int(np.count_nonzero(move & np.isfinite(m)))
+                f = np.where(move & np.isfinite(m),
+                             np.exp2(np.where(move & np.isfinite(m), m - m_new, 0.0)), 1.0)
+                acc *= f[:, None]
+                l *= f
+                m = np.where(move, m_new, m)
+                p = np.zeros_like(x)
+                fin = np.isfinite(x) & np.isfinite(m)[:, None]
+                np.exp2(np.where(fin, x - np.where(np.isfinite(m), m, 0.0)[:, None], 0.0),
+                        out=p, where=fin)
+                l += p.sum(axis=1)
+                acc += p @ v[b, h, cols]
+            ok = l > 0
+            ls = np.where(ok, l, 1.0)
+            O[b, h] = np.where(ok[:, None], acc / ls[:, None], 0.0)
+            LSE[b, h] = np.where(ok, LN2 * (np.where(ok, m, 0.0) + np.log2(ls)), -np.inf)
+    if count_rescales:
+        return O, LSE, rescales
+    return O, LSE
+
+
+def split_bounds(Nkv: int, num_splits: int):
+    """Key ranges of a split-KV decode: equal chunks of ceil(Nkv / splits) keys
+    (the last ones may be short or empty)."""
+    chunk = -(-Nkv // num_splits)
+    return [(min(Nkv, c * chunk), min(Nkv, (c + 1) * chunk)) for c in range(num_splits)]
+
+
+def decode_partials(q, k, v, scale: float | None = None, num_splits: int = 16):
+    """Per split c: attention of the query rows over keys of chunk c alone,
+    giving (O_c, LSE_c).  An empty chunk gives O_c = 0, LSE_c = -inf.
+
+    Returns (O_parts [S,B,H,Nq,d], LSE_parts [S,B,H,Nq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Os, Ls = [], []
+    for lo, hi in split_bounds(k.shape[2], num_splits):
+        if hi <= lo:
+            Os.append(np.zeros((B, H, Nq, v.shape[3])))
+            Ls.append(np.full((B, H, Nq), -np.inf))
+            continue
+        o, lse = attention(q, k[:, :, lo:hi], v[:, :, lo:hi], False, scale)
+        Os.append(o)
+        Ls.append(lse)
+    return np.stack(Os), np.stack(Ls)
+
+
+def combine(O_parts, LSE_parts):
+    """LSE-weighted merge of split results: LSE = log sum_c exp(LSE_c) and
+    O = sum_c exp(LSE_c - LSE) O_c.  The same identity as the online-softmax
+    recurrence ([FA-trading] "Online softmax recurrence"), applied once to
+    whole chunks instead of tile by tile."""
+    O_parts, LSE_parts = _f64(O_parts), _f64(LSE_parts)
+    mx = LSE_parts.max(axis=0)
+    alive = np.isfinite(mx)
+    mxs = np.where(alive, mx, 0.0)
+    w = _exp_shift(LSE_parts, mxs[None])
+    tot = w.sum(axis=0)
+    tots = np.where(alive, tot, 1.0)
+    O = np.where(alive[..., None], (w[..., None] * O_parts).sum(axis=0) / tots[..., None], 0.0)
+    LSE = np.where(alive, mxs + np.log(tots), -np.inf)
+    return O, LSE
+
+
+def decode(q, k, v, scale: float | None = None):
+    """Decode reference: one (or a few) query rows against the whole cache,
+    which is the plain definition (non-causal over all cached keys)."""
+    return attention(q, k, v, causal=False, scale=scale)

@@ -1,0 +1,192 @@
+"""Pins of the fp64 oracle (bf16 path and decode) to facts fixed outside it.
+
+Closed forms, invariants, an independent library routine (PyTorch's fp64
+scaled_dot_product_attention on the CPU, the drop-in named by the
+Flash Attention trading-models page, "Integration in eight lines"), brute force
+on tiny inputs, and the pages' own blockwise algorithm.  No GPU.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+
+RNG = np.random.default_rng(1234)
+
+
+def rand(*shape, scale=1.0):
+    return RNG.standard_normal(shape) * scale
+
+
+def test_single_key_gives_that_value_row():
+    q, k, v = rand(2, 3, 5, 8), rand(2, 3, 1, 8), rand(2, 3, 1, 8)
+    O, L = A.attention(q, k, v, False, 0.3)
+    assert np.array_equal(O, np.broadcast_to(v, O.shape))
+    np.testing.assert_allclose(L, 0.3 * np.einsum("bhid,bhjd->bhi", q, k), rtol=0, atol=1e-14)
+
+
+def test_equal_scores_give_mean_of_values():
+    q = np.zeros((1, 2, 4, 16))
+    k, v = rand(1, 2, 37, 16), rand(1, 2, 37, 16)
+    O, L = A.attention(q, k, v, False, 0.125)
+    np.testing.assert_allclose(O, np.broadcast_to(v.mean(axis=2, keepdims=True), O.shape),
+                               rtol=0, atol=1e-14)
+    np.testing.assert_allclose(L, math.log(37.0), rtol=0, atol=1e-14)
+
+
+def test_causal_first_row_sees_only_first_key():
+    q, k, v = rand(1, 2, 9, 4), rand(1, 2, 9, 4), rand(1, 2, 9, 4)
+    O, L = A.attention(q, k, v, True, 0.5)
+    np.testing.assert_array_equal(O[:, :, 0], v[:, :, 0])
+    np.testing.assert_allclose(L[:, :, 0], 0.5 * (q[:, :, 0] * k[:, :, 0]).sum(-1), atol=1e-15)
+
+
+def test_probability_rows_sum_to_one_and_mask_future():
+    q, k = rand(1, 3, 11, 8, scale=3), rand(1, 3, 11, 8, scale=3)
+    for causal in (False, True):
+        P = A.softmax_rows(q, k, causal, 0.7)
+        assert (P >= 0).all()
+        np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-12)
+        if causal:
+            assert (P[..., np.triu_indices(11, 1)[0], np.triu_indices(11, 1)[1]] == 0).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nkv,d", [(1, 1, 1), (5, 7, 3), (7, 5, 3), (33, 70, 16), (64, 64, 64)])
+def test_matches_torch_sdpa_fp64(causal, Nq, Nkv, d):
+    """Independent library routine.  torch's is_causal is top-left aligned; the
+    oracle is bottom-right aligned, so causal cases use an explicit bool mask."""
+    q, k, v = rand(2, 3, Nq, d), rand(2, 3, Nkv, d), rand(2, 3, Nkv, d)
+    scale = 1.0 / math.sqrt(d)
+    O, L = A.attention(q, k, v, causal, scale)
+    tq, tk, tv = (torch.from_numpy(t) for t in (q, k, v))
+    mask = None
+    if causal:
+        i = torch.arange(Nq)[:, None]
+        j = torch.arange(Nkv)[None, :]
+        mask = j <= i + (Nkv - Nq)
+    dead = (mask is not None) and (~mask.any(dim=1)).any().item()
+    if not dead:
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                               scale=scale).numpy()
+        np.testing.assert_allclose(O, ref, rtol=0, atol=1e-12)
+    S = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
+    if mask is not None:
+        S = S.masked_fill(~mask, float("-inf"))
+    np.testing.assert_allclose(L, torch.logsumexp(S, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_fully_masked_rows_are_zero_with_minus_inf_lse():
+    # Nq > Nkv with bottom-right alignment: the first Nq - Nkv rows see nothing.
+    q, k, v = rand(1, 1, 6, 4), rand(1, 1, 3, 4), rand(1, 1, 3, 4)
+    O, L = A.attention(q, k, v, True, 1.0)
+    assert (O[0, 0, :3] == 0).all() and np.isneginf(L[0, 0, :3]).all()
+    np.testing.assert_array_equal(O[0, 0, 3], v[0, 0, 0])
+
+
+def test_brute_force_loops_tiny():
+    q, k, v = rand(1, 1, 3, 2), rand(1, 1, 4, 2), rand(1, 1, 4, 2)
+    scale = 0.9
+    for causal in (False, True):
+        O, L = A.attention(q, k, v, causal, scale)
+        for i in range(3):
+            w = []
+            for j in range(4):
+                if causal and j > i + 1:
+                    continue
+                w.append((j, math.exp(scale * sum(q[0, 0, i, c] * k[0, 0, j, c] for c in range(2)))))
+            z = sum(e for _, e in w)
+            for c in range(2):
+                o = sum(e * v[0, 0, j, c] for j, e in w) / z
+                assert abs(O[0, 0, i, c] - o) < 1e-13
+            assert abs(L[0, 0, i] - math.log(z)) < 1e-13
+
+
+def test_causal_future_perturbation_leaves_rows_unchanged():
+    q, k, v = rand(1, 2, 16, 8), rand(1, 2, 16, 8), rand(1, 2, 16, 8)
+    O, L = A.attention(q, k, v, True, 0.4)
+    for i in (0, 5, 14):
+        k2, v2 = k.copy(), v.copy()
+        k2[:, :, i + 1:] = rand(1, 2, 15 - i, 8, scale=50)
+        v2[:, :, i + 1:] = rand(1, 2, 15 - i, 8, scale=50)
+        O2, L2 = A.attention(q, k2, v2, True, 0.4)
+        assert np.array_equal(O2[:, :, :i + 1], O[:, :, :i + 1])
+        assert np.array_equal(L2[:, :, :i + 1], L[:, :, :i + 1])
+
+
+def test_key_shift_and_permutation_invariance():
+    q, k, v = rand(1, 2, 8, 6), rand(1, 2, 13, 6), rand(1, 2, 13, 6)
+    O, L = A.attention(q, k, v, False, 0.3)
+    c = rand(6)
+    O2, L2 = A.attention(q, k + c, v, False, 0.3)
+    np.testing.assert_allclose(O2, O, atol=1e-12)
+    np.testing.assert_allclose(L2, L + 0.3 * q @ c, atol=1e-12)
+    perm = RNG.permutation(13)
+    O3, L3 = A.attention(q, k[:, :, perm], v[:, :, perm], False, 0.3)
+    np.testing.assert_allclose(O3, O, atol=1e-13)
+    np.testing.assert_allclose(L3, L, atol=1e-13)
+
+
+def _adversarial(N, d):
+    """Scores that grow block after block (every block raises the max) mixed
+    with +-1e3 magnitudes."""
+    q = rand(1, 1, N, d)
+    k = rand(1, 1, N, d)
+    k *= np.linspace(0.1, 30, N)[None, None, :, None]
+    k[0, 0, N // 2] *= 1e3 / max(1.0, np.abs(k[0, 0, N // 2]).max())
+    return q, k, rand(1, 1, N, d)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Br,Bc", [(1, 1), (2, 3), (3, 2), (4, 9), (9, 9)])
+def test_pages_blockwise_algorithm_equals_definition(causal, Br, Bc):
+    q, k, v = _adversarial(9, 3)
+    O, L = A.attention(q, k, v, causal, 0.8)
+    Ob, Lb = A.attention_blockwise(q, k, v, causal, 0.8, Br, Bc)
+    np.testing.assert_allclose(Ob, O, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(Lb, L, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Bc", [1, 2, 3, 9])
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_lazy_rescale_equals_definition(causal, Bc, tau):
+    q, k, v = _adversarial(9, 3)
+    O, L = A.attention(q, k, v, causal, 0.8)
+    Ol, Ll = A.attention_lazy_rescale(q, k, v, causal, 0.8, Bc, tau)
+    np.testing.assert_allclose(Ol, O, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(Ll, L, rtol=1e-12, atol=1e-12)
+
+
+def test_lazy_rescale_moves_the_reference_less_often():
+    q, k, v = rand(1, 2, 256, 32), rand(1, 2, 1024, 32), rand(1, 2, 1024, 32)
+    *_, r0 = A.attention_lazy_rescale(q, k, v, False, 1 / math.sqrt(32), 64, 0.0, True)
+    *_, r8 = A.attention_lazy_rescale(q, k, v, False, 1 / math.sqrt(32), 64, 8.0, True)
+    assert r8 < r0 and r8 == 0
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 16, 40])
+def test_split_kv_combine_equals_unsplit(splits):
+    q, k, v = rand(3, 2, 1, 16), rand(3, 2, 37, 16), rand(3, 2, 37, 16)
+    O, L = A.decode(q, k, v, 0.25)
+    Op, Lp = A.decode_partials(q, k, v, 0.25, splits)
+    Oc, Lc = A.combine(Op, Lp)
+    np.testing.assert_allclose(Oc, O, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(Lc, L, rtol=0, atol=1e-13)
+
+
+def test_split_bounds_cover_all_keys_once():
+    for N, s in [(8192, 16), (37, 40), (1, 3), (100, 7)]:
+        b = A.split_bounds(N, s)
+        assert len(b) == s and b[0][0] == 0 and b[-1][1] == N
+        assert all(b[i][1] == b[i + 1][0] for i in range(s - 1))
+
+
+def test_bf16_inputs_convert_exactly():
+    t = torch.randn(2, 2, 5, 8).to(torch.bfloat16)
+    O, _ = A.attention(t, t, t, False, 0.1)
+    O2, _ = A.attention(t.float().numpy().astype(np.float64), t.float().numpy(), t.float().numpy(),
+                        False, 0.1)
+    assert np.array_equal(O, O2)
