@@ -1,0 +1,136 @@
+/*
+ * tiledattn -- fused tiled scaled-dot-product attention forward for NVIDIA
+ * B200 (sm_100a), C ABI.
+ *
+ * Sources, cited by page title and section:
+ *   [FA-trading]   "Can a full-day context beat one minute? Flash attention and
+ *                  the sequence-length question" (marketmaker.cc blog)
+ *   [FA4-overview] "FlashAttention 4: fast, memory-saving attention for LLMs"
+ *                  (linux-konsole)
+ *   [FP4-FA4]      "Hardware-Aware FP4 FlashAttention-4" (gist.science summary)
+ *   [INT-FA]       "INT-FlashAttention: an INT8 quantisation architecture
+ *                  compatible with FlashAttention" (hoodcat.net)
+ *
+ * Conventions shared by every call
+ *   - Tensor arguments are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or retains them.  Layout is contiguous row-major
+ *     [B][H][N][d] (q, k, v shaped (batch, heads, seq, head_dim) as in
+ *     [FA-trading] "Integration in eight lines"); LSE is [B][H][N_q].
+ *   - bf16 tensors are passed as `attn_bf16_t` (the raw 16-bit pattern).
+ *   - Tensor pointers must be 16-byte aligned (TMA and vector loads);
+ *     float outputs 4-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous: the return value reports argument
+ *     errors and launch errors only.  A device-side watchdog (every wait in a
+ *     kernel has a time limit) reports ATTN_ERR_TIMEOUT through
+ *     attn_check_status().
+ *   - Causal semantics: key j is visible to query i iff j <= i + (N_kv - N_q)
+ *     (the last query sees every key; for N_q == N_kv this is the usual
+ *     lower-triangular mask, [FA-trading] "Causal masking").  A query row that
+ *     sees no key gets O = 0 and LSE = -inf.
+ *   - LSE is the natural-log log-sum-exp of the scaled scores of the row, the
+ *     O(N) softmax statistic kept for the backward pass ([FA-trading]
+ *     "Backward: recompute instead of store").
+ *   - scale must be finite and > 0 (normally 1/sqrt(d)).
+ *   - There is no fallback: an unsupported shape returns an error code.
+ */
+#ifndef TILEDATTN_H
+#define TILEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+typedef uint16_t attn_bf16_t;
+
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad scale      */
+  ATTN_ERR_UNSUPPORTED = -2, /* head dim or shape outside what is built     */
+  ATTN_ERR_MISALIGNED = -3,  /* pointer not 16-byte aligned                 */
+  ATTN_ERR_CUDA = -4,        /* CUDA runtime/driver error at launch         */
+  ATTN_ERR_TIMEOUT = -5      /* a kernel wait ran past its time limit       */
+};
+
+/* Human-readable name of a status code (static string). */
+ATTN_API const char* attn_status_string(int status);
+
+/* Library version, e.g. "tiledattn 0.1 sm_100a". */
+ATTN_API const char* attn_version(void);
+
+/*
+ * attn_fwd -- bf16 attention forward, fp32 accumulation.
+ *
+ * [FA-trading] "The Flash Attention algorithm" (Q in B_r-row blocks, K/V in
+ * B_c-column blocks, S_ij never leaves the chip), "Online softmax recurrence"
+ * (running max m, running sum l, retroactive rescale of O), "FA2" (one
+ * division by l after the inner loop; parallel over query blocks), "Causal
+ * masking" (tiles entirely in the future are skipped); [FA4-overview]
+ * "What is new in FlashAttention 4" (warp-specialised load / MMA / softmax /
+ * correction / store roles) and "Smarter online softmax rescaling" (the
+ * reference max only moves when it rises by more than 8 in log2 units).
+ *
+ *   q   [B][H][Nq][d]  bf16      k, v [B][H][Nkv][d] bf16
+ *   o   [B][H][Nq][d]  bf16 out  lse  [B][H][Nq]     fp32 out (natural log)
+ *   d in {64, 128}; Nq, Nkv >= 0 (Nq == 0 or B*H == 0: nothing to do;
+ *   Nkv == 0: every row gets O = 0, LSE = -inf).
+ */
+ATTN_API int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+             float* lse, int B, int H, int Nq, int Nkv, int d, int causal, float scale,
+             void* stream);
+
+/*
+ * attn_decode -- split-KV decode: ONE query row per (batch, head) against a
+ * KV cache of Nkv keys; the key range is cut into num_splits equal chunks of
+ * ceil(Nkv / num_splits) keys, each chunk gives a partial (O_c, LSE_c) in the
+ * workspace, and a combine kernel merges them:
+ *   LSE = log sum_c exp(LSE_c),  O = sum_c exp(LSE_c - LSE) O_c.
+ * The merge is the online-softmax identity ([FA-trading] "Online softmax
+ * recurrence") applied to whole chunks.
+ *
+ *   q [B][H][1][d] bf16, k, v [B][H][Nkv][d] bf16, o [B][H][1][d] bf16 out,
+ *   lse [B][H] fp32 out; d in {64, 128}; 1 <= num_splits <= 1024; Nkv >= 1.
+ *   workspace: device scratch of at least attn_decode_workspace_bytes(...)
+ *   bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *   matter and are overwritten.  Calls that share a workspace must not
+ *   overlap in time.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits);
+ATTN_API int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                float* lse, int B, int H, int Nkv, int d, float scale, int num_splits,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_check_status -- synchronise `stream`, read the device status word
+ * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT), clear it and
+ * return it; also returns ATTN_ERR_CUDA if the synchronisation itself fails.
+ */
+ATTN_API int attn_check_status(void* stream);
+
+/*
+ * attn_set_wait_limit_ns -- time limit of every in-kernel wait (default
+ * 1e9 ns).  Applies to launches made after the call.  0 restores the default.
+ */
+ATTN_API void attn_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * attn_watchdog_selftest -- launch one CTA that waits on a barrier nothing
+ * ever arrives at, with a limit of `limit_ns`.  The wait gives up, the kernel
+ * records ATTN_ERR_TIMEOUT and returns normally; attn_check_status() then
+ * reports it.  Exercises the timeout path without a fault or a hang.
+ */
+ATTN_API int attn_watchdog_selftest(unsigned long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TILEDATTN_H */

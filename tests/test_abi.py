@@ -1,0 +1,88 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/tiledattn.h declares, and rejects bad arguments on the host before
+touching the device.  No GPU (no call here reaches CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(attn_\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_24_b200 import build
+    build.build()
+    from tiled_attention_24_b200 import _binding
+    return _binding.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"attn_fwd", "attn_decode", "attn_check_status"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+def test_binding_covers_every_declared_symbol():
+    from tiled_attention_24_b200 import _binding
+    assert _declared() == {n for n, _, _ in _binding.SIGNATURES}
+
+
+def test_status_strings(lib):
+    assert lib.attn_status_string(0) == b"ATTN_OK"
+    assert lib.attn_status_string(-5) == b"ATTN_ERR_TIMEOUT"
+    assert b"sm_100a" in lib.attn_version()
+
+
+P = ctypes.c_void_p(16 * 1000)  # never dereferenced: validation rejects first
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(d=96), -2), (dict(d=32), -2), (dict(scale=0.0), -1), (dict(scale=float("nan")), -1),
+    (dict(scale=-1.0), -1), (dict(B=-1), -1), (dict(Nq=-3), -1), (dict(q=None), -1),
+    (dict(q=ctypes.c_void_p(16 * 1000 + 2)), -3), (dict(lse=ctypes.c_void_p(16 * 1000 + 1)), -3),
+    (dict(B=0), 0), (dict(Nq=0), 0),
+])
+def test_fwd_host_validation(lib, args, code):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Nq=8, Nkv=8, d=64, causal=0, scale=0.125, stream=None)
+    a.update(args)
+    rc = lib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"], a["Nkv"],
+                      a["d"], a["causal"], a["scale"], a["stream"])
+    assert rc == code
+
+
+def test_decode_workspace_size_and_validation(lib):
+    n = lib.attn_decode_workspace_bytes(64, 32, 128, 16)
+    assert n >= 64 * 32 * 16 * (128 + 1) * 4
+    assert lib.attn_decode_workspace_bytes(1, 1, 96, 4) == 0
+    ws = ctypes.c_void_p(16 * 4096)
+    def call(**kw):
+        a = dict(B=2, H=2, Nkv=100, d=128, scale=0.1, S=4, ws_bytes=n)
+        a.update(kw)
+        return lib.attn_decode(P, P, P, P, P, a["B"], a["H"], a["Nkv"], a["d"], a["scale"], a["S"], ws,
+                               a["ws_bytes"], None)
+    assert call(S=0) == -1 and call(S=2000) == -1 and call(Nkv=0) == -1
+    assert call(d=80) == -2 and call(ws_bytes=16) == -1 and call(scale=0.0) == -1
+    assert call(B=0) == 0
+
+
+def test_product_path_never_imports_the_oracle():
+    """The package must not reach the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "tiled_attention_24_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.replace("oracle/", ""), f

@@ -1,0 +1,126 @@
+"""ctypes binding of libtiledattn (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and takes
+torch tensors (device memory) or raw integers.  All computation happens in the
+CUDA library; there is no Python or CPU fallback -- if the library cannot be
+loaded, or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtiledattn.so")
+
+ATTN_OK = 0
+STATUS_NAMES = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
+                -3: "ATTN_ERR_MISALIGNED", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_TIMEOUT"}
+
+# (name, restype, argtypes)
+_VP, _I, _F, _SZ, _ULL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_ulonglong
+SIGNATURES = [
+    ("attn_status_string", ctypes.c_char_p, [_I]),
+    ("attn_version", ctypes.c_char_p, []),
+    ("attn_fwd", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    ("attn_decode_workspace_bytes", _SZ, [_I, _I, _I, _I]),
+    ("attn_decode", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
+    ("attn_check_status", _I, [_VP]),
+    ("attn_set_wait_limit_ns", None, [_ULL]),
+    ("attn_watchdog_selftest", _I, [_ULL, _VP]),
+]
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the shared library (once) and declare every entry point."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with `python -m tiled_attention_24_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, res, args in SIGNATURES:
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn, rc):
+    if rc != ATTN_OK:
+        raise AttnError(fn, rc)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """bf16 forward: q [B,H,Nq,d], k/v [B,H,Nkv,d] -> o (bf16), lse (fp32)."""
+    _need_cuda(q, k, v, o, lse)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nkv, d, int(bool(causal)),
+                         float(scale), _stream(stream))
+    _check("attn_fwd", rc)
+
+
+def attn_decode_workspace_bytes(B: int, H: int, d: int, num_splits: int) -> int:
+    return int(load().attn_decode_workspace_bytes(B, H, d, num_splits))
+
+
+def attn_decode(q, k, v, o, lse, scale: float, num_splits: int, workspace, stream=None):
+    """Split-KV decode: q [B,H,1,d], k/v [B,H,Nkv,d] -> o [B,H,1,d], lse [B,H,1]."""
+    _need_cuda(q, k, v, o, lse, workspace)
+    B, H, _, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
+                            int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream))
+    _check("attn_decode", rc)
+
+
+def attn_check_status(stream=None) -> int:
+    return int(load().attn_check_status(_stream(stream)))
+
+
+def attn_set_wait_limit_ns(ns: int) -> None:
+    load().attn_set_wait_limit_ns(int(ns))
+
+
+def attn_watchdog_selftest(limit_ns: int, stream=None) -> None:
+    _check("attn_watchdog_selftest", load().attn_watchdog_selftest(int(limit_ns), _stream(stream)))
+
+
+def attn_version() -> str:
+    return load().attn_version().decode()
+
+
+def attn_status_string(code: int) -> str:
+    return load().attn_status_string(int(code)).decode()

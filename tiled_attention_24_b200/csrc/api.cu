@@ -1,0 +1,208 @@
+// C-ABI entry points of libtiledattn (declared in include/tiledattn.h):
+// argument validation, TMA descriptor construction, launches.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "tiledattn.h"
+#include "ptx.cuh"
+#include "fwd_bf16.cuh"
+#include "decode.cuh"
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitNs = 1000000000ull;
+unsigned long long g_wait_ns = kDefaultWaitNs;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [BH][N][d] bf16 viewed as a 3-D tensor (d, N, BH); boxes of 64 x 128 x 1
+// with 128-byte swizzle.  Rows past N read as zero and are not written.
+int make_tmap_bf16(CUtensorMap* m, const void* ptr, int d, int N, int BH) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename K>
+int set_smem_attr(K kernel, int bytes) {
+  // cheap, idempotent; done per call so that every device the caller uses is covered
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nkv,
+               int causal, float scale, cudaStream_t st) {
+  using C = ta::FwdCfg<D>;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  int rc;
+  if ((rc = make_tmap_bf16(&tq, q, D, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, D, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, D, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&to, o, D, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::fwd_bf16_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
+  ta::FwdParams p;
+  p.lse = lse;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.n_qp = (Nq + 255) / 256;
+  p.Tc = (Nkv + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_ns;
+  const long long grid = (long long)BH * p.n_qp;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  ta::fwd_bf16_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t decode_ws_bytes(long long BH, int d, int S) {
+  const size_t o_bytes = (size_t)BH * S * d * sizeof(float);
+  const size_t l_bytes = (size_t)BH * S * sizeof(float);
+  return ((o_bytes + 255) & ~size_t(255)) + l_bytes;
+}
+
+__global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ta::mbar_init(ta::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ta::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives: the bounded wait must give up and record a timeout
+    ta::wait_bar(ta::smem_u32(&bar), 0, &abort_flag, limit_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+const char* attn_version(void) { return "tiledattn 0.1 sm_100a"; }
+
+void attn_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
+
+int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+             int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;
+  if (!q || !o || !lse || (Nkv > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned4(lse) || (Nkv > 0 && (!aligned16(k) || !aligned16(v))))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Nkv == 0) {
+    const long long rows = (long long)B * H * Nq;
+    const long long n = rows * d;
+    const long long blocks = (n + 255) / 256;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    ta::fill_empty_kernel<<<(unsigned)blocks, 256, 0, st>>>(o, lse, rows, d);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  return d == 128 ? launch_fwd<128>(q, k, v, o, lse, B, H, Nq, Nkv, causal, scale, st)
+                  : launch_fwd<64>(q, k, v, o, lse, B, H, Nq, Nkv, causal, scale, st);
+}
+
+size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || num_splits <= 0 || (d != 64 && d != 128)) return 0;
+  return decode_ws_bytes((long long)B * H, d, num_splits);
+}
+
+int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+                int B, int H, int Nkv, int d, float scale, int num_splits, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || Nkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return ATTN_OK;
+  const long long BH = (long long)B * H;
+  if (BH * num_splits > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(lse) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(o) & 1u))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < decode_ws_bytes(BH, d, num_splits)) return ATTN_ERR_INVALID_ARG;
+  const int chunk = (int)((Nkv + (long long)num_splits - 1) / num_splits);
+  float* o_part = static_cast<float*>(workspace);
+  float* l_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           (((size_t)BH * num_splits * d * sizeof(float) + 255) & ~size_t(255)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sl2 = scale * 1.4426950408889634f;
+  const unsigned grid = (unsigned)(BH * num_splits);
+  if (d == 128) {
+    ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
+                                                                    chunk, sl2);
+    ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  } else {
+    ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
+                                                                   chunk, sl2);
+    ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_check_status(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, ta::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (h != 0 && cudaMemcpyToSymbol(ta::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return h;
+}
+
+int attn_watchdog_selftest(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

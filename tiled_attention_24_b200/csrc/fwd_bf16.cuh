@@ -1,0 +1,400 @@
+// bf16 tiled attention forward for sm_100a (TMA + tcgen05 + TMEM).
+//
+// What it computes ("Can a full-day context beat one minute? Flash attention
+// and the sequence-length question", sections "The Flash Attention algorithm"
+// and "Online softmax recurrence"): O = softmax(scale * Q K^T) V and the
+// natural-log LSE per query row, with Q split into B_r = 128-row blocks and
+// K/V into B_c = 128-key blocks; S_ij = Q_i K_j^T lives only in tensor memory,
+// the running row max m, running sum l and the unnormalised O accumulator are
+// updated block by block and O is divided by l once at the end ("FA2" item 1).
+//
+// CTA = one (batch, head) and TWO query tiles of 128 rows (256 rows).  Roles
+// (warp specialisation, "FlashAttention 4" section "What is new"):
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j into a smem ring
+//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+//   warps 2-5   softmax warpgroup of query tile 0 (thread = TMEM lane = row)
+//   warps 6-9   softmax warpgroup of query tile 1
+// The two softmax warpgroups ping-pong: while one turns S into P, the tensor
+// core runs the other tile's P V and next S ("FA3" item 2, interleaving matmul
+// and softmax).  Each softmax warpgroup also does its own (rare, lazy) O
+// correction and the epilogue (O / l -> bf16 -> smem -> TMA store, LSE).
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   S_t  : columns [128 t, 128 t + 128)   fp32 scores of tile t
+//   P_t  : columns [128 t, 128 t + 64)    bf16x2 probabilities, aliasing S_t
+//   O_t  : columns [256 + D t, 256 + D t + D)   fp32 accumulator of tile t
+//
+// Shared memory (128-byte swizzled, the TMA and UMMA canonical layout): each
+// 128 x D bf16 tile is stored as D/64 column blocks of 128 rows x 128 bytes.
+// Q0, Q1, then NSLOT ring slots holding K_0, V_0, K_1, V_1, ... in load order.
+#pragma once
+#include "ptx.cuh"
+
+namespace ta {
+
+struct FwdParams {
+  float* lse;
+  int Nq, Nkv, n_qp, Tc;
+  int causal;
+  float sl2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BR = 128, BC = 128;
+  static constexpr int TILE = 128 * D * 2;       // bytes of one 128 x D bf16 tile
+  static constexpr int HALF = 128 * 128;         // one 64-column block (128 rows x 128 B)
+  static constexpr int NSLOT = (D == 128) ? 5 : 10;
+  static constexpr int Q_OFF = 0;
+  static constexpr int SLOT_OFF = 2 * TILE;
+  static constexpr int BAR_OFF = SLOT_OFF + NSLOT * TILE;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);
+  static constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
+  static constexpr float TAU = 8.0f;  // lazy-rescale threshold, log2 units
+};
+
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t kv_full[10];
+  uint64_t kv_empty[10];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t epi[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(FwdBars) <= 256, "barrier block too large");
+
+__device__ __forceinline__ int fwd_tile_kv_count(int r0, int Nq, int Nkv, int Tc, int causal) {
+  if (r0 >= Nq) return 0;
+  if (!causal) return Tc;
+  const long long r_last = min(r0 + 127, Nq - 1);
+  const long long last_key = r_last + (long long)(Nkv - Nq);
+  if (last_key < 0) return 0;
+  return (int)min((long long)Tc, last_key / 128 + 1);
+}
+
+// Bounded wait that ignores the abort flag (used to drain work in flight).
+__device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  int dummy = 0;
+  return wait_bar(bar, parity, &dummy, limit_ns);
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::BAR_OFF);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: (batch*head, pair of query tiles); heaviest pairs first when causal
+  const int bh = blockIdx.x / p.n_qp;
+  const int qpi = blockIdx.x % p.n_qp;
+  const int qp = p.causal ? (p.n_qp - 1 - qpi) : qpi;
+  int r0[2], n[2];
+  bool present[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    r0[t] = qp * 256 + t * 128;
+    present[t] = r0[t] < p.Nq;
+    n[t] = fwd_tile_kv_count(r0[t], p.Nq, p.Nkv, p.Tc, p.causal);
+  }
+  const int nmax = max(n[0], n[1]);
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->p_full[t]), 128);
+      mbar_init(smem_u32(&bars->o_full[t]), 1);
+      mbar_init(smem_u32(&bars->epi[t]), 128);
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint32_t qbar = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qbar, (present[0] + present[1]) * C::TILE);
+      for (int t = 0; t < 2; ++t) {
+        if (!present[t]) continue;
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < nmax && ok; ++j) {
+        for (int w = 0; w < 2 && ok; ++w, ++it) {
+          const int slot = it % C::NSLOT;
+          const uint32_t ph = (it / C::NSLOT) & 1;
+          ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+          mbar_arrive_expect_tx(fb, C::TILE);
+          const uint32_t dst = sbase + C::SLOT_OFF + slot * C::TILE;
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(dst + h * C::HALF, w == 0 ? &tmK : &tmV, fb, h * 64, j * 128, bh);
+        }
+      }
+      // Never leave a copy in flight: wait for the last load of every slot.
+      if (!ok) {
+        wait_bar_drain(qbar, 0, p.timeout_ns);
+        for (int back = 1; back <= C::NSLOT && it - back >= 0; ++back) {
+          const int i2 = it - back;
+          wait_bar_drain(smem_u32(&bars->kv_full[i2 % C::NSLOT]), (i2 / C::NSLOT) & 1, p.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
+      tc_fence_after();
+      auto slot_of = [&](int it) { return it % C::NSLOT; };
+      auto par_of = [&](int it) { return (uint32_t)((it / C::NSLOT) & 1); };
+      auto issue_S = [&](int t, int j) {
+        const int s = slot_of(2 * j);
+        const uint32_t qa = sbase + C::Q_OFF + t * C::TILE;
+        const uint32_t ka = sbase + C::SLOT_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
+          mma_f16_ss(tbase + t * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), C::ID_S,
+                     kk > 0);
+        }
+        tc_commit(smem_u32(&bars->s_full[t]));
+      };
+      auto issue_PV = [&](int t, int j) {
+        const int s = slot_of(2 * j + 1);
+        const uint32_t va = sbase + C::SLOT_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          mma_f16_ts(tbase + 256 + t * D, tbase + t * 128 + kk * 8, smem_desc(va + kk * 2048, C::HALF, 1024),
+                     C::ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (ok && nmax > 0) {
+        ok = wait_bar(smem_u32(&bars->kv_full[slot_of(0)]), par_of(0), abort_flag, p.timeout_ns);
+        tc_fence_after();
+        if (ok) {
+          if (n[0] > 0) issue_S(0, 0);
+          if (n[1] > 0) issue_S(1, 0);
+          tc_commit(smem_u32(&bars->kv_empty[slot_of(0)]));
+        }
+      }
+      if (ok) {
+        for (int t = 0; t < 2; ++t)
+          if (present[t] && n[t] == 0) tc_commit(smem_u32(&bars->o_full[t]));
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        ok = wait_bar(smem_u32(&bars->kv_full[slot_of(2 * j + 1)]), par_of(2 * j + 1), abort_flag, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        if (j < n[0]) {
+          ok = wait_bar(smem_u32(&bars->p_full[0]), j & 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_PV(0, j);
+          if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
+        }
+        const bool nextK = j + 1 < nmax;
+        if (nextK) {
+          ok = wait_bar(smem_u32(&bars->kv_full[slot_of(2 * j + 2)]), par_of(2 * j + 2), abort_flag, p.timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (j + 1 < n[0]) issue_S(0, j + 1);
+        if (j < n[1]) {
+          ok = wait_bar(smem_u32(&bars->p_full[1]), j & 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_PV(1, j);
+          if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
+        }
+        tc_commit(smem_u32(&bars->kv_empty[slot_of(2 * j + 1)]));
+        if (j + 1 < n[1]) issue_S(1, j + 1);
+        if (nextK) tc_commit(smem_u32(&bars->kv_empty[slot_of(2 * j + 2)]));
+      }
+      if (!ok) {
+        // drain: every MMA issued so far must finish before TMEM is freed
+        tc_commit(smem_u32(&bars->drain));
+        wait_bar_drain(smem_u32(&bars->drain), 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int rr = quarter * 32 + lane;  // row within the tile == TMEM lane
+    const int row = r0[t] + rr;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tbase + lane_off + t * 128;
+    const uint32_t tO = tbase + lane_off + 256 + t * D;
+    const float sl2 = p.sl2;
+    const int off = p.Nkv - p.Nq;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = present[t];
+    for (int j = 0; j < n[t] && ok; ++j) {
+      ok = wait_bar(smem_u32(&bars->s_full[t]), j & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      const int kb = j * 128;
+      const bool tail = kb + 128 > p.Nkv;
+      const bool diag = p.causal && (kb + 127 > r0[t] + off);
+      if (tail || diag) {
+        int lim = p.Nkv - 1 - kb;                       // last visible column of this row
+        if (p.causal) lim = min(lim, row + off - kb);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim) s[c][i] = 0xFF800000u;  // -inf
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[0][i]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[1][i]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[2][i]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[3][i]));
+      }
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      // lazy rescale: move the reference max only when it rises by more than TAU
+      const bool need = m_blk > m_ref + C::TAU;
+      float factor = 1.f;
+      if (need) {
+        factor = ex2(m_ref - m_blk);  // 0 when m_ref == -inf
+        l *= factor;
+        m_ref = m_blk;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+          tmem_st32(tO + cc * 32, o);
+        }
+      }
+      const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float ls0 = 0.f, ls1 = 0.f;
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c][2 * i]), sl2, negm));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c][2 * i + 1]), sl2, negm));
+          ls0 += p0;
+          ls1 += p1;
+          pk[c >> 1][(c & 1) * 16 + i] = pack_bf16(p0, p1);
+        }
+      }
+      l += ls0 + ls1;
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->p_full[t]));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (present[t] && ok) {
+      ok = wait_bar(smem_u32(&bars->o_full[t]), 0, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (present[t] && ok) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      uint8_t* stage = smem + C::Q_OFF + t * C::TILE;  // Q_t is no longer read
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = (l > 0.f) ? __uint_as_float(o[g * 8 + 2 * e]) * inv : 0.f;
+            const float b = (l > 0.f) ? __uint_as_float(o[g * 8 + 2 * e + 1]) * inv : 0.f;
+            w[e] = pack_bf16(a, b);
+          }
+          const int c16 = cc * 4 + g;  // 16-byte chunk within the row
+          const int h = c16 >> 3, ch = c16 & 7;
+          uint8_t* dst = stage + h * C::HALF + rr * 128 + ((ch ^ (rr & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      if (row < p.Nq)
+        p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&bars->epi[t]));
+      if (warp == 2 + 4 * t && lane == 0) {
+        if (wait_bar(smem_u32(&bars->epi[t]), 0, abort_flag, p.timeout_ns)) {
+          for (int h = 0; h < D / 64; ++h)
+            tma_store_3d(&tmO, sbase + C::Q_OFF + t * C::TILE + h * C::HALF, h * 64, r0[t], bh);
+          bulk_commit();
+          bulk_wait_all();
+        }
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// Empty key set: every query row sees nothing -> O = 0, LSE = -inf.
+__global__ void fill_empty_kernel(uint16_t* o, float* lse, long long n_rows, int d) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i < n_rows * d) o[i] = 0;
+  if (i < n_rows) lse[i] = -INFINITY;
+}
+
+}  // namespace ta
