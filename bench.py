@@ -1,0 +1,387 @@
+"""Benchmark of the tiled attention forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the hot path over the seeded synthetic workloads:
+  * prefill  B=4 H=16 N=4096 d=128 bf16: attn_fwd non-causal + attn_fwd causal
+             (the headline: attention forward TFLOP/s, 4*B*H*N*N*d, halved
+             for causal);
+  * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine
+             (KV-read GB/s against HBM).
+Inputs are resident in HBM before timing starts and are larger than the
+126 MB L2 (prefill Q+K+V = 201 MB, decode K+V = 8.6 GB), so no L2 flush is
+needed between steps.  Every launch is bracketed by CUDA events on the
+launching stream; `value` is prefill FLOPs / summed prefill kernel time.
+
+`e2e` measures the same metric through the public API with host buffers:
+each step copies Q, K, V from pinned host memory, runs both forwards and
+copies O and LSE back.
+
+Multi-GPU (torchrun): the workload is replicated per rank (independent
+problems, no collective on the data path, weak scaling); times are the max
+over ranks.  `--impl reference` times the fp64 CPU oracle on a bounded sample
+of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_qkv  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample(seconds_cap: float = 30.0):
+    """fp64 oracle on a bounded sample of the prefill workload: rows of the first
+    heads, non-causal then causal, until ~seconds_cap of work.  Returns
+    (TFLOP/s, description, threads)."""
+    from oracle import attention as A  # test infrastructure: CPU baseline only
+    w = WORKLOADS["prefill"]
+    q, k, v = make_qkv(w, seed=0, B=1, H=2)
+    flops = 0.0
+    t0 = time.perf_counter()
+    done = []
+    for h in range(2):
+        for causal in (False, True):
+            A.attention(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], causal, w.scale)
+            flops += w.flops(causal) / (w.B * w.H)
+            done.append(f"h{h}{'c' if causal else 'n'}")
+            if time.perf_counter() - t0 > seconds_cap:
+                break
+    dt = time.perf_counter() - t0
+    desc = (f"fp64 numpy oracle, prefill shape (N=4096, d=128), {len(done)} (head, mode) "
+            f"passes of the full 4096x4096 score matrix: {','.join(done)}")
+    return flops / dt / 1e12, desc, cpu_threads(), dt
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    vals = []
+    desc, thr = "", 1
+    for _ in range(args.warmup_ref):
+        oracle_sample(5.0)
+    t_all = time.perf_counter()
+    for _ in range(args.steps_ref):
+        v, desc, thr, _ = oracle_sample(20.0)
+        vals.append(v)
+    wall = time.perf_counter() - t_all
+    val = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": "attn fwd TFLOP/s (prefill B4 H16 N4096 d128, non-causal + causal)",
+        "value": val, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps_ref, "warmup": args.warmup_ref,
+        "ms_per_step": wall / max(1, args.steps_ref) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": "prefill", "B": 4, "H": 16, "Nq": 4096, "Nkv": 4096, "d": 128,
+                   "causal": ["false", "true"], "sample": "bounded oracle sample"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import tiled_attention_24_b200 as ta
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ta.load()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- inputs, resident in HBM
+    wp = WORKLOADS["prefill"]
+    q, k, v = (t.to(dev) for t in make_qkv(wp, seed=0))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    wd = WORKLOADS["decode"]
+    parts = set(args.only.split(","))
+    dq, dk, dv = make_qkv(wd, seed=0, device=dev, B=args.decode_batch or wd.B)
+    do = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
+    dws = torch.empty(ta.attn_decode_workspace_bytes(dq.shape[0], wd.H, wd.d, wd.num_splits),
+                      dtype=torch.uint8, device=dev)
+
+    flops_nc, flops_c = wp.flops(False), wp.flops(True)
+    kv_bytes = 2 * dk.numel() * dk.element_size()
+
+    def step(ev):
+        ev[0].record(stream)
+        if "prefill" in parts:
+            ta.attn_fwd(q, k, v, o, lse, False, wp.scale, stream)
+        ev[1].record(stream)
+        if "prefill" in parts:
+            ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream)
+        ev[2].record(stream)
+        if "decode" in parts:
+            ta.attn_decode(dq, dk, dv, do, dlse, wd.scale, wd.num_splits, dws, stream)
+        ev[3].record(stream)
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        step(evs[0])
+    torch.cuda.synchronize()
+    if ta.attn_check_status() != 0:
+        raise RuntimeError("device watchdog fired during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    status = ta.attn_check_status()
+    if status != 0:
+        raise RuntimeError(f"device watchdog status {status}")
+
+    total_ms = t_start.elapsed_time(t_end)
+    nc_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    c_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    sums = torch.tensor([total_ms, sum(nc_ms), sum(c_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(sums, op=dist.ReduceOp.MAX)
+    total_ms, nc_tot, c_tot, dec_tot = sums.tolist()
+
+    prefill_ms = nc_tot + c_tot
+    value = ws * args.steps * (flops_nc + flops_c) / (prefill_ms * 1e-3) / 1e12
+    nc_avg = nc_tot / args.steps
+    c_avg = c_tot / args.steps
+    dec_avg = dec_tot / args.steps
+    tflops_nc = flops_nc / (nc_avg * 1e-3) / 1e12
+    tflops_c = flops_c / (c_avg * 1e-3) / 1e12
+    dec_gbs = kv_bytes / (dec_avg * 1e-3) / 1e9
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        hl2 = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        ho2 = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            ta.attn_fwd(q, k, v, o, lse, False, wp.scale, stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream)
+            ho2.copy_(o, non_blocking=True)
+            hl2.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = e_ms.item()
+        h2d = 3 * q.numel() * q.element_size()
+        d2h = 2 * (o.numel() * o.element_size() + lse.numel() * lse.element_size())
+        e2e = {"value": ws * args.e2e_steps * (flops_nc + flops_c) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cv, desc, thr, _ = oracle_sample(args.cpu_seconds)
+        cpu = {"value": cv, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc}
+
+    gpu_launches = args.steps * (2 * ("prefill" in parts) + 2 * ("decode" in parts))
+    traffic = load_traffic()
+    line = {
+        "metric": "attn fwd TFLOP/s (prefill B4 H16 N4096 d128, non-causal + causal)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, resident in HBM)",
+        "config": {"workload": "prefill", "B": wp.B, "H": wp.H, "Nq": wp.Nq, "Nkv": wp.Nkv, "d": wp.d,
+                   "causal": ["false", "true"], "parallelism": f"replicas x{ws}",
+                   "l2": "inputs (201 MB) larger than L2 (126 MB); no flush"},
+        "prefill": {"noncausal_tflops": tflops_nc, "causal_tflops": tflops_c,
+                    "noncausal_ms": nc_avg, "causal_ms": c_avg,
+                    "frac_of_peak_noncausal": tflops_nc / peak_tc, "frac_of_peak_causal": tflops_c / peak_tc},
+        "decode": None if "decode" not in parts else {
+                   "workload": f"decode B{dq.shape[0]} H32 Nkv8192 d128 splits16", "ms": dec_avg, "kv_gbs": dec_gbs,
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peak_hbm, "unit": "GB/s",
+                                "frac": dec_gbs / peak_hbm, "traffic": traffic.get("decode_split"),
+                                "peak_source": peak_src}},
+        "roofline": {"bound": "tensor", "achieved": tflops_nc, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": tflops_nc / peak_tc, "traffic": traffic.get("fwd_bf16"),
+                     "kernel": "fwd_bf16_kernel<128> non-causal prefill",
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summaries (null if absent
+    or stale)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="prefill,decode",
+                    help="comma list of step parts to run (prefill, decode); profiling aid")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="decode batch override (profiling aid; 0 = the workload's 64)")
+    args = ap.parse_args()
+    args.steps_ref = max(1, min(args.steps, 3))
+    args.warmup_ref = 0
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
