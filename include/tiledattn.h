@@ -58,7 +58,9 @@ enum {
   ATTN_ERR_UNSUPPORTED = -2, /* head dim or shape outside what is built     */
   ATTN_ERR_MISALIGNED = -3,  /* pointer not 16-byte aligned                 */
   ATTN_ERR_CUDA = -4,        /* CUDA runtime/driver error at launch         */
-  ATTN_ERR_TIMEOUT = -5      /* a kernel wait ran past its time limit       */
+  ATTN_ERR_TIMEOUT = -5,     /* a kernel wait ran past its time limit       */
+  ATTN_ERR_TOO_LARGE = -6    /* request needs more than the library's fixed
+                                scratch (attn_decode_noalloc)               */
 };
 
 /* Human-readable name of a status code (static string). */
@@ -108,6 +110,38 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits)
 ATTN_API int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
                 float* lse, int B, int H, int Nkv, int d, float scale, int num_splits,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_decode_noalloc -- the same split-KV decode as attn_decode, for callers
+ * that cannot allocate device memory: code that runs where cudaMalloc is not
+ * allowed or not wanted (inside a caller's own memory pool or allocator hook,
+ * a plug-in with no allocator of its own, a latency-critical path that must
+ * never enter the driver's allocator).  The pages have no counterpart: this
+ * is a packaging variant, not part of the method.
+ *
+ * The per-split partial results live in one fixed device array inside the
+ * library, ATTN_DECODE_NOALLOC_SCRATCH_BYTES (20 MiB) in size.  Every GPU that
+ * loads the library holds that array until the process exits.  A request
+ * whose partials need more than that -- B*H*num_splits*(d+1)*4 bytes plus
+ * alignment, as attn_decode_workspace_bytes() reports -- is rejected with
+ * ATTN_ERR_TOO_LARGE before anything is launched (the decode workload
+ * B=64, H=32, d=128, 16 splits needs 16.1 MiB and fits).
+ *
+ * The function calls no allocator (no cudaMalloc/cudaFree, no library
+ * routine that allocates).  The first call on a device looks up the device
+ * address of the array with cudaGetSymbolAddress while that device is
+ * current; make that first call before any stream capture.  All calls share
+ * the array and it keeps the last call's contents; every partial is written
+ * before it is read, so nothing needs clearing between calls.  Calls that
+ * overlap on the GPU (different streams, or different host threads) race on
+ * the array and must be serialised by the caller.
+ *
+ * Arguments, layouts and errors otherwise as attn_decode.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (20u * 1024u * 1024u)
+ATTN_API int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v,
+                                 attn_bf16_t* o, float* lse, int B, int H, int Nkv, int d, float scale,
+                                 int num_splits, void* stream);
 
 /*
  * attn_check_status -- synchronise `stream`, read the device status word

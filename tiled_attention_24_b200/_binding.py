@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libtiledattn.so")
 
 ATTN_OK = 0
 STATUS_NAMES = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
-                -3: "ATTN_ERR_MISALIGNED", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_TIMEOUT"}
+                -3: "ATTN_ERR_MISALIGNED", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_TIMEOUT",
+                -6: "ATTN_ERR_TOO_LARGE"}
 
 # (name, restype, argtypes)
 _VP, _I, _F, _SZ, _ULL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_ulonglong
@@ -27,6 +28,7 @@ SIGNATURES = [
     ("attn_fwd", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_decode_workspace_bytes", _SZ, [_I, _I, _I, _I]),
     ("attn_decode", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
+    ("attn_decode_noalloc", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP]),
     ("attn_check_status", _I, [_VP]),
     ("attn_set_wait_limit_ns", None, [_ULL]),
     ("attn_watchdog_selftest", _I, [_ULL, _VP]),
@@ -104,6 +106,17 @@ def attn_decode(q, k, v, o, lse, scale: float, num_splits: int, workspace, strea
                             int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream))
     _check("attn_decode", rc)
+
+
+def attn_decode_noalloc(q, k, v, o, lse, scale: float, num_splits: int, stream=None):
+    """attn_decode with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate device memory)."""
+    _need_cuda(q, k, v, o, lse)
+    B, H, _, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
+                                    int(num_splits), _stream(stream))
+    _check("attn_decode_noalloc", rc)
 
 
 def attn_check_status(stream=None) -> int:

@@ -91,6 +91,29 @@ size_t decode_ws_bytes(long long BH, int d, int S) {
   return ((o_bytes + 255) & ~size_t(255)) + l_bytes;
 }
 
+// Fixed scratch for attn_decode_noalloc: split partials (O then LSE), shared
+// by every call of that entry point on a device.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array per device, looked up once per device
+// with cudaGetSymbolAddress (in host code the array's name is only a stand-in).
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
 __global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -119,6 +142,7 @@ const char* attn_status_string(int s) {
     case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_TOO_LARGE: return "ATTN_ERR_TOO_LARGE";
     default: return "ATTN_ERR_UNKNOWN";
   }
 }
@@ -173,6 +197,41 @@ int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v
   const int chunk = (int)((Nkv + (long long)num_splits - 1) / num_splits);
   float* o_part = static_cast<float*>(workspace);
   float* l_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           (((size_t)BH * num_splits * d * sizeof(float) + 255) & ~size_t(255)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sl2 = scale * 1.4426950408889634f;
+  const unsigned grid = (unsigned)(BH * num_splits);
+  if (d == 128) {
+    ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
+                                                                    chunk, sl2);
+    ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  } else {
+    ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
+                                                                   chunk, sl2);
+    ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                        float* lse, int B, int H, int Nkv, int d, float scale, int num_splits, void* stream) {
+  if (B < 0 || H < 0 || Nkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return ATTN_OK;
+  const long long BH = (long long)B * H;
+  if (BH * num_splits > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (decode_ws_bytes(BH, d, num_splits) > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_TOO_LARGE;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(lse) || (reinterpret_cast<uintptr_t>(o) & 1u))
+    return ATTN_ERR_MISALIGNED;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != ATTN_OK) return rc;
+  const int chunk = (int)((Nkv + (long long)num_splits - 1) / num_splits);
+  float* o_part = static_cast<float*>(scratch);
+  float* l_part = reinterpret_cast<float*>(static_cast<char*>(scratch) +
                                            (((size_t)BH * num_splits * d * sizeof(float) + 255) & ~size_t(255)));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float sl2 = scale * 1.4426950408889634f;
