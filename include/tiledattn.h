@@ -144,6 +144,45 @@ ATTN_API int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, con
                                  int num_splits, void* stream);
 
 /*
+ * attn_quantize_int8 -- symmetric INT8 quantisation of a bf16 tensor
+ * [B][H][N][d] ([INT-FA]: token-level post-training quantisation of Q, K, V).
+ *   per_head == 0: one scale per token row, xs [B][H][N]   (Q and K);
+ *   per_head != 0: one scale per (batch, head), xs [B][H] (V: P V contracts
+ *                  over tokens, so V's scale must be shared by a head's tokens).
+ * s = amax / 127 (IEEE fp32 divide; amax == 0 gives s = 1),
+ * xq = clamp(rne(x / s), -127, 127) (IEEE divide, round to nearest even).
+ *   x bf16 16-byte aligned, xq int8 [B][H][N][d] 16-byte aligned, xs fp32.
+ *   d in {64, 128}.
+ */
+ATTN_API int attn_quantize_int8(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H, int N, int d,
+                                int per_head, void* stream);
+
+/*
+ * attn_fwd_int8 -- INT8 attention forward ([INT-FA]: INT8 GEMMs for Q K^T and
+ * P V inside the FlashAttention forward, int32 accumulation):
+ *   S = q_i8 . k_i8 (int32, exact); x = S * q_scale[i] * k_scale[j] * scale;
+ *   running row max moved on every increase; P8 = rne(127 * exp(x - m)) in
+ *   [0, 127]; O accumulates P8 . v_i8 in int32 per block and in fp32 across
+ *   max changes, times v_scale / 127; l sums P8 / 127; O = acc / l,
+ *   LSE = m + ln l.
+ *   q [B][H][Nq][128] int8 + q_scale [B][H][Nq]; k [B][H][Nkv][128] int8 +
+ *   k_scale [B][H][Nkv]; v [B][H][Nkv][128] int8 + v_scale [B][H];
+ *   o [B][H][Nq][128] fp32 out, lse [B][H][Nq] fp32 out.
+ *   d must be 128; Nkv >= 1.
+ */
+ATTN_API int attn_fwd_int8(const int8_t* q, const float* q_scale, const int8_t* k, const float* k_scale,
+                           const int8_t* v, const float* v_scale, float* o, float* lse, int B, int H, int Nq,
+                           int Nkv, int d, int causal, float scale, void* stream);
+
+/*
+ * attn_int8_scores -- the int32 score tiles S = q_i8 k_i8^T of the INT8
+ * forward, computed by the same tensor-core MMA path and written to
+ * s [B][H][Nq][Nkv] int32 (a check of the integer GEMM; small sizes).
+ */
+ATTN_API int attn_int8_scores(const int8_t* q, const int8_t* k, int32_t* s, int B, int H, int Nq, int Nkv, int d,
+                              void* stream);
+
+/*
  * attn_check_status -- synchronise `stream`, read the device status word
  * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT), clear it and
  * return it; also returns ATTN_ERR_CUDA if the synchronisation itself fails.

@@ -95,31 +95,35 @@ def _near_half(y, band):
 
 
 def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
-                   with_flip_bound=False):
+                   with_flip_bound=False, rows=None):
     """Emulated INT8 forward (steps 2-5 of the module docstring).
 
     qi, ki, vi: int8 [B,H,N,d]; qs, ks: fp32 [B,H,N]; vs: fp32 [B,H].
-    Returns (O, LSE) float64 and, with ``with_flip_bound``, (flip_bound [B,H,Nq,d],
+    ``rows`` restricts the computation to those query rows (rows are
+    independent).  Returns (O, LSE) float64 and, with ``with_flip_bound``,
+    (flip_bound [B,H,Nq,d],
     lse_flip_bound [B,H,Nq], flips): how far O and LSE can move when an element
     of 127 * 2^(x - m) that lies within the fp32 evaluation error of a rounding
     midpoint rounds the other way on a device that computes x and 2^x in fp32.
     """
     qi, ki, vi = np.asarray(qi), np.asarray(ki), np.asarray(vi)
     qs, ks, vs = _f64(qs), _f64(ks), _f64(vs)
-    B, H, Nq, d = qi.shape
+    B, H, Nq_all, d = qi.shape
     Nkv = ki.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    ridx = np.arange(Nq_all) if rows is None else np.asarray(rows, dtype=np.int64)
+    Nq = ridx.size
     O = np.zeros((B, H, Nq, d))
     LSE = np.full((B, H, Nq), -np.inf)
     FB = np.zeros((B, H, Nq, d))
     LB = np.zeros((B, H, Nq))
     flips = 0
-    vis = visible_mask(Nq, Nkv, causal)
+    vis = visible_mask(Nq_all, Nkv, causal, ridx)
     for b in range(B):
         for h in range(H):
-            S = qi[b, h].astype(np.int64) @ ki[b, h].astype(np.int64).T
-            x = S * (qs[b, h][:, None] * ks[b, h][None, :]) * (scale * LOG2E)
+            S = qi[b, h, ridx].astype(np.int64) @ ki[b, h].astype(np.int64).T
+            x = S * (qs[b, h, ridx][:, None] * ks[b, h][None, :]) * (scale * LOG2E)
             x = np.where(vis, x, -np.inf)
             acc = np.zeros((Nq, d))
             l = np.zeros(Nq)
@@ -131,7 +135,8 @@ def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
                 xb = x[:, cols]
                 m_new = np.maximum(m, xb.max(axis=1))
                 grow = np.isfinite(m) & (m_new > m)
-                f = np.where(grow, np.exp2(np.where(grow, m - m_new, 0.0)), 1.0)
+                f = np.ones_like(m)
+                np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
                 m = m_new
@@ -306,7 +311,8 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
                 xb = x[:, cols]
                 m_new = np.maximum(m, xb.max(axis=1))
                 grow = np.isfinite(m) & (m_new > m)
-                f = np.where(grow, np.exp2(np.where(grow, m - m_new, 0.0)), 1.0)
+                f = np.ones_like(m)
+                np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
                 m = m_new

@@ -11,12 +11,14 @@ import math
 import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
-                       attn_decode_workspace_bytes, attn_fwd, attn_set_wait_limit_ns,
-                       attn_status_string, attn_version, attn_watchdog_selftest, load)
+                       attn_decode_noalloc, attn_decode_workspace_bytes, attn_fwd, attn_fwd_int8,
+                       attn_int8_scores, attn_quantize_int8, attn_set_wait_limit_ns, attn_status_string,
+                       attn_version, attn_watchdog_selftest, load)
 
 __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "attn_check_status",
            "attn_set_wait_limit_ns", "attn_watchdog_selftest", "attn_version", "attn_status_string",
-           "AttnError", "forward", "decode"]
+           "AttnError", "forward", "decode", "quantize_int8", "forward_int8",
+           "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc"]
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
@@ -41,4 +43,27 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | Non
     o = torch.empty_like(q)
     lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
     attn_decode(q, k, v, o, lse, scale, num_splits, workspace, stream)
+    return o, lse
+
+
+def quantize_int8(x: torch.Tensor, per_head: bool = False, stream=None):
+    """INT8 symmetric quantisation (per token row, or per (batch, head))."""
+    B, H, N, d = x.shape
+    xq = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    xs = torch.empty((B, H) if per_head else (B, H, N), dtype=torch.float32, device=x.device)
+    attn_quantize_int8(x, xq, xs, per_head, stream)
+    return xq, xs
+
+
+def forward_int8(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Quantise bf16 q, k (per token) and v (per head) and run the INT8 forward.
+    Returns (o fp32, lse fp32)."""
+    B, H, Nq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    qi, qs = quantize_int8(q, False, stream)
+    ki, ks = quantize_int8(k, False, stream)
+    vi, vs = quantize_int8(v, True, stream)
+    o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    attn_fwd_int8(qi, qs, ki, ks, vi, vs, o, lse, causal, scale, stream)
     return o, lse

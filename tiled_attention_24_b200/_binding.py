@@ -13,7 +13,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libtiledattn.so")
+# TILEDATTN_LIB selects another build of the same library (tuning sweeps)
+LIB_PATH = os.environ.get("TILEDATTN_LIB") or os.path.join(_PKG, "libtiledattn.so")
 
 ATTN_OK = 0
 STATUS_NAMES = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
@@ -29,6 +30,9 @@ SIGNATURES = [
     ("attn_decode_workspace_bytes", _SZ, [_I, _I, _I, _I]),
     ("attn_decode", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_decode_noalloc", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP]),
+    ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    ("attn_fwd_int8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    ("attn_int8_scores", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_check_status", _I, [_VP]),
     ("attn_set_wait_limit_ns", None, [_ULL]),
     ("attn_watchdog_selftest", _I, [_ULL, _VP]),
@@ -117,6 +121,32 @@ def attn_decode_noalloc(q, k, v, o, lse, scale: float, num_splits: int, stream=N
     rc = load().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
                                     int(num_splits), _stream(stream))
     _check("attn_decode_noalloc", rc)
+
+
+def attn_quantize_int8(x, xq, xs, per_head: bool, stream=None):
+    """bf16 [B,H,N,d] -> int8 xq, fp32 xs ([B,H,N] per token or [B,H] per head)."""
+    _need_cuda(x, xq, xs)
+    B, H, N, d = x.shape
+    _check("attn_quantize_int8", load().attn_quantize_int8(_ptr(x), _ptr(xq), _ptr(xs), B, H, N, d,
+                                                             int(bool(per_head)), _stream(stream)))
+
+
+def attn_fwd_int8(q, qs, k, ks, v, vs, o, lse, causal: bool, scale: float, stream=None):
+    """INT8 forward: int8 q/k/v [B,H,N,128] with scales -> o fp32, lse fp32."""
+    _need_cuda(q, qs, k, ks, v, vs, o, lse)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_fwd_int8(_ptr(q), _ptr(qs), _ptr(k), _ptr(ks), _ptr(v), _ptr(vs), _ptr(o), _ptr(lse),
+                              B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _stream(stream))
+    _check("attn_fwd_int8", rc)
+
+
+def attn_int8_scores(q, k, s, stream=None):
+    """int32 S = q k^T of int8 [B,H,N,128] operands, through the INT8 MMA path."""
+    _need_cuda(q, k, s)
+    B, H, Nq, d = q.shape
+    _check("attn_int8_scores", load().attn_int8_scores(_ptr(q), _ptr(k), _ptr(s), B, H, Nq, k.shape[2], d,
+                                                         _stream(stream)))
 
 
 def attn_check_status(stream=None) -> int:

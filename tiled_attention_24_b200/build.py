@@ -43,12 +43,16 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and up_to_date():
+def build(verbose: bool = False, force: bool = False, out: str | None = None, defines=()) -> str:
+    """Compile libtiledattn.so (or `out`, with extra -D `defines`, for tuning
+    sweeps of compile-time kernel parameters)."""
+    lib = out or LIB
+    if not force and out is None and not defines and up_to_date():
         return LIB
     cmd = [nvcc_path(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
+           "-I", INCLUDE, "-I", CSRC, "-o", lib + ".tmp"]
+    cmd += ["-D" + d for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
@@ -57,10 +61,15 @@ def build(verbose: bool = False, force: bool = False) -> str:
         sys.stderr.write(res.stdout + res.stderr)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed (%d)" % res.returncode)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(verbose="--verbose" in sys.argv, force=True)
-    print(LIB)
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--out", default=None)
+    ap.add_argument("-D", dest="defines", action="append", default=[])
+    a = ap.parse_args()
+    print(build(verbose=a.verbose, force=True, out=a.out, defines=a.defines))

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include <cuda.h>
@@ -13,6 +14,8 @@
 #include "ptx.cuh"
 #include "fwd_bf16.cuh"
 #include "decode.cuh"
+#include "quant.cuh"
+#include "fwd_int8.cuh"
 
 namespace {
 
@@ -48,6 +51,56 @@ int make_tmap_bf16(CUtensorMap* m, const void* ptr, int d, int N, int BH) {
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// [BH][N][128] int8 viewed as (128, N, BH); boxes of 128 x 128 x 1 bytes with
+// 128-byte swizzle.
+int make_tmap_i8(CUtensorMap* m, const void* ptr, int N, int BH) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool SCORES_ONLY>
+int launch_int8(const void* q, const float* qs, const void* k, const float* ks, const void* v, const float* vs,
+                float* o, float* lse, int* s_out, int B, int H, int Nq, int Nkv, int causal, float scale,
+                cudaStream_t st) {
+  using C = ta::FwdI8Cfg;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_i8(&tq, q, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_i8(&tk, k, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_i8(&tv, SCORES_ONLY ? k : v, Nkv, BH)) != ATTN_OK) return rc;
+  if (cudaFuncSetAttribute(ta::fwd_int8_kernel<SCORES_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  ta::FwdI8Params p;
+  p.q_scale = qs;
+  p.k_scale = ks;
+  p.v_scale = vs;
+  p.o = o;
+  p.lse = lse;
+  p.s_out = s_out;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.n_qt = (Nq + 127) / 128;
+  p.Tc = (Nkv + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.ks_vec = (ks != nullptr) && (Nkv % 4 == 0) && aligned16(ks);
+  p.sl2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_ns;
+  const long long grid = (long long)BH * p.n_qt;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  ta::fwd_int8_kernel<SCORES_ONLY><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <typename K>
@@ -246,6 +299,64 @@ int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_b
     ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_quantize_int8(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H, int N, int d, int per_head,
+                       void* stream) {
+  if (B < 0 || H < 0 || N < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!x || !xq || !xs) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned4(xs)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long BH = (long long)B * H;
+  if (!per_head) {
+    const long long rows = BH * N;
+    const long long blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (d == 128)
+      ta::quant_int8_rows_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
+    else
+      ta::quant_int8_rows_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
+  } else {
+    if (BH > 65535) return ATTN_ERR_UNSUPPORTED;
+    const long long per_head_n = (long long)N * d;  // multiple of 8 (d is)
+    unsigned* amax = reinterpret_cast<unsigned*>(xs);
+    if (cudaMemsetAsync(amax, 0, BH * sizeof(float), st) != cudaSuccess) return ATTN_ERR_CUDA;
+    const unsigned gx = (unsigned)std::min<long long>(64, (per_head_n + 2047) / 2048);
+    ta::head_amax_kernel<<<dim3(gx, (unsigned)BH), 256, 0, st>>>(x, amax, per_head_n);
+    ta::quant_int8_heads_kernel<<<dim3(gx, (unsigned)BH), 256, 0, st>>>(x, xq, amax, per_head_n);
+    ta::head_scale_kernel<<<(unsigned)((BH + 255) / 256), 256, 0, st>>>(amax, (int)BH);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_fwd_int8(const int8_t* q, const float* q_scale, const int8_t* k, const float* k_scale, const int8_t* v,
+                  const float* v_scale, float* o, float* lse, int B, int H, int Nq, int Nkv, int d, int causal,
+                  float scale, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;
+  if (Nkv == 0) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !q_scale || !k || !k_scale || !v || !v_scale || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(q_scale) ||
+      !aligned4(k_scale) || !aligned4(v_scale) || !aligned4(lse))
+    return ATTN_ERR_MISALIGNED;
+  return launch_int8<false>(q, q_scale, k, k_scale, v, v_scale, o, lse, nullptr, B, H, Nq, Nkv, causal, scale,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_int8_scores(const int8_t* q, const int8_t* k, int32_t* s, int B, int H, int Nq, int Nkv, int d,
+                     void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0 || Nkv == 0) return ATTN_OK;
+  if (!q || !k || !s) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(s)) return ATTN_ERR_MISALIGNED;
+  return launch_int8<true>(q, nullptr, k, nullptr, nullptr, nullptr, nullptr, nullptr, s, B, H, Nq, Nkv, 0, 1.f,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_check_status(void* stream) {

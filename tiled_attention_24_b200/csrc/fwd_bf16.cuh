@@ -12,8 +12,10 @@
 // (warp specialisation, "FlashAttention 4" section "What is new"):
 //   warp 0      TMA producer: Q tiles once, then K_j, V_j into a smem ring
 //   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
-//   warps 2-5   softmax warpgroup of query tile 0 (thread = TMEM lane = row)
-//   warps 6-9   softmax warpgroup of query tile 1
+//   warps 2-3   idle (they complete warpgroup 0, whose registers are handed
+//               to the softmax warpgroups with setmaxnreg)
+//   warps 4-7   softmax warpgroup of query tile 0 (thread = TMEM lane = row)
+//   warps 8-11  softmax warpgroup of query tile 1
 // The two softmax warpgroups ping-pong: while one turns S into P, the tensor
 // core runs the other tile's P V and next S ("FA3" item 2, interleaving matmul
 // and softmax).  Each softmax warpgroup also does its own (rare, lazy) O
@@ -29,6 +31,13 @@
 // Q0, Q1, then NSLOT ring slots holding K_0, V_0, K_1, V_1, ... in load order.
 #pragma once
 #include "ptx.cuh"
+
+#ifndef TA_POLY_PERIOD
+#define TA_POLY_PERIOD 4
+#endif
+#ifndef TA_POLY_PAIRS
+#define TA_POLY_PAIRS 0
+#endif
 
 namespace ta {
 
@@ -51,10 +60,15 @@ struct FwdCfg {
   static constexpr int BAR_OFF = SLOT_OFF + NSLOT * TILE;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
+  // register split (launch: 384 threads x 168): warpgroup 0 drops to 56,
+  // the two softmax warpgroups rise to 224: 128*56 + 256*224 = 64512 = 384*168
+  static constexpr int REG_LOW = 56, REG_HIGH = 224;
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);
   static constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
   static constexpr float TAU = 8.0f;  // lazy-rescale threshold, log2 units
+  // of every POLY_PERIOD element pairs, POLY_PAIRS take 2^x from the cubic
+  static constexpr int POLY_PERIOD = TA_POLY_PERIOD, POLY_PAIRS = TA_POLY_PAIRS;
 };
 
 struct FwdBars {
@@ -87,7 +101,7 @@ __device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, ui
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                     const FwdParams p) {
@@ -99,9 +113,11 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item: (batch*head, pair of query tiles); heaviest pairs first when causal
-  const int bh = blockIdx.x / p.n_qp;
-  const int qpi = blockIdx.x % p.n_qp;
-  const int qp = p.causal ? (p.n_qp - 1 - qpi) : qpi;
+  // non-causal: a head's query pairs are consecutive (its K/V stay in L2);
+  // causal: all heads' heaviest pairs first (longest-processing-time order)
+  const int BH = gridDim.x / p.n_qp;
+  const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qp);
+  const int qp = p.causal ? p.n_qp - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qp);
   int r0[2], n[2];
   bool present[2];
 #pragma unroll
@@ -138,7 +154,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   reg_dealloc<C::REG_LOW>();
+   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -253,9 +271,11 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
+   }
   } else {
+    reg_alloc<C::REG_HIGH>();
     // ================================================================ softmax
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;  // row within the tile == TMEM lane
     const int row = r0[t] + rr;
@@ -290,11 +310,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[0][i]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[1][i]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[2][i]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[3][i]));
+      for (int i = 0; i < 32; i += 2) {
+        mx0 = fmax3(mx0, __uint_as_float(s[0][i]), __uint_as_float(s[0][i + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(s[1][i]), __uint_as_float(s[1][i + 1]));
+        mx2 = fmax3(mx2, __uint_as_float(s[2][i]), __uint_as_float(s[2][i + 1]));
+        mx3 = fmax3(mx3, __uint_as_float(s[3][i]), __uint_as_float(s[3][i + 1]));
       }
       const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
       // lazy rescale: move the reference max only when it rises by more than TAU
@@ -317,19 +337,44 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float ls0 = 0.f, ls1 = 0.f;
+      const uint64_t sl2x2 = f2(sl2, sl2), negmx2 = f2(negm, negm);
+      uint64_t lsA = f2(0.f, 0.f), lsB = f2(0.f, 0.f);
       uint32_t pk[2][32];
+      if ((tail || diag) || C::POLY_PAIRS == 0) {
+        // hardware ex2 throughout (masked tiles: -inf scores must give exactly 0)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[c][2 * i]), sl2, negm));
-          const float p1 = ex2(fmaf(__uint_as_float(s[c][2 * i + 1]), sl2, negm));
-          ls0 += p0;
-          ls1 += p1;
-          pk[c >> 1][(c & 1) * 16 + i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negmx2), x0,
+                     x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (i & 1) lsB = fadd2(lsB, f2(p0, p1));
+            else lsA = fadd2(lsA, f2(p0, p1));
+            pk[c >> 1][(c & 1) * 16 + i] = pack_bf16(p0, p1);
+          }
+        }
+      } else {
+        // split the exponentials between the MUFU unit and the FMA pipes
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sl2x2, negmx2), x0,
+                     x1);
+            const bool soft = (i % C::POLY_PERIOD) >= C::POLY_PERIOD - C::POLY_PAIRS;
+            const float p0 = soft ? exp2_poly(x0) : ex2(x0);
+            const float p1 = soft ? exp2_poly(x1) : ex2(x1);
+            if (i & 1) lsB = fadd2(lsB, f2(p0, p1));
+            else lsA = fadd2(lsA, f2(p0, p1));
+            pk[c >> 1][(c & 1) * 16 + i] = pack_bf16(p0, p1);
+          }
         }
       }
+      float ls0, ls1;
+      f2_split(fadd2(lsA, lsB), ls0, ls1);
       l += ls0 + ls1;
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
@@ -370,7 +415,7 @@ __global__ void __launch_bounds__(320, 1)
         p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&bars->epi[t]));
-      if (warp == 2 + 4 * t && lane == 0) {
+      if (warp == 4 + 4 * t && lane == 0) {
         if (wait_bar(smem_u32(&bars->epi[t]), 0, abort_flag, p.timeout_ns)) {
           for (int h = 0; h < D / 64; ++h)
             tma_store_3d(&tmO, sbase + C::Q_OFF + t * C::TILE + h * C::HALF, h * 64, r0[t], bh);

@@ -1,0 +1,414 @@
+// INT8 tiled attention forward for sm_100a (TMA + tcgen05 kind::i8 + TMEM).
+//
+// "INT-FlashAttention" page: Q, K and V quantised to INT8 with token-level
+// scales, and the two matmuls of the FlashAttention forward run as INT8 GEMMs
+// with int32 accumulation.  Steps per 128-key block j (same tiling, masking
+// and online softmax as the bf16 kernel, "Can a full-day context beat one
+// minute? ..." sections "The Flash Attention algorithm" and "Online softmax
+// recurrence"):
+//   S_j  = Q_i8 K_j,i8^T                         int32, exact (tensor core)
+//   x    = S_j * s_Q[row] * s_K[key] * scale * log2(e)          fp32
+//   m    = running row max, moved on EVERY increase (P must stay <= 1)
+//   P8   = rne(127 * 2^(x - m)) in [0, 127]    int8, written to TMEM
+//   ACC += P8 V_j,i8                             int32 (tensor core)
+//   l    = l * 2^(m_old - m) + sum(P8) / 127
+// When the max of a row moves, the int32 accumulator cannot be rescaled in
+// place, so the row's ACC is folded into an fp32 accumulator OF
+// (OF = (OF + ACC * s_V / 127) * 2^(m_old - m_new), ACC = 0).  At the end
+// O = (OF + ACC * s_V / 127) / l (fp32 output) and LSE = ln2 * (m + log2 l).
+//
+// CTA = one (batch, head) x one 128-row query tile.  Warps: 0 TMA producer,
+// 1 MMA issuer, 2-5 softmax/fold/epilogue (thread = TMEM lane = query row).
+// TMEM: S_0 cols [0,128), S_1 [128,256) (double-buffered scores, so S_{j+1}
+// is computed while block j is in the softmax; P8_j aliases the first 32
+// columns of S_{j%2}), ACC [256,384) int32, OF [384,512) fp32.
+// Shared memory: Q tile (128 x 128 int8 = 16 KB) and a ring of K/V tiles,
+// 128-byte swizzled.  d = 128 only.
+#pragma once
+#include "ptx.cuh"
+#include "fwd_bf16.cuh"  // fwd_tile_kv_count, wait_bar_drain
+
+namespace ta {
+
+struct FwdI8Params {
+  const float* q_scale;  // [BH][Nq]
+  const float* k_scale;  // [BH][Nkv]
+  const float* v_scale;  // [BH]
+  float* o;              // [BH][Nq][128] fp32
+  float* lse;            // [BH][Nq]
+  int* s_out;            // optional [BH][Nq][Nkv] int32 scores (debug export), else null
+  int Nq, Nkv, n_qt, Tc;
+  int causal;
+  int ks_vec;  // k_scale rows are 16-byte aligned (Nkv % 4 == 0): vector loads
+  float sl2;
+  unsigned long long timeout_ns;
+};
+
+// kind::i8 instruction descriptor: D = s32 (2), A = B = signed 8-bit (1),
+// M = 128; b_mn: B stored MN-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int N, bool b_mn) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(128 >> 4) << 24);
+}
+
+struct FwdI8Cfg {
+  static constexpr int D = 128;
+  static constexpr int TILE = 128 * 128;  // bytes of a 128 x 128 int8 tile
+  static constexpr int NSLOT = 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int SLOT_OFF = TILE;
+  static constexpr int BAR_OFF = SLOT_OFF + NSLOT * TILE;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t ID_S = idesc_i8(128, false);
+  static constexpr uint32_t ID_PV = idesc_i8(128, true);  // V is MN-major
+};
+
+struct FwdI8Bars {
+  uint64_t q_full;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t o_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(FwdI8Bars) <= 256, "barrier block too large");
+
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// exact int32 -> fp32 for |v| < 2^22 (|S| <= 127 * 127 * 128 < 2^21)
+__device__ __forceinline__ float i2f_small(uint32_t v) {
+  return __int_as_float((int)v + 0x4B400000) - 12582912.f;
+}
+
+template <bool SCORES_ONLY>
+__global__ void __launch_bounds__(192, 1)
+    fwd_int8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdI8Params p) {
+  using C = FwdI8Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FwdI8Bars* bars = reinterpret_cast<FwdI8Bars*>(smem + C::BAR_OFF);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int BH = gridDim.x / p.n_qt;
+  const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qt);
+  const int qt = p.causal ? p.n_qt - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qt);
+  const int r0 = qt * 128;
+  const int n = fwd_tile_kv_count(r0, p.Nq, p.Nkv, p.Tc, p.causal);
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full[0]), 1);
+    mbar_init(smem_u32(&bars->s_full[1]), 1);
+    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->pv_done), 1);
+    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tmem_base;
+  // load order: K_0, V_0, K_1, V_1, ... (scores-only: K_0, K_1, ...)
+  auto kidx = [&](int j) { return SCORES_ONLY ? j : 2 * j; };
+  auto vidx = [&](int j) { return 2 * j + 1; };
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      if (!SCORES_ONLY) prefetch_tmap(&tmV);
+      const uint32_t qbar = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qbar, C::TILE);
+      tma_load_3d(sbase + C::Q_OFF, &tmQ, qbar, 0, r0, bh);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        for (int w = 0; w < (SCORES_ONLY ? 1 : 2) && ok; ++w, ++it) {
+          const int slot = it % C::NSLOT;
+          const uint32_t ph = (it / C::NSLOT) & 1;
+          ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+          mbar_arrive_expect_tx(fb, C::TILE);
+          tma_load_3d(sbase + C::SLOT_OFF + slot * C::TILE, w == 0 ? &tmK : &tmV, fb, 0, j * 128, bh);
+        }
+      }
+      if (!ok) {
+        wait_bar_drain(qbar, 0, p.timeout_ns);
+        for (int back = 1; back <= C::NSLOT && it - back >= 0; ++back) {
+          const int i2 = it - back;
+          wait_bar_drain(smem_u32(&bars->kv_full[i2 % C::NSLOT]), (i2 / C::NSLOT) & 1, p.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
+      tc_fence_after();
+      auto issue_S = [&](int j) -> bool {
+        const int it = kidx(j), s = it % C::NSLOT;
+        if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t ka = sbase + C::SLOT_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = 32 int8 per MMA
+          mma_i8_ss(tbase + (j & 1) * 128, smem_desc(sbase + C::Q_OFF + kk * 32, 16, 1024),
+                    smem_desc(ka + kk * 32, 16, 1024), C::ID_S, kk > 0);
+        tc_commit(smem_u32(&bars->s_full[j & 1]));
+        tc_commit(smem_u32(&bars->kv_empty[s]));
+        return true;
+      };
+      if (ok && n == 0) tc_commit(smem_u32(&bars->o_full));
+      if (ok && n > 0) ok = issue_S(0);
+      if (ok && n > 1) ok = issue_S(1);
+      for (int j = 0; j < n && ok && !SCORES_ONLY; ++j) {
+        const int it = vidx(j), s = it % C::NSLOT;
+        ok = wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        ok = wait_bar(smem_u32(&bars->p_full), j & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t va = sbase + C::SLOT_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // 32 keys per MMA: 32 rows x 128 B of V
+          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + kk * 8, smem_desc(va + kk * 4096, C::TILE, 1024),
+                    C::ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bars->pv_done));
+        tc_commit(smem_u32(&bars->kv_empty[s]));
+        if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
+        if (j + 2 < n) ok = issue_S(j + 2);
+      }
+      if (SCORES_ONLY) {
+        for (int j = 2; j < n && ok; ++j) {
+          // the score buffer of j is free once the softmax warps read block j-2
+          ok = wait_bar(smem_u32(&bars->p_full), (j - 2) & 1, abort_flag, p.timeout_ns);
+          if (ok) ok = issue_S(j);
+        }
+      }
+      if (!ok) {
+        tc_commit(smem_u32(&bars->drain));
+        wait_bar_drain(smem_u32(&bars->drain), 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax
+    const int quarter = warp & 3;
+    const int rr = quarter * 32 + lane;
+    const int row = r0 + rr;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tACC = tbase + lane_off + 256;
+    const uint32_t tOF = tbase + lane_off + 384;
+    const int off = p.Nkv - p.Nq;
+    const float crow = (!SCORES_ONLY && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] * p.sl2 : 0.f;
+    const float sv127 = SCORES_ONLY ? 0.f : p.v_scale[bh] * (1.f / 127.f);
+    const float* ksrow = p.k_scale + (size_t)bh * p.Nkv;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    if (!SCORES_ONLY) {
+      uint32_t z[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_st32(tOF + cc * 32, z);
+      tmem_st_wait();
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int kb = j * 128;
+      ok = wait_bar(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tbase + lane_off + (j & 1) * 128;
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      if (SCORES_ONLY) {
+        if (row < p.Nq) {
+          int* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (kb + c * 32 + i < p.Nkv) dst[c * 32 + i] = (int)s[c][i];
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->p_full));
+        continue;
+      }
+      // x = S * s_Q * s_K * scale * log2e, masked
+      const bool tail = kb + 128 > p.Nkv;
+      const bool diag = p.causal && (kb + 127 > r0 + off);
+      int lim = 127;
+      if (tail || diag) {
+        lim = p.Nkv - 1 - kb;
+        if (p.causal) lim = min(lim, row + off - kb);
+      }
+      float x[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const int col = c * 32 + i;
+          float4 ks;
+          if (!tail && p.ks_vec) {
+            ks = __ldg(reinterpret_cast<const float4*>(ksrow + kb + col));
+          } else {
+            ks.x = (kb + col + 0 < p.Nkv) ? ksrow[kb + col + 0] : 0.f;  // scalar path
+            ks.y = (kb + col + 1 < p.Nkv) ? ksrow[kb + col + 1] : 0.f;
+            ks.z = (kb + col + 2 < p.Nkv) ? ksrow[kb + col + 2] : 0.f;
+            ks.w = (kb + col + 3 < p.Nkv) ? ksrow[kb + col + 3] : 0.f;
+          }
+          x[c][i + 0] = (col + 0 <= lim) ? i2f_small(s[c][i + 0]) * (ks.x * crow) : -INFINITY;
+          x[c][i + 1] = (col + 1 <= lim) ? i2f_small(s[c][i + 1]) * (ks.y * crow) : -INFINITY;
+          x[c][i + 2] = (col + 2 <= lim) ? i2f_small(s[c][i + 2]) * (ks.z * crow) : -INFINITY;
+          x[c][i + 3] = (col + 3 <= lim) ? i2f_small(s[c][i + 3]) * (ks.w * crow) : -INFINITY;
+        }
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        mx0 = fmax3(mx0, x[0][i], x[0][i + 1]);
+        mx1 = fmax3(mx1, x[1][i], x[1][i + 1]);
+        mx2 = fmax3(mx2, x[2][i], x[2][i + 1]);
+        mx3 = fmax3(mx3, x[3][i], x[3][i + 1]);
+      }
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      // tau = 0: move the reference on every increase
+      const bool grow = m_blk > m_ref;
+      const bool had = m_ref != -INFINITY;  // rows with earlier content need a fold
+      float factor = 1.f;
+      if (grow) {
+        factor = had ? ex2(m_ref - m_blk) : 0.f;
+        l *= factor;
+        m_ref = m_blk;
+      }
+      const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      uint32_t isum = 0;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          uint32_t t[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float y = ex2(x[c][i + e] + negm) * 127.f;
+            t[e] = __float_as_uint(y + 12582912.f);  // low bits: rne(y) in [0, 127]
+            isum += t[e];
+          }
+          const uint32_t lo = __byte_perm(t[0], t[1], 0x0040);
+          const uint32_t hi = __byte_perm(t[2], t[3], 0x0040);
+          pk[c * 8 + i / 4] = __byte_perm(lo, hi, 0x5410);
+        }
+      }
+      isum -= 128u * 0x4B400000u;  // remove the magic offsets (mod 2^32)
+      l += (float)isum * (1.f / 127.f);
+      tmem_st32(tS, pk);  // P8 of block j -> first 32 columns of its score buffer
+      if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
+        // fold ACC (P V of blocks < j, reference m_old) into OF
+        ok = wait_bar(smem_u32(&bars->pv_done), (j - 1) & 1, abort_flag, p.timeout_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float f = (grow && had) ? factor : 1.f;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t a[32], o[32];
+          tmem_ld32(tACC + cc * 32, a);
+          tmem_ld32(tOF + cc * 32, o);
+          tmem_ld_wait(a);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            o[i] = __float_as_uint((__uint_as_float(o[i]) + (float)(int)a[i] * sv127) * f);
+            a[i] = 0u;
+          }
+          tmem_st32(tOF + cc * 32, o);
+          tmem_st32(tACC + cc * 32, a);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->p_full));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (!SCORES_ONLY && ok) {
+      ok = wait_bar(smem_u32(&bars->o_full), 0, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        float* orow = p.o + ((size_t)bh * p.Nq + row) * C::D;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t a[32], o[32];
+          tmem_ld32(tACC + cc * 32, a);
+          tmem_ld32(tOF + cc * 32, o);
+          tmem_ld_wait(a);
+          tmem_ld_wait(o);
+          if (row < p.Nq) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 v;
+              v.x = (l > 0.f) ? (__uint_as_float(o[i + 0]) + (float)(int)a[i + 0] * sv127) * inv : 0.f;
+              v.y = (l > 0.f) ? (__uint_as_float(o[i + 1]) + (float)(int)a[i + 1] * sv127) * inv : 0.f;
+              v.z = (l > 0.f) ? (__uint_as_float(o[i + 2]) + (float)(int)a[i + 2] * sv127) * inv : 0.f;
+              v.w = (l > 0.f) ? (__uint_as_float(o[i + 3]) + (float)(int)a[i + 3] * sv127) * inv : 0.f;
+              *reinterpret_cast<float4*>(orow + cc * 32 + i) = v;
+            }
+          }
+        }
+        if (row < p.Nq)
+          p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace ta
