@@ -116,6 +116,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise MAX of a list of floats over all ranks (a no-op without an
+    initialised process group).  Timings of replicated work are reduced this
+    way: the job is as slow as its slowest rank."""
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world_size, steps, work_per_step, max_ms):
+    """Whole-job rate: every rank processed `steps` x `work_per_step` units in
+    at most `max_ms` (weak scaling: the work grows with the ranks)."""
+    return world_size * steps * work_per_step / (max_ms * 1e-3)
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -251,14 +268,10 @@ def run_ours(args):
     nc_ms = [e[0].elapsed_time(e[1]) for e in evs]
     c_ms = [e[1].elapsed_time(e[2]) for e in evs]
     dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    sums = torch.tensor([total_ms, sum(nc_ms), sum(c_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.all_reduce(sums, op=dist.ReduceOp.MAX)
-    total_ms, nc_tot, c_tot, dec_tot = sums.tolist()
+    total_ms, nc_tot, c_tot, dec_tot = max_over_ranks([total_ms, sum(nc_ms), sum(c_ms), sum(dec_ms)], dev)
 
     prefill_ms = nc_tot + c_tot
-    value = ws * args.steps * (flops_nc + flops_c) / (prefill_ms * 1e-3) / 1e12
+    value = job_throughput(ws, args.steps, flops_nc + flops_c, prefill_ms) / 1e12
     nc_avg = nc_tot / args.steps
     c_avg = c_tot / args.steps
     dec_avg = dec_tot / args.steps
@@ -298,14 +311,10 @@ def run_ours(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if ws > 1:
-            import torch.distributed as dist
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e_ms = e_ms.item()
+        e_ms = max_over_ranks([a.elapsed_time(b)], dev)[0]
         h2d = 3 * q.numel() * q.element_size()
         d2h = 2 * (o.numel() * o.element_size() + lse.numel() * lse.element_size())
-        e2e = {"value": ws * args.e2e_steps * (flops_nc + flops_c) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_throughput(ws, args.e2e_steps, flops_nc + flops_c, e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps}
 

@@ -169,12 +169,11 @@ __global__ void __launch_bounds__(384, 1)
         for (int h = 0; h < D / 64; ++h)
           tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
       }
-      int it = 0;
+      int it = 0, slot = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int j = 0; j < nmax && ok; ++j) {
-        for (int w = 0; w < 2 && ok; ++w, ++it) {
-          const int slot = it % C::NSLOT;
-          const uint32_t ph = (it / C::NSLOT) & 1;
+        for (int w = 0; w < 2 && ok; ++w, ++it, (++slot == C::NSLOT) ? (slot = 0, ph ^= 1u) : 0u) {
           ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
           if (!ok) break;
           const uint32_t fb = smem_u32(&bars->kv_full[slot]);
@@ -196,73 +195,110 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // The tensor pipe holds little beyond the MMA in flight, so anything the
+    // issuing thread does between two MMAs idles it.  Hence: descriptors are
+    // built once (one 64-bit add per MMA), slot/phase counters advance
+    // incrementally, and the barrier of the NEXT group is tested (without
+    // blocking) just before the last MMA of the current group is issued, so
+    // that the test's latency hides behind that MMA.
     if (lane == 0) {
       bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
       tc_fence_after();
-      auto slot_of = [&](int it) { return it % C::NSLOT; };
-      auto par_of = [&](int it) { return (uint32_t)((it / C::NSLOT) & 1); };
-      auto issue_S = [&](int t, int j) {
-        const int s = slot_of(2 * j);
-        const uint32_t qa = sbase + C::Q_OFF + t * C::TILE;
-        const uint32_t ka = sbase + C::SLOT_OFF + s * C::TILE;
+      const uint64_t dQ0 = smem_desc(sbase + C::Q_OFF, 16, 1024);
+      const uint64_t dQ1 = smem_desc(sbase + C::Q_OFF + C::TILE, 16, 1024);
+      const uint64_t dK0 = smem_desc(sbase + C::SLOT_OFF, 16, 1024);
+      const uint64_t dV0 = smem_desc(sbase + C::SLOT_OFF, C::HALF, 1024);
+      // K_j is load number 2j, V_j number 2j+1 (slot = number % NSLOT,
+      // phase = (number / NSLOT) & 1)
+      int sK = 0, sV = 1 % C::NSLOT;
+      uint32_t pK = 0, pV = (1 >= C::NSLOT) ? 1u : 0u;
+      auto adv = [&](int& sl, uint32_t& ph) {
+        sl += 2;
+        if (sl >= C::NSLOT) { sl -= C::NSLOT; ph ^= 1u; }
+      };
+      // Issue one S group; before its last MMA, test barrier (nb, np).
+      auto issue_S = [&](int t, int sl, uint32_t nb, uint32_t np) -> bool {
+        const uint64_t dq = t ? dQ1 : dQ0;
+        const uint64_t dk = dK0 + (uint64_t)(sl * (C::TILE >> 4));
+        const uint32_t dS = tbase + t * 128;
+        bool ready = true;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
-          mma_f16_ss(tbase + t * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), C::ID_S,
-                     kk > 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
+          if (kk == D / 16 - 1 && nb) ready = mbar_test_wait(nb, np);
+          mma_f16_ss(dS, dq + off, dk + off, C::ID_S, kk > 0);
         }
         tc_commit(smem_u32(&bars->s_full[t]));
+        return ready;
       };
-      auto issue_PV = [&](int t, int j) {
-        const int s = slot_of(2 * j + 1);
-        const uint32_t va = sbase + C::SLOT_OFF + s * C::TILE;
+      auto issue_PV = [&](int t, int sl, int j, uint32_t nb, uint32_t np) -> bool {
+        const uint64_t dv = dV0 + (uint64_t)(sl * (C::TILE >> 4));
+        const uint32_t dO = tbase + 256 + t * D, aP = tbase + t * 128;
+        const uint32_t acc0 = (j > 0) ? 1u : 0u;
+        bool ready = true;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
-          mma_f16_ts(tbase + 256 + t * D, tbase + t * 128 + kk * 8, smem_desc(va + kk * 2048, C::HALF, 1024),
-                     C::ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          if (kk == 7 && nb) ready = mbar_test_wait(nb, np);
+          mma_f16_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), C::ID_PV, kk > 0 ? 1u : acc0);
         }
+        return ready;
       };
+      // wait for (bar, parity) unless a speculative test already saw it
+      auto need = [&](bool seen, uint32_t bar, uint32_t par) -> bool {
+        if (!seen && !wait_bar(bar, par, abort_flag, p.timeout_ns)) return false;
+        tc_fence_after();
+        return true;
+      };
+      const uint32_t pf0 = smem_u32(&bars->p_full[0]), pf1 = smem_u32(&bars->p_full[1]);
       if (ok && nmax > 0) {
-        ok = wait_bar(smem_u32(&bars->kv_full[slot_of(0)]), par_of(0), abort_flag, p.timeout_ns);
+        ok = wait_bar(smem_u32(&bars->kv_full[sK]), pK, abort_flag, p.timeout_ns);
         tc_fence_after();
         if (ok) {
-          if (n[0] > 0) issue_S(0, 0);
-          if (n[1] > 0) issue_S(1, 0);
-          tc_commit(smem_u32(&bars->kv_empty[slot_of(0)]));
+          if (n[0] > 0) issue_S(0, sK, 0, 0);
+          if (n[1] > 0) issue_S(1, sK, 0, 0);
+          tc_commit(smem_u32(&bars->kv_empty[sK]));
         }
       }
       if (ok) {
         for (int t = 0; t < 2; ++t)
           if (present[t] && n[t] == 0) tc_commit(smem_u32(&bars->o_full[t]));
       }
+      bool seenV = false;
       for (int j = 0; j < nmax && ok; ++j) {
-        ok = wait_bar(smem_u32(&bars->kv_full[slot_of(2 * j + 1)]), par_of(2 * j + 1), abort_flag, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
+        // V_j is needed by both P V groups of this step
+        if (!(ok = need(seenV, smem_u32(&bars->kv_full[sV]), pV))) break;
+        const bool nextK = j + 1 < nmax;
+        int sK1 = sK;
+        uint32_t pK1 = pK;
+        if (nextK) adv(sK1, pK1);
+        const uint32_t kbar = nextK ? smem_u32(&bars->kv_full[sK1]) : 0u;
+        bool seenK = !nextK;
         if (j < n[0]) {
-          ok = wait_bar(smem_u32(&bars->p_full[0]), j & 1, abort_flag, p.timeout_ns);
-          if (!ok) break;
-          tc_fence_after();
-          issue_PV(0, j);
+          if (!(ok = need(false, pf0, j & 1))) break;
+          seenK = issue_PV(0, sV, j, kbar, pK1) || !nextK;
           if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
         }
-        const bool nextK = j + 1 < nmax;
         if (nextK) {
-          ok = wait_bar(smem_u32(&bars->kv_full[slot_of(2 * j + 2)]), par_of(2 * j + 2), abort_flag, p.timeout_ns);
-          if (!ok) break;
-          tc_fence_after();
+          if (!(ok = need(seenK, kbar, pK1))) break;
         }
-        if (j + 1 < n[0]) issue_S(0, j + 1);
+        bool seenP1 = false;
+        if (j + 1 < n[0]) seenP1 = issue_S(0, sK1, (j < n[1]) ? pf1 : 0u, j & 1);
         if (j < n[1]) {
-          ok = wait_bar(smem_u32(&bars->p_full[1]), j & 1, abort_flag, p.timeout_ns);
-          if (!ok) break;
-          tc_fence_after();
-          issue_PV(1, j);
+          if (!(ok = need(seenP1, pf1, j & 1))) break;
+          issue_PV(1, sV, j, 0, 0);
           if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
         }
-        tc_commit(smem_u32(&bars->kv_empty[slot_of(2 * j + 1)]));
-        if (j + 1 < n[1]) issue_S(1, j + 1);
-        if (nextK) tc_commit(smem_u32(&bars->kv_empty[slot_of(2 * j + 2)]));
+        tc_commit(smem_u32(&bars->kv_empty[sV]));
+        int sV1 = sV;
+        uint32_t pV1 = pV;
+        adv(sV1, pV1);
+        seenV = false;
+        if (j + 1 < n[1]) seenV = issue_S(1, sK1, (j + 1 < nmax) ? smem_u32(&bars->kv_full[sV1]) : 0u, pV1);
+        if (nextK) tc_commit(smem_u32(&bars->kv_empty[sK1]));
+        sK = sK1;
+        pK = pK1;
+        sV = sV1;
+        pV = pV1;
       }
       if (!ok) {
         // drain: every MMA issued so far must finish before TMEM is freed

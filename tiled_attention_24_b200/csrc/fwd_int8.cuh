@@ -181,15 +181,17 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
       tc_fence_after();
+      const uint64_t dQ = smem_desc(sbase + C::Q_OFF, 16, 1024);
+      const uint64_t dK0 = smem_desc(sbase + C::SLOT_OFF, 16, 1024);
+      const uint64_t dV0 = smem_desc(sbase + C::SLOT_OFF, C::TILE, 1024);
       auto issue_S = [&](int j) -> bool {
         const int it = kidx(j), s = it % C::NSLOT;
         if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t ka = sbase + C::SLOT_OFF + s * C::TILE;
+        const uint64_t dk = dK0 + (uint64_t)(s * (C::TILE >> 4));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // K = 32 int8 per MMA
-          mma_i8_ss(tbase + (j & 1) * 128, smem_desc(sbase + C::Q_OFF + kk * 32, 16, 1024),
-                    smem_desc(ka + kk * 32, 16, 1024), C::ID_S, kk > 0);
+          mma_i8_ss(tbase + (j & 1) * 128, dQ + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), C::ID_S, kk > 0);
         tc_commit(smem_u32(&bars->s_full[j & 1]));
         tc_commit(smem_u32(&bars->kv_empty[s]));
         return true;
@@ -204,11 +206,12 @@ __global__ void __launch_bounds__(192, 1)
         ok = wait_bar(smem_u32(&bars->p_full), j & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t va = sbase + C::SLOT_OFF + s * C::TILE;
+        const uint64_t dv = dV0 + (uint64_t)(s * (C::TILE >> 4));
+        const uint32_t acc0 = (j > 0) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 keys per MMA: 32 rows x 128 B of V
-          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + kk * 8, smem_desc(va + kk * 4096, C::TILE, 1024),
-                    C::ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + kk * 8, dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV,
+                    kk > 0 ? 1u : acc0);
         tc_commit(smem_u32(&bars->pv_done));
         tc_commit(smem_u32(&bars->kv_empty[s]));
         if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
