@@ -183,6 +183,52 @@ ATTN_API int attn_int8_scores(const int8_t* q, const int8_t* k, int32_t* s, int 
                               void* stream);
 
 /*
+ * NVFP4 operands ([FP4-FA4]: FP4 Q, K, V on the FP4 tensor cores).
+ * Blocks of 16 elements, e2m1 codes (RNE, saturating at +-6) with one unsigned
+ * e4m3 scale per block: sf = e4m3_rne(amax / 6), code = e2m1_rne(x / sf)
+ * (IEEE fp32 divides; a zero block gets scale 0 and codes 0).  Two codes per
+ * byte, the lower-index element in the low nibble.  d must be 128.
+ *   mode 0 (Q, K): blocks run along d; codes [B][H][N][64 bytes];
+ *   mode 1 (V):    blocks run along tokens (P V contracts over tokens) and the
+ *                  codes are written transposed, [B][H][128][ceil(N/128)*64
+ *                  bytes] (tokens padded to a multiple of 128 with zeros).
+ * Scales: one 1 KB block per 128 rows (mode 0) or per 128 tokens (mode 1),
+ * [B][H][ceil(N/128)][1024 bytes], byte (r % 32) * 16 + (r / 32) * 4 + (b % 4)
+ * + (b / 4) * 512 for row (mode 1: channel) r of the tile and block b (0..7)
+ * -- the order in which the tensor core reads block scales.
+ * attn_nvfp4_codes_bytes / attn_nvfp4_sf_bytes give the buffer sizes (0 for
+ * an unsupported shape).
+ */
+ATTN_API size_t attn_nvfp4_codes_bytes(int B, int H, int N, int d, int mode);
+ATTN_API size_t attn_nvfp4_sf_bytes(int B, int H, int N, int d, int mode);
+ATTN_API int attn_quantize_nvfp4(const attn_bf16_t* x, uint8_t* codes, uint8_t* sf, int B, int H, int N, int d,
+                                 int mode, void* stream);
+
+/*
+ * attn_fwd_fp4 -- FP4 attention forward with block-scaled FP4 tensor-core
+ * MMAs for Q K^T and P V ([FP4-FA4]).  P is encoded either with Direct-P
+ * (p_mode 0: the score maps straight to the e2m1 code of 6 * exp(x - m),
+ * every P block scale 1) or quantised after the exponential (p_mode 1: per
+ * 16 keys, sf = e4m3_rne(amax(p) / 6), code = e2m1_rne(p / sf)).  The running
+ * max moves on every increase; l sums the dequantised P (divided by 6 for
+ * Direct-P); O = acc / l (fp32), LSE = m + ln l.
+ *   q, k: mode-0 codes + scales of Q [B][H][Nq][128], K [B][H][Nkv][128];
+ *   vt, vt_sf: mode-1 codes + scales of V; o [B][H][Nq][128] fp32 out,
+ *   lse [B][H][Nq] fp32 out.  d must be 128; Nkv >= 1.
+ */
+ATTN_API int attn_fwd_fp4(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                          const uint8_t* vt, const uint8_t* vt_sf, float* o, float* lse, int B, int H, int Nq,
+                          int Nkv, int d, int causal, float scale, int p_mode, void* stream);
+
+/*
+ * attn_fp4_scores -- S = deq(q) deq(k)^T (fp32, [B][H][Nq][Nkv]) through the
+ * same block-scaled tensor-core path as attn_fwd_fp4 (a check of the FP4
+ * GEMM; small sizes).
+ */
+ATTN_API int attn_fp4_scores(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf, float* s,
+                             int B, int H, int Nq, int Nkv, int d, void* stream);
+
+/*
  * attn_check_status -- synchronise `stream`, read the device status word
  * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT), clear it and
  * return it; also returns ATTN_ERR_CUDA if the synchronisation itself fails.

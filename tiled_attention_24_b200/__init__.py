@@ -11,14 +11,19 @@ import math
 import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
-                       attn_decode_noalloc, attn_decode_workspace_bytes, attn_fwd, attn_fwd_int8,
-                       attn_int8_scores, attn_quantize_int8, attn_set_wait_limit_ns, attn_status_string,
-                       attn_version, attn_watchdog_selftest, load)
+                       attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores, attn_fwd,
+                       attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
+                       attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
+                       attn_status_string, attn_version, attn_watchdog_selftest, load)
 
 __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "attn_check_status",
            "attn_set_wait_limit_ns", "attn_watchdog_selftest", "attn_version", "attn_status_string",
            "AttnError", "forward", "decode", "quantize_int8", "forward_int8",
-           "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc"]
+           "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc",
+           "attn_quantize_nvfp4", "attn_fwd_fp4", "attn_fp4_scores", "quantize_nvfp4", "forward_fp4",
+           "DIRECT_P", "QUANT_AFTER_EXP"]
+
+DIRECT_P, QUANT_AFTER_EXP = 0, 1
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
@@ -66,4 +71,28 @@ def forward_int8(q, k, v, causal: bool = False, scale: float | None = None, stre
     o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     attn_fwd_int8(qi, qs, ki, ks, vi, vs, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def quantize_nvfp4(x: torch.Tensor, mode: int, stream=None):
+    """NVFP4 codes + tiled scales of a bf16 [B,H,N,128] tensor (mode 0: Q/K,
+    mode 1: V, written transposed)."""
+    B, H, N, d = x.shape
+    codes = torch.empty(attn_nvfp4_codes_bytes(B, H, N, d, mode), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(attn_nvfp4_sf_bytes(B, H, N, d, mode), dtype=torch.uint8, device=x.device)
+    attn_quantize_nvfp4(x, codes, sf, mode, stream)
+    return codes, sf
+
+
+def forward_fp4(q, k, v, causal: bool = False, scale: float | None = None, p_mode: int = DIRECT_P, stream=None):
+    """Quantise bf16 q, k, v to NVFP4 and run the FP4 forward.  Returns (o fp32, lse fp32)."""
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    qc, qs = quantize_nvfp4(q, 0, stream)
+    kc, ks = quantize_nvfp4(k, 0, stream)
+    vc, vs = quantize_nvfp4(v, 1, stream)
+    o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    attn_fwd_fp4(qc, qs, kc, ks, vc, vs, o, lse, B, H, Nq, Nkv, causal, scale, p_mode, stream)
     return o, lse

@@ -33,6 +33,11 @@ SIGNATURES = [
     ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_fwd_int8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_int8_scores", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    ("attn_nvfp4_codes_bytes", _SZ, [_I, _I, _I, _I, _I]),
+    ("attn_nvfp4_sf_bytes", _SZ, [_I, _I, _I, _I, _I]),
+    ("attn_quantize_nvfp4", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    ("attn_fwd_fp4", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
+    ("attn_fp4_scores", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_check_status", _I, [_VP]),
     ("attn_set_wait_limit_ns", None, [_ULL]),
     ("attn_watchdog_selftest", _I, [_ULL, _VP]),
@@ -147,6 +152,38 @@ def attn_int8_scores(q, k, s, stream=None):
     B, H, Nq, d = q.shape
     _check("attn_int8_scores", load().attn_int8_scores(_ptr(q), _ptr(k), _ptr(s), B, H, Nq, k.shape[2], d,
                                                          _stream(stream)))
+
+
+def attn_nvfp4_codes_bytes(B: int, H: int, N: int, d: int, mode: int) -> int:
+    return int(load().attn_nvfp4_codes_bytes(B, H, N, d, mode))
+
+
+def attn_nvfp4_sf_bytes(B: int, H: int, N: int, d: int, mode: int) -> int:
+    return int(load().attn_nvfp4_sf_bytes(B, H, N, d, mode))
+
+
+def attn_quantize_nvfp4(x, codes, sf, mode: int, stream=None):
+    """bf16 [B,H,N,128] -> packed e2m1 codes + tiled e4m3 scales (mode 0: Q/K, 1: V^T)."""
+    _need_cuda(x, codes, sf)
+    B, H, N, d = x.shape
+    _check("attn_quantize_nvfp4", load().attn_quantize_nvfp4(_ptr(x), _ptr(codes), _ptr(sf), B, H, N, d, int(mode),
+                                                               _stream(stream)))
+
+
+def attn_fwd_fp4(q, qsf, k, ksf, vt, vtsf, o, lse, B, H, Nq, Nkv, causal: bool, scale: float, p_mode: int,
+                 stream=None):
+    """FP4 forward (codes/scales from attn_quantize_nvfp4) -> o fp32 [B,H,Nq,128], lse fp32."""
+    _need_cuda(q, qsf, k, ksf, vt, vtsf, o, lse)
+    rc = load().attn_fwd_fp4(_ptr(q), _ptr(qsf), _ptr(k), _ptr(ksf), _ptr(vt), _ptr(vtsf), _ptr(o), _ptr(lse),
+                             B, H, Nq, Nkv, 128, int(bool(causal)), float(scale), int(p_mode), _stream(stream))
+    _check("attn_fwd_fp4", rc)
+
+
+def attn_fp4_scores(q, qsf, k, ksf, s, B, H, Nq, Nkv, stream=None):
+    """fp32 S = deq(q) deq(k)^T through the block-scaled FP4 MMA path."""
+    _need_cuda(q, qsf, k, ksf, s)
+    _check("attn_fp4_scores", load().attn_fp4_scores(_ptr(q), _ptr(qsf), _ptr(k), _ptr(ksf), _ptr(s), B, H, Nq, Nkv,
+                                                       128, _stream(stream)))
 
 
 def attn_check_status(stream=None) -> int:

@@ -16,6 +16,7 @@
 #include "decode.cuh"
 #include "quant.cuh"
 #include "fwd_int8.cuh"
+#include "fwd_fp4.cuh"
 
 namespace {
 
@@ -66,6 +67,61 @@ int make_tmap_i8(CUtensorMap* m, const void* ptr, int N, int BH) {
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// packed e2m1 codes viewed as (row_bytes, rows, BH) bytes; boxes of 64 x 128 x 1
+// with 64-byte swizzle (one swizzle span per 128-code row)
+int make_tmap_fp4(CUtensorMap* m, const void* ptr, long long row_bytes, int rows, int BH) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * rows};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool SCORES_ONLY>
+int launch_fp4(const void* q, const void* qsf, const void* k, const void* ksf, const void* vt, const void* vsf,
+               float* o, float* lse, float* s_out, int B, int H, int Nq, int Nkv, int causal, float scale,
+               int p_mode, cudaStream_t st) {
+  using C = ta::FwdF4Cfg;
+  const int BH = B * H;
+  const int KT = (Nkv + 127) / 128;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_fp4(&tq, q, 64, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_fp4(&tk, k, 64, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_fp4(&tv, SCORES_ONLY ? k : vt, SCORES_ONLY ? 64 : (long long)KT * 64,
+                          SCORES_ONLY ? Nkv : 128, BH)) != ATTN_OK)
+    return rc;
+  if (cudaFuncSetAttribute(ta::fwd_fp4_kernel<SCORES_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  ta::FwdF4Params p;
+  p.q_sf = static_cast<const uint8_t*>(qsf);
+  p.k_sf = static_cast<const uint8_t*>(ksf);
+  p.v_sf = static_cast<const uint8_t*>(vsf);
+  p.o = o;
+  p.lse = lse;
+  p.s_out = s_out;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.n_qt = (Nq + 127) / 128;
+  p.Tc = KT;
+  p.RTq = (Nq + 127) / 128;
+  p.KT = KT;
+  p.causal = causal ? 1 : 0;
+  p.p_mode = p_mode;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_ns;
+  const long long grid = (long long)BH * p.n_qt;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  ta::fwd_fp4_kernel<SCORES_ONLY><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <bool SCORES_ONLY>
@@ -357,6 +413,67 @@ int attn_int8_scores(const int8_t* q, const int8_t* k, int32_t* s, int B, int H,
   if (!aligned16(q) || !aligned16(k) || !aligned4(s)) return ATTN_ERR_MISALIGNED;
   return launch_int8<true>(q, nullptr, k, nullptr, nullptr, nullptr, nullptr, nullptr, s, B, H, Nq, Nkv, 0, 1.f,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_nvfp4_codes_bytes(int B, int H, int N, int d, int mode) {
+  if (B <= 0 || H <= 0 || N <= 0 || d != 128) return 0;
+  const size_t BH = (size_t)B * H;
+  return mode ? BH * 128 * (size_t)((N + 127) / 128) * 64 : BH * (size_t)N * 64;
+}
+
+size_t attn_nvfp4_sf_bytes(int B, int H, int N, int d, int mode) {
+  if (B <= 0 || H <= 0 || N <= 0 || d != 128) return 0;
+  (void)mode;  // both modes: one 1 KB block per 128-row (or 128-token) tile
+  return (size_t)B * H * (size_t)((N + 127) / 128) * 1024;
+}
+
+int attn_quantize_nvfp4(const attn_bf16_t* x, uint8_t* codes, uint8_t* sf, int B, int H, int N, int d, int mode,
+                        void* stream) {
+  if (B < 0 || H < 0 || N < 0 || (mode != 0 && mode != 1)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!x || !codes || !sf) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long BH = (long long)B * H;
+  const int T = (N + 127) / 128;
+  if (mode == 0) {
+    const long long total = BH * T * 128 * 8;
+    ta::quant_nvfp4_rows_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(x, codes, sf, N, T, total);
+  } else {
+    const long long total = BH * T * 8 * 128;
+    ta::quant_nvfp4_cols_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(x, codes, sf, N, T, total);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_fwd_fp4(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf, const uint8_t* vt,
+                 const uint8_t* vt_sf, float* o, float* lse, int B, int H, int Nq, int Nkv, int d, int causal,
+                 float scale, int p_mode, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || (p_mode != 0 && p_mode != 1)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;
+  if (Nkv == 0) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(q_sf) || !aligned16(k_sf) ||
+      !aligned16(vt_sf) || !aligned16(o) || !aligned4(lse))
+    return ATTN_ERR_MISALIGNED;
+  return launch_fp4<false>(q, q_sf, k, k_sf, vt, vt_sf, o, lse, nullptr, B, H, Nq, Nkv, causal, scale, p_mode,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fp4_scores(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf, float* s, int B,
+                    int H, int Nq, int Nkv, int d, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0 || Nkv == 0) return ATTN_OK;
+  if (!q || !q_sf || !k || !k_sf || !s) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sf) || !aligned16(k_sf) || !aligned4(s))
+    return ATTN_ERR_MISALIGNED;
+  return launch_fp4<true>(q, q_sf, k, k_sf, nullptr, k_sf, nullptr, nullptr, s, B, H, Nq, Nkv, 0, 1.f, 0,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_check_status(void* stream) {

@@ -1,0 +1,467 @@
+// FP4 (NVFP4) tiled attention forward for sm_100a: tcgen05 kind::mxf4nvf4
+// block-scaled MMAs (e2m1 operands, one unsigned-e4m3 scale per 16 elements).
+//
+// "Hardware-Aware FP4 FlashAttention-4" page: the FP4 tensor cores multiply
+// fast, but turning scores into FP4 probabilities -- exponentiate, find a
+// block scale, divide, round -- stalls the pipeline; Direct-P maps the raw
+// scores straight to the hardware codes instead.  Both P encodings are here:
+//   p_mode 0, Direct-P:           P~ = e2m1_rne(6 * 2^(x - m)), block scale 1
+//   p_mode 1, quantise-after-exp: p = 2^(x - m); per 16 keys
+//                                 sf = e4m3_rne(amax(p) / 6), P~ = e2m1_rne(p / sf) * sf
+// Steps per 128-key block j (tiling, masking and online softmax as in the
+// bf16 kernel; the running max moves on every increase, so P <= 1):
+//   S  = deq(Q) deq(K_j)^T               fp32 in TMEM (block-scaled MMA)
+//   x  = S * scale * log2(e), masked
+//   m, O and l rescaled by 2^(m_old - m) when the max grows
+//   O += P~ deq(V_j)                     fp32 in TMEM (block-scaled MMA)
+//   l += sum(P~)
+//   O / l (fp32 output), LSE = ln2 * (m + log2(l / p_unit)), p_unit = 6 for
+//   Direct-P (whose P~ approximates 6 * 2^(x - m)), 1 otherwise
+//
+// CTA = one (batch, head) x one 128-row query tile; warps: 0 TMA producer,
+// 1 MMA issuer, 2-5 softmax / correction / epilogue (thread = row).
+// Operands in shared memory (64-byte swizzled, K-major, 64 bytes = 128 e2m1
+// codes per row): Q tile, ring of K and V^T tiles; each with its 1 KB of
+// scale factors, which tcgen05.cp copies into TMEM in the layout the MMA reads
+// (32 lanes x 16 bytes, replicated over the 4 lane quarters).  P is written
+// by the softmax threads into a shared-memory tile (the A operand of a
+// block-scaled MMA comes from shared memory), double-buffered, with its scale
+// factors.  TMEM: S_0 [0,128), S_1 [128,256), O [256,384), scale factors from
+// column 384.  d = 128 only.
+#pragma once
+#include "ptx.cuh"
+#include "fwd_bf16.cuh"
+#include "quant.cuh"
+
+namespace ta {
+
+struct FwdF4Params {
+  const uint8_t* q_sf;  // [BH][ceil(Nq/128)][1 KB]
+  const uint8_t* k_sf;  // [BH][KT][1 KB]
+  const uint8_t* v_sf;  // [BH][KT][1 KB]
+  float* o;             // [BH][Nq][128]
+  float* lse;           // [BH][Nq]
+  float* s_out;         // optional [BH][Nq][Nkv] scores (check of the block-scaled GEMM)
+  int Nq, Nkv, n_qt, Tc, RTq, KT;
+  int causal, p_mode;
+  float sl2;
+  unsigned long long timeout_ns;
+};
+
+// kind::mxf4nvf4 instruction descriptor: A = B = e2m1 (1), K-major, scale
+// factors ue4m3 (0), K = 64 per MMA.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+struct FwdF4Cfg {
+  static constexpr int TILE = 128 * 64;  // 128 rows x 64 bytes of codes
+  static constexpr int SF = 1024;
+  static constexpr int SLOTB = 10240;    // codes + scales, 1 KB aligned
+  static constexpr int NSLOT = 16;      // also keeps one CTA per SM (TMEM)
+  static constexpr int Q_OFF = 0;
+  static constexpr int QSF_OFF = TILE;
+  static constexpr int SLOT_OFF = 10240;
+  static constexpr int P_OFF = SLOT_OFF + NSLOT * SLOTB;
+  static constexpr int PSF_OFF = P_OFF + 2 * TILE;
+  static constexpr int BAR_OFF = PSF_OFF + 2 * SF;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t ID = idesc_nvf4(128, 128);
+  // TMEM columns of the scale factors (8 columns = 2 MMA steps x 4)
+  static constexpr uint32_t T_SFQ = 384, T_SFK = 392, T_SFV = 408, T_SFP = 424;
+};
+
+struct FwdF4Bars {
+  uint64_t q_full;
+  uint64_t kv_full[16];
+  uint64_t kv_empty[16];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t o_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(FwdF4Bars) <= 512, "barrier block too large");
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// shared-memory descriptor with an explicit layout (0: no swizzle, 4: 64-byte swizzle)
+__device__ __forceinline__ uint64_t smem_desc_l(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+// 32 rows x 16 bytes of shared memory -> TMEM, replicated to all 4 lane quarters
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+// two e2m1 codes (one byte) -> f16x2 values
+__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+  return r;
+}
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float f16x2_sum(uint32_t v) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(v));
+  return lo + hi;
+}
+
+template <bool SCORES_ONLY>
+__global__ void __launch_bounds__(192, 1)
+    fwd_fp4_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdF4Params p) {
+  using C = FwdF4Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FwdF4Bars* bars = reinterpret_cast<FwdF4Bars*>(smem + C::BAR_OFF);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int BH = gridDim.x / p.n_qt;
+  const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qt);
+  const int qt = p.causal ? p.n_qt - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qt);
+  const int r0 = qt * 128;
+  const int n = fwd_tile_kv_count(r0, p.Nq, p.Nkv, p.Tc, p.causal);
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full[0]), 1);
+    mbar_init(smem_u32(&bars->s_full[1]), 1);
+    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->pv_done), 1);
+    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tmem_base;
+  auto kidx = [&](int j) { return SCORES_ONLY ? j : 2 * j; };
+  auto vidx = [&](int j) { return 2 * j + 1; };
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      if (!SCORES_ONLY) prefetch_tmap(&tmV);
+      const uint32_t qbar = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qbar, C::TILE + C::SF);
+      tma_load_3d(sbase + C::Q_OFF, &tmQ, qbar, 0, r0, bh);
+      bulk_load(sbase + C::QSF_OFF, p.q_sf + ((size_t)bh * p.RTq + qt) * C::SF, C::SF, qbar);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        for (int w = 0; w < (SCORES_ONLY ? 1 : 2) && ok; ++w, ++it) {
+          const int slot = it % C::NSLOT;
+          ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ((it / C::NSLOT) & 1) ^ 1, abort_flag, p.timeout_ns);
+          if (!ok) break;
+          const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+          const uint32_t dst = sbase + C::SLOT_OFF + slot * C::SLOTB;
+          mbar_arrive_expect_tx(fb, C::TILE + C::SF);
+          if (w == 0) {
+            tma_load_3d(dst, &tmK, fb, 0, j * 128, bh);
+            bulk_load(dst + C::TILE, p.k_sf + ((size_t)bh * p.KT + j) * C::SF, C::SF, fb);
+          } else {
+            tma_load_3d(dst, &tmV, fb, j * 64, 0, bh);
+            bulk_load(dst + C::TILE, p.v_sf + ((size_t)bh * p.KT + j) * C::SF, C::SF, fb);
+          }
+        }
+      }
+      if (!ok) {
+        wait_bar_drain(qbar, 0, p.timeout_ns);
+        for (int back = 1; back <= C::NSLOT && it - back >= 0; ++back) {
+          const int i2 = it - back;
+          wait_bar_drain(smem_u32(&bars->kv_full[i2 % C::NSLOT]), (i2 / C::NSLOT) & 1, p.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
+      tc_fence_after();
+      const uint64_t dQ = smem_desc_l(sbase + C::Q_OFF, 16, 512, 4);
+      const uint64_t dSlot0 = smem_desc_l(sbase + C::SLOT_OFF, 16, 512, 4);
+      const uint64_t dSf0 = smem_desc_l(sbase + C::SLOT_OFF + C::TILE, 16, 128, 0);
+      const uint64_t dP0 = smem_desc_l(sbase + C::P_OFF, 16, 512, 4);
+      const uint64_t dPsf0 = smem_desc_l(sbase + C::PSF_OFF, 16, 128, 0);
+      if (ok) {
+        const uint64_t dQsf = smem_desc_l(sbase + C::QSF_OFF, 16, 128, 0);
+        tc_cp_sf(tbase + C::T_SFQ, dQsf);
+        tc_cp_sf(tbase + C::T_SFQ + 4, dQsf + (512 >> 4));
+      }
+      auto issue_S = [&](int j) -> bool {
+        const int it = kidx(j), s = it % C::NSLOT;
+        if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)(s * (C::SLOTB >> 4));
+        const uint32_t sfk = tbase + C::T_SFK + (j & 1) * 8;
+        tc_cp_sf(sfk, dSf0 + so);
+        tc_cp_sf(sfk + 4, dSf0 + so + (512 >> 4));
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)  // K = 64 e2m1 (32 bytes) per MMA
+          mma_nvf4(tbase + (j & 1) * 128, dQ + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID,
+                   tbase + C::T_SFQ + ks * 4, sfk + ks * 4, ks > 0);
+        tc_commit(smem_u32(&bars->s_full[j & 1]));
+        tc_commit(smem_u32(&bars->kv_empty[s]));
+        return true;
+      };
+      if (ok && n == 0) tc_commit(smem_u32(&bars->o_full));
+      if (ok && n > 0) ok = issue_S(0);
+      if (ok && n > 1) ok = issue_S(1);
+      for (int j = 0; j < n && ok && !SCORES_ONLY; ++j) {
+        const int it = vidx(j), s = it % C::NSLOT;
+        ok = wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        ok = wait_bar(smem_u32(&bars->p_full), j & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)(s * (C::SLOTB >> 4));
+        const uint32_t sfv = tbase + C::T_SFV + (j & 1) * 8, sfp = tbase + C::T_SFP + (j & 1) * 8;
+        const uint64_t po = (uint64_t)((j & 1) * (C::TILE >> 4)), pso = (uint64_t)((j & 1) * (C::SF >> 4));
+        tc_cp_sf(sfv, dSf0 + so);
+        tc_cp_sf(sfv + 4, dSf0 + so + (512 >> 4));
+        tc_cp_sf(sfp, dPsf0 + pso);
+        tc_cp_sf(sfp + 4, dPsf0 + pso + (512 >> 4));
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_nvf4(tbase + 256, dP0 + po + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID, sfp + ks * 4,
+                   sfv + ks * 4, (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bars->pv_done));
+        tc_commit(smem_u32(&bars->kv_empty[s]));
+        if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
+        if (j + 2 < n) ok = issue_S(j + 2);
+      }
+      if (SCORES_ONLY) {
+        for (int j = 2; j < n && ok; ++j) {
+          ok = wait_bar(smem_u32(&bars->p_full), (j - 2) & 1, abort_flag, p.timeout_ns);
+          if (ok) ok = issue_S(j);
+        }
+      }
+      if (!ok) {
+        tc_commit(smem_u32(&bars->drain));
+        wait_bar_drain(smem_u32(&bars->drain), 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax
+    const int quarter = warp & 3;
+    const int rr = quarter * 32 + lane;
+    const int row = r0 + rr;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tO = tbase + lane_off + 256;
+    const int off = p.Nkv - p.Nq;
+    const float sl2 = p.sl2;
+    const bool direct = p.p_mode == 0;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    if (!SCORES_ONLY && direct) {
+      // Direct-P: every P block scale is 1.0 (0x38); both buffers, written once
+      for (int i = threadIdx.x - 64; i < 2 * C::SF / 4; i += 128)
+        *reinterpret_cast<uint32_t*>(smem + C::PSF_OFF + i * 4) = 0x38383838u;
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int kb = j * 128;
+      ok = wait_bar(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tbase + lane_off + (j & 1) * 128;
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      if (SCORES_ONLY) {
+        if (row < p.Nq) {
+          float* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (kb + c * 32 + i < p.Nkv) dst[c * 32 + i] = __uint_as_float(s[c][i]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->p_full));
+        continue;
+      }
+      const bool tail = kb + 128 > p.Nkv;
+      const bool diag = p.causal && (kb + 127 > r0 + off);
+      if (tail || diag) {
+        int lim = p.Nkv - 1 - kb;
+        if (p.causal) lim = min(lim, row + off - kb);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim) s[c][i] = 0xFF800000u;
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        mx0 = fmax3(mx0, __uint_as_float(s[0][i]), __uint_as_float(s[0][i + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(s[1][i]), __uint_as_float(s[1][i + 1]));
+        mx2 = fmax3(mx2, __uint_as_float(s[2][i]), __uint_as_float(s[2][i + 1]));
+        mx3 = fmax3(mx3, __uint_as_float(s[3][i]), __uint_as_float(s[3][i + 1]));
+      }
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const bool grow = m_blk > m_ref;  // the reference moves on every increase
+      const bool had = m_ref != -INFINITY;
+      float factor = 1.f;
+      if (grow) {
+        factor = had ? ex2(m_ref - m_blk) : 0.f;
+        l *= factor;
+        m_ref = m_blk;
+      }
+      const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      // ---- P codes (row rr of the P tile, 64 bytes, 64-byte swizzle) and scales
+      uint8_t* ptile = smem + C::P_OFF + (j & 1) * C::TILE + rr * 64;
+      uint8_t* psf = smem + C::PSF_OFF + (j & 1) * C::SF;
+      float lsum = 0.f;
+#pragma unroll
+      for (int blk = 0; blk < 8; ++blk) {  // 16 keys per block
+        const int c = blk >> 1, i0 = (blk & 1) * 16;
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = ex2(fmaf(__uint_as_float(s[c][i0 + e]), sl2, negm));
+        float sc = 1.f;
+        if (!direct) {
+          float amax = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, v[e]);
+          const uint32_t sfc = (amax > 0.f) ? e4m3_rne(__fdiv_rn(fmaxf(amax, 1e-30f), 6.f)) : 0u;
+          sc = e4m3_value(sfc);
+          psf[sf_offset(rr, blk)] = (uint8_t)sfc;
+          // a zero scale (an all-zero block) gives zero codes; the divisor is
+          // kept nonzero so that no element takes the IEEE divide's slow path
+          // codes from p * (1 / sf): within an ulp of p / sf, so only a value
+          // on an e2m1 rounding boundary can round differently; a zero scale
+          // (an all-zero block) gives zero codes
+          const float r = (sc > 0.f) ? __frcp_rn(sc) : 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] *= r;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] *= 6.f;
+        }
+        uint32_t w[2] = {0u, 0u};
+        uint32_t hs = 0u;  // f16x2 running sum of the decoded codes
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const uint32_t b = e2m1x2(v[e], v[e + 1]);
+          w[e >> 3] |= b << (8 * ((e >> 1) & 3));
+          hs = hadd2(hs, e2m1x2_f16x2(b));
+        }
+        lsum += f16x2_sum(hs) * sc;  // l sums the P values the MMA multiplies into V
+        // 8 bytes = keys [16 blk, 16 blk + 16) -> chunk blk / 2, half blk % 2
+        const int chunk = blk >> 1;
+        uint8_t* dst = ptile + ((chunk ^ ((rr >> 1) & 3)) << 4) + (blk & 1) * 8;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+      }
+      l += lsum;
+      if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
+        // rescale O (P V of blocks < j) to the new reference
+        ok = wait_bar(smem_u32(&bars->pv_done), (j - 1) & 1, abort_flag, p.timeout_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float f = (grow && had) ? factor : 1.f;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+          tmem_st32(tO + cc * 32, o);
+        }
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();  // P tile and scales are read by the tensor core
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->p_full));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (!SCORES_ONLY && ok) {
+      ok = wait_bar(smem_u32(&bars->o_full), 0, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        float* orow = p.o + ((size_t)bh * p.Nq + row) * 128;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+          if (row < p.Nq) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 v;
+              v.x = (l > 0.f) ? __uint_as_float(o[i + 0]) * inv : 0.f;
+              v.y = (l > 0.f) ? __uint_as_float(o[i + 1]) * inv : 0.f;
+              v.z = (l > 0.f) ? __uint_as_float(o[i + 2]) * inv : 0.f;
+              v.w = (l > 0.f) ? __uint_as_float(o[i + 3]) * inv : 0.f;
+              *reinterpret_cast<float4*>(orow + cc * 32 + i) = v;
+            }
+          }
+        }
+        if (row < p.Nq)
+          // Direct-P values are 6 * 2^(x - m): LSE = m + log2(l / 6)
+          p.lse[(size_t)bh * p.Nq + row] =
+              (l > 0.f) ? (m_ref + log2f(l) - (direct ? 2.5849625007211562f : 0.f)) * 0.69314718055994531f
+                        : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace ta

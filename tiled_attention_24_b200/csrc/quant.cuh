@@ -118,4 +118,110 @@ __global__ void head_scale_kernel(unsigned* amax_bits, int n) {
   amax_bits[i] = __float_as_uint(s);
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 ("Hardware-Aware FP4 FlashAttention-4" page: FP4 operands): blocks of
+// 16 elements, e2m1 codes (RNE, saturating at +-6) scaled by one unsigned
+// e4m3 factor per block, sf = e4m3_rne(amax / 6), code = e2m1_rne(x / sf),
+// both divides IEEE fp32.  Negative values that round to zero keep code 0.
+//
+// Scale factors are stored in the layout the tensor core reads them in: per
+// 128-row tile and per group of 4 consecutive blocks (one 64-element MMA
+// step), 512 bytes with byte (r % 32) * 16 + (r / 32) * 4 + block % 4 for row
+// r of the tile; a 128 x 128 tile has two such groups (1 KB).
+// mode 0 (Q, K): blocks along d, codes [BH][N][64 B], sf [BH][ceil(N/128)][1 KB]
+// mode 1 (V):    blocks along tokens, written transposed: codes [BH][128][KT*64 B]
+//                and sf [BH][KT][1 KB] with KT = ceil(N/128); rows = channels.
+// Rows / tokens past N are zero (codes 0, scale 0).
+
+__device__ __forceinline__ uint32_t e4m3_rne(float v) {  // v >= 0, saturating
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(v));
+  return r & 0xFFu;
+}
+__device__ __forceinline__ float e4m3_value(uint32_t c) {  // from the format definition
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0x1p-9f;
+}
+// two fp32 -> e2m1 codes, `lo` in the low nibble; negative zero -> code 0
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  if ((r & 0xFu) == 8u) r &= 0xF0u;
+  if ((r >> 4) == 8u) r &= 0x0Fu;
+  return r;
+}
+__device__ __forceinline__ uint32_t sf_offset(int r, int blk) {  // within a 1 KB tile
+  return (uint32_t)((blk >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (blk & 3));
+}
+// quantise 16 values; returns the scale code, fills 8 code bytes
+__device__ __forceinline__ uint32_t nvfp4_block(const float (&v)[16], uint32_t (&out)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sfc = e4m3_rne(__fdiv_rn(amax, 6.f));
+  const float s = e4m3_value(sfc);
+  out[0] = out[1] = 0u;
+  if (s > 0.f) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const uint32_t b = e2m1x2(__fdiv_rn(v[i], s), __fdiv_rn(v[i + 1], s));
+      out[i >> 3] |= b << (8 * ((i >> 1) & 3));
+    }
+  }
+  return sfc;
+}
+
+// mode 0: one thread per (bh, padded row, block of 16 along d = 128)
+__global__ void __launch_bounds__(256) quant_nvfp4_rows_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf, int N, int RT, long long total) {
+  const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (i >= total) return;
+  const int blk = (int)(i & 7);
+  const long long rowg = i >> 3;              // bh * RT*128 + row
+  const int row = (int)(rowg % (RT * 128));
+  const long long bh = rowg / (RT * 128);
+  float v[16];
+  if (row < N) {
+    const uint16_t* src = x + ((bh * N + row) * 128 + blk * 16);
+    const uint4 w0 = *reinterpret_cast<const uint4*>(src), w1 = *reinterpret_cast<const uint4*>(src + 8);
+    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v[2 * e] = __uint_as_float(ws[e] << 16);
+      v[2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = 0.f;
+  }
+  uint32_t out[2];
+  const uint32_t sfc = nvfp4_block(v, out);
+  if (row < N) *reinterpret_cast<uint2*>(codes + (bh * N + row) * 64 + blk * 8) = make_uint2(out[0], out[1]);
+  sf[((bh * RT + row / 128) * 1024) + sf_offset(row & 127, blk)] = (uint8_t)sfc;
+}
+
+// mode 1: one thread per (bh, token block of 16, channel); consecutive threads
+// take consecutive channels so the loads are coalesced
+__global__ void __launch_bounds__(256) quant_nvfp4_cols_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf, int N, int KT, long long total) {
+  const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (i >= total) return;
+  const int c = (int)(i & 127);
+  const long long rest = i >> 7;
+  const int tb = (int)(rest % (KT * 8));
+  const long long bh = rest / (KT * 8);
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int tok = tb * 16 + e;
+    v[e] = (tok < N) ? __uint_as_float((uint32_t)x[(bh * N + tok) * 128 + c] << 16) : 0.f;
+  }
+  uint32_t out[2];
+  const uint32_t sfc = nvfp4_block(v, out);
+  *reinterpret_cast<uint2*>(codes + (bh * 128 + c) * (long long)(KT * 64) + tb * 8) = make_uint2(out[0], out[1]);
+  sf[((bh * KT + tb / 8) * 1024) + sf_offset(c, tb & 7)] = (uint8_t)sfc;
+}
+
 }  // namespace ta
