@@ -7,11 +7,16 @@ A step is one pass of the hot path over the seeded synthetic workloads:
              (the headline: attention forward TFLOP/s, 4*B*H*N*N*d, halved
              for causal);
   * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine
-             (KV-read GB/s against HBM).
+             (KV-read GB/s against HBM);
+  * longseq  B=1 H=12 N=23400 d=64 bf16, non-causal + causal;
+  * lowp     B=2 H=24 N=8192 d=128 with outlier channels: bf16 forward, INT8
+             quantisers + INT8 forward, NVFP4 quantisers + FP4 forward with
+             Direct-P and with quantise-after-exp.
 Inputs are resident in HBM before timing starts and are larger than the
 126 MB L2 (prefill Q+K+V = 201 MB, decode K+V = 8.6 GB), so no L2 flush is
 needed between steps.  Every launch is bracketed by CUDA events on the
-launching stream; `value` is prefill FLOPs / summed prefill kernel time.
+launching stream; `value` is prefill FLOPs / summed prefill kernel time and
+`parts` gives every segment's rate against its roofline.
 
 `e2e` measures the same metric through the public API with host buffers:
 each step copies Q, K, V from pinned host memory, runs both forwards and
@@ -205,41 +210,99 @@ def run_ours(args):
     ta.load()
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
-
-    # ---- inputs, resident in HBM
-    wp = WORKLOADS["prefill"]
-    q, k, v = (t.to(dev) for t in make_qkv(wp, seed=0))
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-    wd = WORKLOADS["decode"]
     parts = set(args.only.split(","))
-    dq, dk, dv = make_qkv(wd, seed=0, device=dev, B=args.decode_batch or wd.B)
-    do = torch.empty_like(dq)
-    dlse = torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
-    dws = torch.empty(ta.attn_decode_workspace_bytes(dq.shape[0], wd.H, wd.d, wd.num_splits),
-                      dtype=torch.uint8, device=dev)
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # dense INT8 / FP4 peaks are not in the measured set: nominal (4.5 POPS,
+    # 9 PFLOPS) scaled by measured/nominal bf16 (1683 / 2250), labelled as such
+    ratio = peak_tc / 2250.0
+    peak_i8 = float(peaks.get("int8_tops", 4500.0 * ratio))
+    peak_f4 = float(peaks.get("fp4_tflops", 9000.0 * ratio))
+    lowp_peak_src = "measured" if "int8_tops" in peaks else "nominal x (measured/nominal bf16)"
 
-    flops_nc, flops_c = wp.flops(False), wp.flops(True)
-    kv_bytes = 2 * dk.numel() * dk.element_size()
+    segs = []   # (name, fn, work, unit, peak, bound, launches)
+
+    def seg(name, fn, work, unit, peak, bound, launches):
+        segs.append((name, fn, work, unit, peak, bound, launches))
+
+    # ---- inputs, resident in HBM (all larger than the 126 MB L2 except as noted)
+    wp = WORKLOADS["prefill"]
+    if "prefill" in parts:
+        q, k, v = (t.to(dev) for t in make_qkv(wp, seed=0))
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        seg("prefill_noncausal", lambda: ta.attn_fwd(q, k, v, o, lse, False, wp.scale, stream),
+            wp.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
+        seg("prefill_causal", lambda: ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream),
+            wp.flops(True), "TFLOP/s", peak_tc, "tensor", 1)
+    wd = WORKLOADS["decode"]
+    if "decode" in parts:
+        dq, dk, dv = make_qkv(wd, seed=0, device=dev, B=args.decode_batch or wd.B)
+        do = torch.empty_like(dq)
+        dlse = torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
+        dws = torch.empty(ta.attn_decode_workspace_bytes(dq.shape[0], wd.H, wd.d, wd.num_splits),
+                          dtype=torch.uint8, device=dev)
+        seg("decode", lambda: ta.attn_decode(dq, dk, dv, do, dlse, wd.scale, wd.num_splits, dws, stream),
+            2 * dk.numel() * dk.element_size(), "GB/s", peak_hbm, "hbm", 2)
+    wl = WORKLOADS["longseq"]
+    if "longseq" in parts:
+        lq, lk, lv = (t.to(dev) for t in make_qkv(wl, seed=0))
+        lo = torch.empty_like(lq)
+        llse = torch.empty(lq.shape[:3], dtype=torch.float32, device=dev)
+        seg("longseq_noncausal", lambda: ta.attn_fwd(lq, lk, lv, lo, llse, False, wl.scale, stream),
+            wl.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
+        seg("longseq_causal", lambda: ta.attn_fwd(lq, lk, lv, lo, llse, True, wl.scale, stream),
+            wl.flops(True), "TFLOP/s", peak_tc, "tensor", 1)
+    wq = WORKLOADS["lowp"]
+    if "lowp" in parts:
+        xq, xk, xv = (t.to(dev) for t in make_qkv(wq, seed=0))
+        B5, H5, N5, D5 = xq.shape
+        xo = torch.empty_like(xq)
+        xl = torch.empty((B5, H5, N5), dtype=torch.float32, device=dev)
+        seg("lowp_bf16", lambda: ta.attn_fwd(xq, xk, xv, xo, xl, False, wq.scale, stream),
+            wq.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
+        i8 = [torch.empty(t.shape, dtype=torch.int8, device=dev) for t in (xq, xk, xv)]
+        s8 = [torch.empty((B5, H5, N5), dtype=torch.float32, device=dev) for _ in range(2)]
+        s8.append(torch.empty((B5, H5), dtype=torch.float32, device=dev))
+        of = torch.empty((B5, H5, N5, D5), dtype=torch.float32, device=dev)
+        lf = torch.empty((B5, H5, N5), dtype=torch.float32, device=dev)
+
+        def q8():
+            ta.attn_quantize_int8(xq, i8[0], s8[0], False, stream)
+            ta.attn_quantize_int8(xk, i8[1], s8[1], False, stream)
+            ta.attn_quantize_int8(xv, i8[2], s8[2], True, stream)
+        seg("lowp_int8_quantise", q8, 3 * xq.numel() * 2 + 3 * xq.numel(), "GB/s", peak_hbm, "hbm", 5)
+        seg("lowp_int8", lambda: ta.attn_fwd_int8(i8[0], s8[0], i8[1], s8[1], i8[2], s8[2], of, lf, False,
+                                                  wq.scale, stream),
+            wq.flops(False), "TOPS", peak_i8, "tensor", 1)
+        c4 = [torch.empty(ta.attn_nvfp4_codes_bytes(B5, H5, N5, D5, m), dtype=torch.uint8, device=dev)
+              for m in (0, 0, 1)]
+        f4 = [torch.empty(ta.attn_nvfp4_sf_bytes(B5, H5, N5, D5, m), dtype=torch.uint8, device=dev)
+              for m in (0, 0, 1)]
+
+        def q4():
+            for t, c, f, m in zip((xq, xk, xv), c4, f4, (0, 0, 1)):
+                ta.attn_quantize_nvfp4(t, c, f, m, stream)
+        seg("lowp_fp4_quantise", q4, 3 * xq.numel() * 2 + sum(c.numel() for c in c4), "GB/s", peak_hbm, "hbm", 3)
+        for mode, nm in ((0, "lowp_fp4_direct_p"), (1, "lowp_fp4_quant_after_exp")):
+            seg(nm, (lambda mode=mode: ta.attn_fwd_fp4(c4[0], f4[0], c4[1], f4[1], c4[2], f4[2], of, lf, B5, H5,
+                                                        N5, N5, False, wq.scale, mode, stream)),
+                wq.flops(False), "TFLOP/s", peak_f4, "tensor", 1)
+
+    nseg = len(segs)
 
     def step(ev):
         ev[0].record(stream)
-        if "prefill" in parts:
-            ta.attn_fwd(q, k, v, o, lse, False, wp.scale, stream)
-        ev[1].record(stream)
-        if "prefill" in parts:
-            ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream)
-        ev[2].record(stream)
-        if "decode" in parts:
-            ta.attn_decode(dq, dk, dv, do, dlse, wd.scale, wd.num_splits, dws, stream)
-        ev[3].record(stream)
+        for i, sg in enumerate(segs):
+            sg[1]()
+            ev[i + 1].record(stream)
 
     def barrier():
         if ws > 1:
             import torch.distributed as dist
             dist.barrier()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nseg + 1)] for _ in range(args.steps)]
     for _ in range(args.warmup):
         step(evs[0])
     torch.cuda.synchronize()
@@ -264,31 +327,30 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device watchdog status {status}")
 
-    total_ms = t_start.elapsed_time(t_end)
-    nc_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    c_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms, nc_tot, c_tot, dec_tot = max_over_ranks([total_ms, sum(nc_ms), sum(c_ms), sum(dec_ms)], dev)
+    sums = [t_start.elapsed_time(t_end)] + [sum(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nseg)]
+    sums = max_over_ranks(sums, dev)
+    total_ms, seg_ms = sums[0], sums[1:]
+    out_parts = {}
+    for (name, _, work, unit, peak, bound, _l), ms in zip(segs, seg_ms):
+        avg = ms / args.steps
+        scale = 1e12 if unit in ("TFLOP/s", "TOPS") else 1e9
+        rate = work / (avg * 1e-3) / scale
+        out_parts[name] = {"ms": avg, "rate": rate, "unit": unit, "bound": bound, "peak": peak,
+                           "frac": rate / peak}
+    pre = [i for i, sg in enumerate(segs) if sg[0].startswith("prefill_")]
+    if pre:
+        value = job_throughput(ws, args.steps, sum(segs[i][2] for i in pre), sum(seg_ms[i] for i in pre)) / 1e12
+    else:
+        value = None
 
-    prefill_ms = nc_tot + c_tot
-    value = job_throughput(ws, args.steps, flops_nc + flops_c, prefill_ms) / 1e12
-    nc_avg = nc_tot / args.steps
-    c_avg = c_tot / args.steps
-    dec_avg = dec_tot / args.steps
-    tflops_nc = flops_nc / (nc_avg * 1e-3) / 1e12
-    tflops_c = flops_c / (c_avg * 1e-3) / 1e12
-    dec_gbs = kv_bytes / (dec_avg * 1e-3) / 1e9
-    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers (prefill)
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and "prefill" in parts:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        ho2 = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         hl2 = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        ho2 = torch.empty(o.shape, dtype=o.dtype).pin_memory()
 
         def e2e_step():
             q.copy_(hq, non_blocking=True)
@@ -314,8 +376,8 @@ def run_ours(args):
         e_ms = max_over_ranks([a.elapsed_time(b)], dev)[0]
         h2d = 3 * q.numel() * q.element_size()
         d2h = 2 * (o.numel() * o.element_size() + lse.numel() * lse.element_size())
-        e2e = {"value": job_throughput(ws, args.e2e_steps, flops_nc + flops_c, e_ms) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        e2e = {"value": job_throughput(ws, args.e2e_steps, wp.flops(False) + wp.flops(True), e_ms) / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps}
 
     cpu = None
@@ -323,8 +385,19 @@ def run_ours(args):
         cv, desc, thr, _ = oracle_sample(args.cpu_seconds)
         cpu = {"value": cv, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc}
 
-    gpu_launches = args.steps * (2 * ("prefill" in parts) + 2 * ("decode" in parts))
     traffic = load_traffic()
+    pn = out_parts.get("prefill_noncausal")
+    roof = None
+    if pn:
+        roof = {"bound": "tensor", "achieved": pn["rate"], "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": pn["rate"] / peak_tc, "traffic": traffic.get("fwd_bf16_prefill_noncausal"),
+                "kernel": "fwd_bf16_kernel<128>, prefill B4 H16 N4096 d128 non-causal",
+                "peak_source": f"{peak_src} bf16 burst"}
+    if "decode" in out_parts:
+        out_parts["decode"]["traffic"] = traffic.get("decode_split")
+    for nm in ("lowp_int8", "lowp_fp4_direct_p", "lowp_fp4_quant_after_exp"):
+        if nm in out_parts:
+            out_parts[nm]["peak_source"] = lowp_peak_src
     line = {
         "metric": "attn fwd TFLOP/s (prefill B4 H16 N4096 d128, non-causal + causal)",
         "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -332,22 +405,13 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, resident in HBM)",
         "config": {"workload": "prefill", "B": wp.B, "H": wp.H, "Nq": wp.Nq, "Nkv": wp.Nkv, "d": wp.d,
                    "causal": ["false", "true"], "parallelism": f"replicas x{ws}",
-                   "l2": "inputs (201 MB) larger than L2 (126 MB); no flush"},
-        "prefill": {"noncausal_tflops": tflops_nc, "causal_tflops": tflops_c,
-                    "noncausal_ms": nc_avg, "causal_ms": c_avg,
-                    "frac_of_peak_noncausal": tflops_nc / peak_tc, "frac_of_peak_causal": tflops_c / peak_tc},
-        "decode": None if "decode" not in parts else {
-                   "workload": f"decode B{dq.shape[0]} H32 Nkv8192 d128 splits16", "ms": dec_avg, "kv_gbs": dec_gbs,
-                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peak_hbm, "unit": "GB/s",
-                                "frac": dec_gbs / peak_hbm, "traffic": traffic.get("decode_split"),
-                                "peak_source": peak_src}},
-        "roofline": {"bound": "tensor", "achieved": tflops_nc, "peak": peak_tc, "unit": "TFLOP/s",
-                     "frac": tflops_nc / peak_tc, "traffic": traffic.get("fwd_bf16"),
-                     "kernel": "fwd_bf16_kernel<128> non-causal prefill",
-                     "peak_source": f"{peak_src} bf16 burst"},
+                   "l2": "every input larger than L2 (126 MB) except the int8/fp4 operands; no flush",
+                   "step": sorted(out_parts)},
+        "roofline": roof,
+        "parts": out_parts,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": gpu_launches,
+        "gpu_launches": args.steps * sum(sg[6] for sg in segs),
         "clocks": clk,
     }
     if rank == 0:
@@ -378,8 +442,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,decode",
-                    help="comma list of step parts to run (prefill, decode); profiling aid")
+    ap.add_argument("--only", default="prefill,decode,longseq,lowp",
+                    help="comma list of step parts to run (prefill, decode, longseq, lowp); profiling aid")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="decode batch override (profiling aid; 0 = the workload's 64)")
     args = ap.parse_args()
