@@ -38,6 +38,9 @@
 #ifndef TA_POLY_PAIRS
 #define TA_POLY_PAIRS 0
 #endif
+#ifndef TA_POLY_PAIRS_D64
+#define TA_POLY_PAIRS_D64 TA_POLY_PAIRS
+#endif
 
 namespace ta {
 
@@ -68,7 +71,7 @@ struct FwdCfg {
   static constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
   static constexpr float TAU = 8.0f;  // lazy-rescale threshold, log2 units
   // of every POLY_PERIOD element pairs, POLY_PAIRS take 2^x from the cubic
-  static constexpr int POLY_PERIOD = TA_POLY_PERIOD, POLY_PAIRS = TA_POLY_PAIRS;
+  static constexpr int POLY_PERIOD = TA_POLY_PERIOD, POLY_PAIRS = (D == 64) ? TA_POLY_PAIRS_D64 : TA_POLY_PAIRS;
 };
 
 struct FwdBars {

@@ -57,7 +57,8 @@ struct FwdI8Cfg {
   static constexpr int NSLOT = 8;
   static constexpr int Q_OFF = 0;
   static constexpr int SLOT_OFF = TILE;
-  static constexpr int BAR_OFF = SLOT_OFF + NSLOT * TILE;
+  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;  // [4 warps][2 bufs][128] floats
+  static constexpr int BAR_OFF = KC_OFF + 4 * 2 * 128 * 4;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
   static constexpr int THREADS = 192;
   static constexpr uint32_t ID_S = idesc_i8(128, false);
@@ -239,9 +240,36 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tACC = tbase + lane_off + 256;
     const uint32_t tOF = tbase + lane_off + 384;
     const int off = p.Nkv - p.Nq;
-    const float crow = (!SCORES_ONLY && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] * p.sl2 : 0.f;
+    const float qs_row = (!SCORES_ONLY && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] : 0.f;
     const float sv127 = SCORES_ONLY ? 0.f : p.v_scale[bh] * (1.f / 127.f);
     const float* ksrow = p.k_scale + (size_t)bh * p.Nkv;
+    // Per-column constants of a key block, kc = s_K * scale * log2(e), kept in
+    // this warp's own shared buffer (x / s_Q = S * kc).  Lane l owns columns
+    // [4l, 4l + 4); the next block's scales are loaded one block ahead.
+    float* kcbuf = reinterpret_cast<float*>(smem + C::KC_OFF) + (warp - 2) * (2 * 128);
+    float4 ks_next = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto load_ks = [&](int jj) {
+      const int c0 = jj * 128 + lane * 4;
+      if (p.ks_vec && c0 + 3 < p.Nkv) {
+        ks_next = __ldg(reinterpret_cast<const float4*>(ksrow + c0));
+      } else {
+        ks_next.x = (c0 + 0 < p.Nkv) ? ksrow[c0 + 0] : 0.f;
+        ks_next.y = (c0 + 1 < p.Nkv) ? ksrow[c0 + 1] : 0.f;
+        ks_next.z = (c0 + 2 < p.Nkv) ? ksrow[c0 + 2] : 0.f;
+        ks_next.w = (c0 + 3 < p.Nkv) ? ksrow[c0 + 3] : 0.f;
+      }
+    };
+    auto stage_ks = [&](int jj) {
+      float* kcb = kcbuf + (jj & 1) * 128;
+      *reinterpret_cast<float4*>(kcb + lane * 4) =
+          make_float4(ks_next.x * p.sl2, ks_next.y * p.sl2, ks_next.z * p.sl2, ks_next.w * p.sl2);
+    };
+    if (!SCORES_ONLY && n > 0) {
+      load_ks(0);
+      stage_ks(0);
+      if (n > 1) load_ks(1);
+      __syncwarp();
+    }
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     if (!SCORES_ONLY) {
@@ -277,7 +305,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(smem_u32(&bars->p_full));
         continue;
       }
-      // x = S * s_Q * s_K * scale * log2e, masked
+      // y = S * s_K * scale * log2e (= x / s_Q), masked; x = y * s_Q
       const bool tail = kb + 128 > p.Nkv;
       const bool diag = p.causal && (kb + 127 > r0 + off);
       int lim = 127;
@@ -285,26 +313,35 @@ __global__ void __launch_bounds__(192, 1)
         lim = p.Nkv - 1 - kb;
         if (p.causal) lim = min(lim, row + off - kb);
       }
+      const float* kcb = kcbuf + (j & 1) * 128;
       float x[4][32];
+      const uint64_t negM2 = f2(-12582912.f, -12582912.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const int col = c * 32 + i;
-          float4 ks;
-          if (!tail && p.ks_vec) {
-            ks = __ldg(reinterpret_cast<const float4*>(ksrow + kb + col));
-          } else {
-            ks.x = (kb + col + 0 < p.Nkv) ? ksrow[kb + col + 0] : 0.f;  // scalar path
-            ks.y = (kb + col + 1 < p.Nkv) ? ksrow[kb + col + 1] : 0.f;
-            ks.z = (kb + col + 2 < p.Nkv) ? ksrow[kb + col + 2] : 0.f;
-            ks.w = (kb + col + 3 < p.Nkv) ? ksrow[kb + col + 3] : 0.f;
-          }
-          x[c][i + 0] = (col + 0 <= lim) ? i2f_small(s[c][i + 0]) * (ks.x * crow) : -INFINITY;
-          x[c][i + 1] = (col + 1 <= lim) ? i2f_small(s[c][i + 1]) * (ks.y * crow) : -INFINITY;
-          x[c][i + 2] = (col + 2 <= lim) ? i2f_small(s[c][i + 2]) * (ks.z * crow) : -INFINITY;
-          x[c][i + 3] = (col + 3 <= lim) ? i2f_small(s[c][i + 3]) * (ks.w * crow) : -INFINITY;
+          const float4 kc = *reinterpret_cast<const float4*>(kcb + col);
+          // exact int32 -> fp32 (|S| < 2^22): bits of 1.5 * 2^23 + S, minus 1.5 * 2^23
+          const uint64_t sa = fadd2(f2(__int_as_float((int)s[c][i + 0] + 0x4B400000),
+                                       __int_as_float((int)s[c][i + 1] + 0x4B400000)), negM2);
+          const uint64_t sb = fadd2(f2(__int_as_float((int)s[c][i + 2] + 0x4B400000),
+                                       __int_as_float((int)s[c][i + 3] + 0x4B400000)), negM2);
+          f2_split(fmul2(sa, f2(kc.x, kc.y)), x[c][i + 0], x[c][i + 1]);
+          f2_split(fmul2(sb, f2(kc.z, kc.w)), x[c][i + 2], x[c][i + 3]);
         }
+      }
+      if (tail || diag) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim) x[c][i] = -INFINITY;
+      }
+      // the next block's scales go to the other buffer while this one is in use
+      if (j + 1 < n) {
+        stage_ks(j + 1);
+        if (j + 2 < n) load_ks(j + 2);
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -314,7 +351,8 @@ __global__ void __launch_bounds__(192, 1)
         mx2 = fmax3(mx2, x[2][i], x[2][i + 1]);
         mx3 = fmax3(mx3, x[3][i], x[3][i + 1]);
       }
-      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      // s_Q > 0, so max(y) * s_Q is the row max of x
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * qs_row;
       // tau = 0: move the reference on every increase
       const bool grow = m_blk > m_ref;
       const bool had = m_ref != -INFINITY;  // rows with earlier content need a fold
@@ -334,7 +372,7 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t t[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float y = ex2(x[c][i + e] + negm) * 127.f;
+            const float y = ex2(fmaf(x[c][i + e], qs_row, negm)) * 127.f;
             t[e] = __float_as_uint(y + 12582912.f);  // low bits: rne(y) in [0, 127]
             isum += t[e];
           }
@@ -370,6 +408,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tmem_st_wait();
+      __syncwarp();  // the staged scales of block j + 1 are visible to the whole warp
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full));
     }
