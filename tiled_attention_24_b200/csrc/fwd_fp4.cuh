@@ -114,6 +114,14 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
       : "memory");
 }
+// two non-negative fp32 -> e2m1 codes (one byte, `lo` in the low nibble)
+__device__ __forceinline__ uint32_t e2m1x2_pos(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
 // two e2m1 codes (one byte) -> f16x2 values
 __device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
   uint32_t r;
@@ -359,45 +367,43 @@ __global__ void __launch_bounds__(192, 1)
       uint8_t* ptile = smem + C::P_OFF + (j & 1) * C::TILE + rr * 64;
       uint8_t* psf = smem + C::PSF_OFF + (j & 1) * C::SF;
       float lsum = 0.f;
+      // Direct-P: 6 * 2^(x - m) = 2^(x - m + log2 6), one exponential per score
+      const float neg_arg = direct ? negm + 2.5849625007211562f : negm;
 #pragma unroll
       for (int blk = 0; blk < 8; ++blk) {  // 16 keys per block
         const int c = blk >> 1, i0 = (blk & 1) * 16;
         float v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = ex2(fmaf(__uint_as_float(s[c][i0 + e]), sl2, negm));
+        for (int e = 0; e < 16; ++e) v[e] = ex2(fmaf(__uint_as_float(s[c][i0 + e]), sl2, neg_arg));
         float sc = 1.f;
         if (!direct) {
-          float amax = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, v[e]);
+          float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]), a2 = fmax3(v[6], v[7], v[8]);
+          float a3 = fmax3(v[9], v[10], v[11]), a4 = fmax3(v[12], v[13], v[14]);
+          const float amax = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]), 0.f);
           const uint32_t sfc = (amax > 0.f) ? e4m3_rne(__fdiv_rn(fmaxf(amax, 1e-30f), 6.f)) : 0u;
           sc = e4m3_value(sfc);
           psf[sf_offset(rr, blk)] = (uint8_t)sfc;
-          // a zero scale (an all-zero block) gives zero codes; the divisor is
-          // kept nonzero so that no element takes the IEEE divide's slow path
           // codes from p * (1 / sf): within an ulp of p / sf, so only a value
           // on an e2m1 rounding boundary can round differently; a zero scale
           // (an all-zero block) gives zero codes
           const float r = (sc > 0.f) ? __frcp_rn(sc) : 0.f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] *= r;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] *= 6.f;
         }
-        uint32_t w[2] = {0u, 0u};
+        uint32_t b[8];
         uint32_t hs = 0u;  // f16x2 running sum of the decoded codes
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const uint32_t b = e2m1x2(v[e], v[e + 1]);
-          w[e >> 3] |= b << (8 * ((e >> 1) & 3));
-          hs = hadd2(hs, e2m1x2_f16x2(b));
+        for (int e = 0; e < 8; ++e) {
+          b[e] = e2m1x2_pos(v[2 * e], v[2 * e + 1]);
+          hs = hadd2(hs, e2m1x2_f16x2(b[e]));
         }
         lsum += f16x2_sum(hs) * sc;  // l sums the P values the MMA multiplies into V
+        const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
         // 8 bytes = keys [16 blk, 16 blk + 16) -> chunk blk / 2, half blk % 2
         const int chunk = blk >> 1;
         uint8_t* dst = ptile + ((chunk ^ ((rr >> 1) & 3)) << 4) + (blk & 1) * 8;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
       }
       l += lsum;
       if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
