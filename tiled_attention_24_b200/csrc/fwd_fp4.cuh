@@ -77,7 +77,7 @@ struct FwdF4Bars {
   uint64_t kv_full[16];
   uint64_t kv_empty[16];
   uint64_t s_full[2];
-  uint64_t p_full;
+  uint64_t p_full[2];  // per block parity: block j + 1 can be released before the MMA thread saw block j
   uint64_t pv_done;
   uint64_t o_full;
   uint64_t drain;
@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(smem_u32(&bars->s_full[0]), 1);
     mbar_init(smem_u32(&bars->s_full[1]), 1);
-    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->p_full[0]), 128);
+    mbar_init(smem_u32(&bars->p_full[1]), 128);
     mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(192, 1)
         const int it = vidx(j), s = it % C::NSLOT;
         ok = wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
-        ok = wait_bar(smem_u32(&bars->p_full), j & 1, abort_flag, p.timeout_ns);
+        ok = wait_bar(smem_u32(&bars->p_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)(s * (C::SLOTB >> 4));
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (SCORES_ONLY) {
         for (int j = 2; j < n && ok; ++j) {
-          ok = wait_bar(smem_u32(&bars->p_full), (j - 2) & 1, abort_flag, p.timeout_ns);
+          ok = wait_bar(smem_u32(&bars->p_full[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns);
           if (ok) ok = issue_S(j);
         }
       }
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(192, 1)
               if (kb + c * 32 + i < p.Nkv) dst[c * 32 + i] = __uint_as_float(s[c][i]);
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_full));
+        mbar_arrive(smem_u32(&bars->p_full[j & 1]));
         continue;
       }
       const bool tail = kb + 128 > p.Nkv;
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       fence_proxy_async_smem();  // P tile and scales are read by the tensor core
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->p_full));
+      mbar_arrive(smem_u32(&bars->p_full[j & 1]));
     }
     // ---------------------------------------------------------- epilogue
     if (!SCORES_ONLY && ok) {

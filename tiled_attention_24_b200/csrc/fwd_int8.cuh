@@ -18,10 +18,17 @@
 // O = (OF + ACC * s_V / 127) / l (fp32 output) and LSE = ln2 * (m + log2 l).
 //
 // CTA = one (batch, head) x one 128-row query tile.  Warps: 0 TMA producer,
-// 1 MMA issuer, 2-5 softmax/fold/epilogue (thread = TMEM lane = query row).
+// 1 MMA issuer, 2-9 softmax/fold/epilogue: TMEM lane quarter q is read by two
+// warps, one taking key columns [0, 64) of every block (warps 2-5), the other
+// [64, 128) (warps 6-9); the two threads of a row exchange their partial row
+// max once per block through a tagged shared-memory slot (xchg_put/get).
+// Two softmax warps per SM sub-partition give the scheduler a second
+// instruction stream while one waits on a dependency.
 // TMEM: S_0 cols [0,128), S_1 [128,256) (double-buffered scores, so S_{j+1}
-// is computed while block j is in the softmax; P8_j aliases the first 32
-// columns of S_{j%2}), ACC [256,384) int32, OF [384,512) fp32.
+// is computed while block j is in the softmax), ACC [256,384) int32,
+// OF [384,512) fp32.  P8_j lives inside S_{j%2}: keys [0, 64) in columns
+// [0, 16) and keys [64, 128) in columns [64, 80), so each half writes only
+// columns it has itself read.
 // Shared memory: Q tile (128 x 128 int8 = 16 KB) and a ring of K/V tiles,
 // 128-byte swizzled.  d = 128 only.
 #pragma once
@@ -57,10 +64,11 @@ struct FwdI8Cfg {
   static constexpr int NSLOT = 8;
   static constexpr int Q_OFF = 0;
   static constexpr int SLOT_OFF = TILE;
-  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;  // [4 warps][2 bufs][128] floats
-  static constexpr int BAR_OFF = KC_OFF + 4 * 2 * 128 * 4;
+  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;  // [8 warps][2 bufs][64] floats
+  static constexpr int XCH_OFF = KC_OFF + 8 * 2 * 64 * 4;  // [3 slots][2 halves][128 rows] u64
+  static constexpr int BAR_OFF = XCH_OFF + 3 * 2 * 128 * 8;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t ID_S = idesc_i8(128, false);
   static constexpr uint32_t ID_PV = idesc_i8(128, true);  // V is MN-major
 };
@@ -70,7 +78,7 @@ struct FwdI8Bars {
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint64_t s_full[2];
-  uint64_t p_full;
+  uint64_t p_full[2];  // per block parity: block j + 1 can be released before the MMA thread saw block j
   uint64_t pv_done;
   uint64_t o_full;
   uint64_t drain;
@@ -102,7 +110,7 @@ __device__ __forceinline__ float i2f_small(uint32_t v) {
 }
 
 template <bool SCORES_ONLY>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fwd_int8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdI8Params p) {
   using C = FwdI8Cfg;
@@ -127,7 +135,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(smem_u32(&bars->s_full[0]), 1);
     mbar_init(smem_u32(&bars->s_full[1]), 1);
-    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->p_full[0]), 256);
+    mbar_init(smem_u32(&bars->p_full[1]), 256);
     mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -137,6 +146,11 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
+  }
+  {
+    // exchange slots start with tag 0 (no block uses it), whatever a previous CTA left
+    unsigned long long* xz = reinterpret_cast<unsigned long long*>(smem + C::XCH_OFF);
+    for (int i = threadIdx.x; i < 3 * 2 * 128; i += C::THREADS) xz[i] = 0ull;
   }
   tc_fence_before();
   __syncthreads();
@@ -204,15 +218,15 @@ __global__ void __launch_bounds__(192, 1)
         const int it = vidx(j), s = it % C::NSLOT;
         ok = wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
-        ok = wait_bar(smem_u32(&bars->p_full), j & 1, abort_flag, p.timeout_ns);
+        ok = wait_bar(smem_u32(&bars->p_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)(s * (C::TILE >> 4));
         const uint32_t acc0 = (j > 0) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 keys per MMA: 32 rows x 128 B of V
-          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + kk * 8, dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV,
-                    kk > 0 ? 1u : acc0);
+          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + (kk >> 1) * 64 + (kk & 1) * 8,
+                    dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV, kk > 0 ? 1u : acc0);
         tc_commit(smem_u32(&bars->pv_done));
         tc_commit(smem_u32(&bars->kv_empty[s]));
         if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(192, 1)
       if (SCORES_ONLY) {
         for (int j = 2; j < n && ok; ++j) {
           // the score buffer of j is free once the softmax warps read block j-2
-          ok = wait_bar(smem_u32(&bars->p_full), (j - 2) & 1, abort_flag, p.timeout_ns);
+          ok = wait_bar(smem_u32(&bars->p_full[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns);
           if (ok) ok = issue_S(j);
         }
       }
@@ -233,36 +247,37 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ================================================================ softmax
+    const int half = (warp - 2) >> 2;  // key columns [64 half, 64 half + 64) of every block
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;
     const int row = r0 + rr;
+    const int cb = half * 64;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tACC = tbase + lane_off + 256;
-    const uint32_t tOF = tbase + lane_off + 384;
+    const uint32_t tACC = tbase + lane_off + 256 + cb;
+    const uint32_t tOF = tbase + lane_off + 384 + cb;
+    // exchange slots: [0], [1] row max of even / odd blocks, [2] final l share
+    unsigned long long* xch = reinterpret_cast<unsigned long long*>(smem + C::XCH_OFF);
     const int off = p.Nkv - p.Nq;
     const float qs_row = (!SCORES_ONLY && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] : 0.f;
     const float sv127 = SCORES_ONLY ? 0.f : p.v_scale[bh] * (1.f / 127.f);
     const float* ksrow = p.k_scale + (size_t)bh * p.Nkv;
     // Per-column constants of a key block, kc = s_K * scale * log2(e), kept in
     // this warp's own shared buffer (x / s_Q = S * kc).  Lane l owns columns
-    // [4l, 4l + 4); the next block's scales are loaded one block ahead.
-    float* kcbuf = reinterpret_cast<float*>(smem + C::KC_OFF) + (warp - 2) * (2 * 128);
-    float4 ks_next = make_float4(0.f, 0.f, 0.f, 0.f);
+    // cb + [2l, 2l + 2); the next block's scales are loaded one block ahead.
+    float* kcbuf = reinterpret_cast<float*>(smem + C::KC_OFF) + (warp - 2) * (2 * 64);
+    float2 ks_next = make_float2(0.f, 0.f);
     auto load_ks = [&](int jj) {
-      const int c0 = jj * 128 + lane * 4;
-      if (p.ks_vec && c0 + 3 < p.Nkv) {
-        ks_next = __ldg(reinterpret_cast<const float4*>(ksrow + c0));
+      const int c0 = jj * 128 + cb + lane * 2;
+      if (p.ks_vec && c0 + 1 < p.Nkv) {
+        ks_next = __ldg(reinterpret_cast<const float2*>(ksrow + c0));
       } else {
         ks_next.x = (c0 + 0 < p.Nkv) ? ksrow[c0 + 0] : 0.f;
         ks_next.y = (c0 + 1 < p.Nkv) ? ksrow[c0 + 1] : 0.f;
-        ks_next.z = (c0 + 2 < p.Nkv) ? ksrow[c0 + 2] : 0.f;
-        ks_next.w = (c0 + 3 < p.Nkv) ? ksrow[c0 + 3] : 0.f;
       }
     };
     auto stage_ks = [&](int jj) {
-      float* kcb = kcbuf + (jj & 1) * 128;
-      *reinterpret_cast<float4*>(kcb + lane * 4) =
-          make_float4(ks_next.x * p.sl2, ks_next.y * p.sl2, ks_next.z * p.sl2, ks_next.w * p.sl2);
+      *reinterpret_cast<float2*>(kcbuf + (jj & 1) * 64 + lane * 2) =
+          make_float2(ks_next.x * p.sl2, ks_next.y * p.sl2);
     };
     if (!SCORES_ONLY && n > 0) {
       load_ks(0);
@@ -270,14 +285,14 @@ __global__ void __launch_bounds__(192, 1)
       if (n > 1) load_ks(1);
       __syncwarp();
     }
-    float m_ref = -INFINITY, l = 0.f;
+    float m_ref = -INFINITY, l = 0.f;  // l: this thread's share (its 64 columns)
     bool ok = true;
     if (!SCORES_ONLY) {
       uint32_t z[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) z[i] = 0u;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_st32(tOF + cc * 32, z);
+      for (int cc = 0; cc < 2; ++cc) tmem_st32(tOF + cc * 32, z);
       tmem_st_wait();
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -286,23 +301,23 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tS = tbase + lane_off + (j & 1) * 128;
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      const uint32_t tS = tbase + lane_off + (j & 1) * 128 + cb;
+      uint32_t s[2][32];
+      tmem_ld32(tS, s[0]);
+      tmem_ld32(tS + 32, s[1]);
+      tmem_ld_wait(s[0]);
+      tmem_ld_wait(s[1]);
       if (SCORES_ONLY) {
         if (row < p.Nq) {
-          int* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb;
+          int* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb + cb;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (kb + c * 32 + i < p.Nkv) dst[c * 32 + i] = (int)s[c][i];
+              if (kb + cb + c * 32 + i < p.Nkv) dst[c * 32 + i] = (int)s[c][i];
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_full));
+        mbar_arrive(smem_u32(&bars->p_full[j & 1]));
         continue;
       }
       // y = S * s_K * scale * log2e (= x / s_Q), masked; x = y * s_Q
@@ -313,15 +328,15 @@ __global__ void __launch_bounds__(192, 1)
         lim = p.Nkv - 1 - kb;
         if (p.causal) lim = min(lim, row + off - kb);
       }
-      const float* kcb = kcbuf + (j & 1) * 128;
-      float x[4][32];
+      lim -= cb;
+      const float* kcb = kcbuf + (j & 1) * 64;
+      float x[2][32];
       const uint64_t negM2 = f2(-12582912.f, -12582912.f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          const int col = c * 32 + i;
-          const float4 kc = *reinterpret_cast<const float4*>(kcb + col);
+          const float4 kc = *reinterpret_cast<const float4*>(kcb + c * 32 + i);
           // exact int32 -> fp32 (|S| < 2^22): bits of 1.5 * 2^23 + S, minus 1.5 * 2^23
           const uint64_t sa = fadd2(f2(__int_as_float((int)s[c][i + 0] + 0x4B400000),
                                        __int_as_float((int)s[c][i + 1] + 0x4B400000)), negM2);
@@ -333,7 +348,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (tail || diag) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > lim) x[c][i] = -INFINITY;
@@ -343,16 +358,24 @@ __global__ void __launch_bounds__(192, 1)
         stage_ks(j + 1);
         if (j + 2 < n) load_ks(j + 2);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         mx0 = fmax3(mx0, x[0][i], x[0][i + 1]);
         mx1 = fmax3(mx1, x[1][i], x[1][i + 1]);
-        mx2 = fmax3(mx2, x[2][i], x[2][i + 1]);
-        mx3 = fmax3(mx3, x[3][i], x[3][i + 1]);
       }
+      // row max over both halves.  Slot j % 2 is rewritten for block j + 2
+      // only after this thread read the partner's block j + 1 value, which the
+      // partner writes after reading ours for block j.
+      const float my_max = fmaxf(mx0, mx1);
+      float other_max;
+      xchg_put(xch + (j & 1) * 256 + half * 128 + rr, (uint32_t)j + 1u, my_max);
+      ok = xchg_get(xch + (j & 1) * 256 + (half ^ 1) * 128 + rr, (uint32_t)j + 1u, other_max, abort_flag,
+                    p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
       // s_Q > 0, so max(y) * s_Q is the row max of x
-      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * qs_row;
+      const float m_blk = fmaxf(my_max, other_max) * qs_row;
       // tau = 0: move the reference on every increase
       const bool grow = m_blk > m_ref;
       const bool had = m_ref != -INFINITY;  // rows with earlier content need a fold
@@ -362,28 +385,33 @@ __global__ void __launch_bounds__(192, 1)
         l *= factor;
         m_ref = m_blk;
       }
-      const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      // P8 = rne(127 * 2^(x - m)) = rne(2^(x - m + log2 127)); the rounding is
+      // the low byte of 1.5 * 2^23 + y
+      const float negm = ((m_ref == -INFINITY) ? 0.f : -m_ref) + 6.9886846867721655f;
+      const uint64_t qs2 = f2(qs_row, qs_row), nm2 = f2(negm, negm);
+      const uint64_t mg2 = f2(12582912.f, 12582912.f);
       uint32_t isum = 0;
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          uint32_t t[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float y = ex2(fmaf(x[c][i + e], qs_row, negm)) * 127.f;
-            t[e] = __float_as_uint(y + 12582912.f);  // low bits: rne(y) in [0, 127]
-            isum += t[e];
-          }
-          const uint32_t lo = __byte_perm(t[0], t[1], 0x0040);
-          const uint32_t hi = __byte_perm(t[2], t[3], 0x0040);
-          pk[c * 8 + i / 4] = __byte_perm(lo, hi, 0x5410);
+          float a0, a1, a2, a3;
+          f2_split(ffma2(f2(x[c][i + 0], x[c][i + 1]), qs2, nm2), a0, a1);
+          f2_split(ffma2(f2(x[c][i + 2], x[c][i + 3]), qs2, nm2), a2, a3);
+          float t0, t1, t2, t3;
+          f2_split(fadd2(f2(ex2(a0), ex2(a1)), mg2), t0, t1);
+          f2_split(fadd2(f2(ex2(a2), ex2(a3)), mg2), t2, t3);
+          const uint32_t lo = __byte_perm(__float_as_uint(t0), __float_as_uint(t1), 0x0040);
+          const uint32_t hi = __byte_perm(__float_as_uint(t2), __float_as_uint(t3), 0x0040);
+          const uint32_t w = __byte_perm(lo, hi, 0x5410);
+          pk[c * 8 + i / 4] = w;
+          isum = __dp4a(w, 0x01010101u, isum);
         }
       }
-      isum -= 128u * 0x4B400000u;  // remove the magic offsets (mod 2^32)
       l += (float)isum * (1.f / 127.f);
-      tmem_st32(tS, pk);  // P8 of block j -> first 32 columns of its score buffer
+      // P8 of keys [cb, cb + 64) -> columns [cb, cb + 16) of this block's score buffer
+      tmem_st16(tS, pk);
       if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
         // fold ACC (P V of blocks < j, reference m_old) into OF
         ok = wait_bar(smem_u32(&bars->pv_done), (j - 1) & 1, abort_flag, p.timeout_ns);
@@ -392,7 +420,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const float f = (grow && had) ? factor : 1.f;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t a[32], o[32];
           tmem_ld32(tACC + cc * 32, a);
           tmem_ld32(tOF + cc * 32, o);
@@ -410,38 +438,45 @@ __global__ void __launch_bounds__(192, 1)
       tmem_st_wait();
       __syncwarp();  // the staged scales of block j + 1 are visible to the whole warp
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->p_full));
+      mbar_arrive(smem_u32(&bars->p_full[j & 1]));
     }
     // ---------------------------------------------------------- epilogue
     if (!SCORES_ONLY && ok) {
       ok = wait_bar(smem_u32(&bars->o_full), 0, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        float* orow = p.o + ((size_t)bh * p.Nq + row) * C::D;
+    }
+    if (!SCORES_ONLY && ok) {
+      float l_other;
+      xchg_put(xch + 2 * 256 + half * 128 + rr, 1u, l);
+      ok = xchg_get(xch + 2 * 256 + (half ^ 1) * 128 + rr, 1u, l_other, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      l += l_other;
+    }
+    if (!SCORES_ONLY && ok) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      float* orow = p.o + ((size_t)bh * p.Nq + row) * C::D + cb;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t a[32], o[32];
-          tmem_ld32(tACC + cc * 32, a);
-          tmem_ld32(tOF + cc * 32, o);
-          tmem_ld_wait(a);
-          tmem_ld_wait(o);
-          if (row < p.Nq) {
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t a[32], o[32];
+        tmem_ld32(tACC + cc * 32, a);
+        tmem_ld32(tOF + cc * 32, o);
+        tmem_ld_wait(a);
+        tmem_ld_wait(o);
+        if (row < p.Nq) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 v;
-              v.x = (l > 0.f) ? (__uint_as_float(o[i + 0]) + (float)(int)a[i + 0] * sv127) * inv : 0.f;
-              v.y = (l > 0.f) ? (__uint_as_float(o[i + 1]) + (float)(int)a[i + 1] * sv127) * inv : 0.f;
-              v.z = (l > 0.f) ? (__uint_as_float(o[i + 2]) + (float)(int)a[i + 2] * sv127) * inv : 0.f;
-              v.w = (l > 0.f) ? (__uint_as_float(o[i + 3]) + (float)(int)a[i + 3] * sv127) * inv : 0.f;
-              *reinterpret_cast<float4*>(orow + cc * 32 + i) = v;
-            }
+          for (int i = 0; i < 32; i += 4) {
+            float4 v;
+            v.x = (l > 0.f) ? (__uint_as_float(o[i + 0]) + (float)(int)a[i + 0] * sv127) * inv : 0.f;
+            v.y = (l > 0.f) ? (__uint_as_float(o[i + 1]) + (float)(int)a[i + 1] * sv127) * inv : 0.f;
+            v.z = (l > 0.f) ? (__uint_as_float(o[i + 2]) + (float)(int)a[i + 2] * sv127) * inv : 0.f;
+            v.w = (l > 0.f) ? (__uint_as_float(o[i + 3]) + (float)(int)a[i + 3] * sv127) * inv : 0.f;
+            *reinterpret_cast<float4*>(orow + cc * 32 + i) = v;
           }
         }
-        if (row < p.Nq)
-          p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
+      if (half == 0 && row < p.Nq)
+        p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

@@ -85,6 +85,36 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Pairwise exchange of one float between two threads of different warps
+// through a 64-bit shared slot {tag, value}: the writer stores (tag << 32 |
+// bits) in one 64-bit access; the reader polls its partner's slot until the
+// tag matches (bounded like wait_bar: abort flag, then time limit).  Unlike a
+// named barrier, a partner that gave up cannot leave this thread stuck.
+__device__ __forceinline__ void xchg_put(unsigned long long* slot, uint32_t tag, float v) {
+  *reinterpret_cast<volatile unsigned long long*>(slot) =
+      ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
+}
+__device__ __forceinline__ bool xchg_get(const unsigned long long* slot, uint32_t tag, float& v,
+                                         volatile int* abort_flag, uint64_t limit_ns) {
+  const volatile unsigned long long* vs = reinterpret_cast<const volatile unsigned long long*>(slot);
+  unsigned long long e = *vs;
+  if ((uint32_t)(e >> 32) != tag) {
+    const uint64_t t0 = global_ns();
+    while (true) {
+      e = *vs;
+      if ((uint32_t)(e >> 32) == tag) break;
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicExch(&g_attn_status, -5 /* ATTN_ERR_TIMEOUT */);
+        return false;
+      }
+    }
+  }
+  v = __uint_as_float((uint32_t)e);
+  return true;
+}
+
 // --------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -220,6 +250,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
       "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
       "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// 32 lanes x 16 columns (thread i: lane base + i, columns [col, col+16)).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() {
