@@ -110,7 +110,7 @@ int launch_fp4(const void* q, const void* qsf, const void* k, const void* ksf, c
   p.s_out = s_out;
   p.Nq = Nq;
   p.Nkv = Nkv;
-  p.n_qt = (Nq + 127) / 128;
+  p.n_qp = (Nq + 255) / 256;
   p.Tc = KT;
   p.RTq = (Nq + 127) / 128;
   p.KT = KT;
@@ -118,7 +118,7 @@ int launch_fp4(const void* q, const void* qsf, const void* k, const void* ksf, c
   p.p_mode = p_mode;
   p.sl2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_ns;
-  const long long grid = (long long)BH * p.n_qt;
+  const long long grid = (long long)BH * p.n_qp;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   ta::fwd_fp4_kernel<SCORES_ONLY><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

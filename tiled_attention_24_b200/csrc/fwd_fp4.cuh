@@ -18,16 +18,24 @@
 //   O / l (fp32 output), LSE = ln2 * (m + log2(l / p_unit)), p_unit = 6 for
 //   Direct-P (whose P~ approximates 6 * 2^(x - m)), 1 otherwise
 //
-// CTA = one (batch, head) x one 128-row query tile; warps: 0 TMA producer,
-// 1 MMA issuer, 2-5 softmax / correction / epilogue (thread = row).
+// CTA = one (batch, head) x two 128-row query tiles; warps: 0 TMA producer,
+// 1 MMA issuer, 2-3 idle (their registers go to the softmax warps through
+// setmaxnreg), 4-7 softmax / correction / epilogue of tile 0, 8-11 of tile 1
+// (thread = row).  The two tiles run concurrently, so each SM sub-partition
+// has two softmax warps at independent phases: while one waits for an MMA or
+// a barrier, or runs integer / fp32 work, the other keeps the exp pipe busy.
 // Operands in shared memory (64-byte swizzled, K-major, 64 bytes = 128 e2m1
-// codes per row): Q tile, ring of K and V^T tiles; each with its 1 KB of
-// scale factors, which tcgen05.cp copies into TMEM in the layout the MMA reads
-// (32 lanes x 16 bytes, replicated over the 4 lane quarters).  P is written
-// by the softmax threads into a shared-memory tile (the A operand of a
-// block-scaled MMA comes from shared memory), double-buffered, with its scale
-// factors.  TMEM: S_0 [0,128), S_1 [128,256), O [256,384), scale factors from
-// column 384.  d = 128 only.
+// codes per row): the two Q tiles, a ring of K and V^T tiles; each with its
+// 1 KB of scale factors, which tcgen05.cp copies into TMEM in the layout the
+// MMA reads (32 lanes x 16 bytes, replicated over the 4 lane quarters).  P is
+// written by the softmax threads into a shared-memory tile per query tile
+// (the A operand of a block-scaled MMA comes from shared memory),
+// double-buffered, with its scale factors.
+// TMEM: one score buffer S [0,128) shared by the tiles (its scores are moved
+// to registers at once, then it is released to the other tile), O_0
+// [128,256), O_1 [256,384), scale factors from column 384.  The next block's
+// S of a tile is issued before that tile's current P V, so a softmax warp
+// finds its next scores ready when it finishes a block.  d = 128 only.
 #pragma once
 #include "ptx.cuh"
 #include "fwd_bf16.cuh"
@@ -42,7 +50,7 @@ struct FwdF4Params {
   float* o;             // [BH][Nq][128]
   float* lse;           // [BH][Nq]
   float* s_out;         // optional [BH][Nq][Nkv] scores (check of the block-scaled GEMM)
-  int Nq, Nkv, n_qt, Tc, RTq, KT;
+  int Nq, Nkv, n_qp, Tc, RTq, KT;  // n_qp: pairs of 128-row query tiles
   int causal, p_mode;
   float sl2;
   unsigned long long timeout_ns;
@@ -58,28 +66,36 @@ struct FwdF4Cfg {
   static constexpr int TILE = 128 * 64;  // 128 rows x 64 bytes of codes
   static constexpr int SF = 1024;
   static constexpr int SLOTB = 10240;    // codes + scales, 1 KB aligned
-  static constexpr int NSLOT = 16;      // also keeps one CTA per SM (TMEM)
-  static constexpr int Q_OFF = 0;
-  static constexpr int QSF_OFF = TILE;
-  static constexpr int SLOT_OFF = 10240;
-  static constexpr int P_OFF = SLOT_OFF + NSLOT * SLOTB;
-  static constexpr int PSF_OFF = P_OFF + 2 * TILE;
-  static constexpr int BAR_OFF = PSF_OFF + 2 * SF;
+  static constexpr int NSLOT = 8;
+  static constexpr int Q_OFF = 0;                      // Q_0, Q_1
+  static constexpr int QSF_OFF = 2 * TILE;             // their scales
+  static constexpr int SLOT_OFF = QSF_OFF + 2 * SF;    // 18 KB
+  static constexpr int P_OFF = SLOT_OFF + NSLOT * SLOTB;  // [tile][buffer] P tiles
+  static constexpr int PSF_OFF = P_OFF + 4 * TILE;        // [tile][buffer] P scales
+  static constexpr int BAR_OFF = PSF_OFF + 4 * SF;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 384;
+  // register split (launch: 384 threads x 168): warpgroup 0 drops to 72, the
+  // two softmax warpgroups rise to 216: 128*72 + 256*216 = 64512 = 384*168
+  static constexpr int REG_LOW = 72, REG_HIGH = 216;
   static constexpr uint32_t ID = idesc_nvf4(128, 128);
-  // TMEM columns of the scale factors (8 columns = 2 MMA steps x 4)
-  static constexpr uint32_t T_SFQ = 384, T_SFK = 392, T_SFV = 408, T_SFP = 424;
+  // TMEM columns: S, O_t, and the scale factors (8 columns = 2 MMA steps x 4)
+  static constexpr uint32_t T_S = 0, T_O = 128;
+  static constexpr uint32_t T_SFQ = 384;  // + 8 t
+  static constexpr uint32_t T_SFK = 400;  // + 8 (j % 2)
+  static constexpr uint32_t T_SFV = 416;  // + 8 (j % 2)
+  static constexpr uint32_t T_SFP = 432;  // + 16 t + 8 (j % 2)
 };
 
 struct FwdF4Bars {
   uint64_t q_full;
-  uint64_t kv_full[16];
-  uint64_t kv_empty[16];
-  uint64_t s_full[2];
-  uint64_t p_full[2];  // per block parity: block j + 1 can be released before the MMA thread saw block j
-  uint64_t pv_done;
-  uint64_t o_full;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_full[2];     // MMA -> softmax of tile t: S_t(j) in the score buffer
+  uint64_t s_free;        // softmax -> MMA: the score buffer's scores are in registers
+  uint64_t p_full[2][2];  // [tile][j % 2]: P_t(j) and its scales in smem, O_t corrected
+  uint64_t pv_done[2];    // [tile]: P V_t(j) finished
+  uint64_t o_full[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -142,7 +158,7 @@ __device__ __forceinline__ float f16x2_sum(uint32_t v) {
 }
 
 template <bool SCORES_ONLY>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_fp4_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdF4Params p) {
   using C = FwdF4Cfg;
@@ -152,11 +168,19 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int BH = gridDim.x / p.n_qt;
-  const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qt);
-  const int qt = p.causal ? p.n_qt - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qt);
-  const int r0 = qt * 128;
-  const int n = fwd_tile_kv_count(r0, p.Nq, p.Nkv, p.Tc, p.causal);
+  // ---- work item: (batch*head, pair of query tiles); heaviest pairs first when causal
+  const int BH = gridDim.x / p.n_qp;
+  const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qp);
+  const int qp = p.causal ? p.n_qp - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qp);
+  int r0[2], n[2];
+  bool present[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    r0[t] = qp * 256 + t * 128;
+    present[t] = r0[t] < p.Nq;
+    n[t] = fwd_tile_kv_count(r0[t], p.Nq, p.Nkv, p.Tc, p.causal);
+  }
+  const int nmax = max(n[0], n[1]);
   volatile int* abort_flag = &bars->abort;
 
   if (threadIdx.x == 0) {
@@ -165,12 +189,14 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
       mbar_init(smem_u32(&bars->kv_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->s_full[0]), 1);
-    mbar_init(smem_u32(&bars->s_full[1]), 1);
-    mbar_init(smem_u32(&bars->p_full[0]), 128);
-    mbar_init(smem_u32(&bars->p_full[1]), 128);
-    mbar_init(smem_u32(&bars->pv_done), 1);
-    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->s_free), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->p_full[t][0]), 128);
+      mbar_init(smem_u32(&bars->p_full[t][1]), 128);
+      mbar_init(smem_u32(&bars->pv_done[t]), 1);
+      mbar_init(smem_u32(&bars->o_full[t]), 1);
+    }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -186,19 +212,24 @@ __global__ void __launch_bounds__(192, 1)
   auto kidx = [&](int j) { return SCORES_ONLY ? j : 2 * j; };
   auto vidx = [&](int j) { return 2 * j + 1; };
 
-  if (warp == 0) {
+  if (warp < 4) {
+   reg_dealloc<C::REG_LOW>();
+   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       if (!SCORES_ONLY) prefetch_tmap(&tmV);
       const uint32_t qbar = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qbar, C::TILE + C::SF);
-      tma_load_3d(sbase + C::Q_OFF, &tmQ, qbar, 0, r0, bh);
-      bulk_load(sbase + C::QSF_OFF, p.q_sf + ((size_t)bh * p.RTq + qt) * C::SF, C::SF, qbar);
+      mbar_arrive_expect_tx(qbar, (present[1] ? 2 : 1) * (C::TILE + C::SF));
+      for (int t = 0; t < 2; ++t) {
+        if (!present[t]) continue;
+        tma_load_3d(sbase + C::Q_OFF + t * C::TILE, &tmQ, qbar, 0, r0[t], bh);
+        bulk_load(sbase + C::QSF_OFF + t * C::SF, p.q_sf + ((size_t)bh * p.RTq + 2 * qp + t) * C::SF, C::SF, qbar);
+      }
       int it = 0;
       bool ok = true;
-      for (int j = 0; j < n && ok; ++j) {
+      for (int j = 0; j < nmax && ok; ++j) {
         for (int w = 0; w < (SCORES_ONLY ? 1 : 2) && ok; ++w, ++it) {
           const int slot = it % C::NSLOT;
           ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ((it / C::NSLOT) & 1) ^ 1, abort_flag, p.timeout_ns);
@@ -224,68 +255,96 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // S sequence S_0(0), S_1(0), S_0(1), S_1(1), ... through the one score
+    // buffer (each waits until the previous one's scores are in registers);
+    // program order: prologue S_0(0), S_1(0), S_0(1); then per block j:
+    // P V_0(j), S_1(j+1), P V_1(j), S_0(j+2).
     if (lane == 0) {
       bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
       tc_fence_after();
-      const uint64_t dQ = smem_desc_l(sbase + C::Q_OFF, 16, 512, 4);
+      const uint64_t dQ0 = smem_desc_l(sbase + C::Q_OFF, 16, 512, 4);
       const uint64_t dSlot0 = smem_desc_l(sbase + C::SLOT_OFF, 16, 512, 4);
       const uint64_t dSf0 = smem_desc_l(sbase + C::SLOT_OFF + C::TILE, 16, 128, 0);
       const uint64_t dP0 = smem_desc_l(sbase + C::P_OFF, 16, 512, 4);
       const uint64_t dPsf0 = smem_desc_l(sbase + C::PSF_OFF, 16, 128, 0);
       if (ok) {
-        const uint64_t dQsf = smem_desc_l(sbase + C::QSF_OFF, 16, 128, 0);
-        tc_cp_sf(tbase + C::T_SFQ, dQsf);
-        tc_cp_sf(tbase + C::T_SFQ + 4, dQsf + (512 >> 4));
+        for (int t = 0; t < 2; ++t) {
+          if (!present[t]) continue;
+          const uint64_t dQsf = smem_desc_l(sbase + C::QSF_OFF + t * C::SF, 16, 128, 0);
+          tc_cp_sf(tbase + C::T_SFQ + 8 * t, dQsf);
+          tc_cp_sf(tbase + C::T_SFQ + 8 * t + 4, dQsf + (512 >> 4));
+        }
       }
-      auto issue_S = [&](int j) -> bool {
+      int n_s = 0;  // S MMAs issued so far (the score buffer's uses)
+      auto issue_S = [&](int t, int j) -> bool {
+        if (n_s > 0) {
+          if (!wait_bar(smem_u32(&bars->s_free), (n_s - 1) & 1, abort_flag, p.timeout_ns)) return false;
+          tc_fence_after();
+        }
         const int it = kidx(j), s = it % C::NSLOT;
-        if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
-        tc_fence_after();
         const uint64_t so = (uint64_t)(s * (C::SLOTB >> 4));
         const uint32_t sfk = tbase + C::T_SFK + (j & 1) * 8;
-        tc_cp_sf(sfk, dSf0 + so);
-        tc_cp_sf(sfk + 4, dSf0 + so + (512 >> 4));
+        const bool first = (t == 0) || (j >= n[0]);   // first user of K_j
+        const bool last = (t == 1) || (j >= n[1]);    // last user of K_j
+        if (first) {
+          if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
+          tc_fence_after();
+          tc_cp_sf(sfk, dSf0 + so);
+          tc_cp_sf(sfk + 4, dSf0 + so + (512 >> 4));
+        }
+        const uint64_t dq = dQ0 + (uint64_t)(t * (C::TILE >> 4));
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)  // K = 64 e2m1 (32 bytes) per MMA
-          mma_nvf4(tbase + (j & 1) * 128, dQ + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID,
-                   tbase + C::T_SFQ + ks * 4, sfk + ks * 4, ks > 0);
-        tc_commit(smem_u32(&bars->s_full[j & 1]));
-        tc_commit(smem_u32(&bars->kv_empty[s]));
+          mma_nvf4(tbase + C::T_S, dq + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID,
+                   tbase + C::T_SFQ + 8 * t + ks * 4, sfk + ks * 4, ks > 0);
+        tc_commit(smem_u32(&bars->s_full[t]));
+        if (last) tc_commit(smem_u32(&bars->kv_empty[s]));
+        ++n_s;
         return true;
       };
-      if (ok && n == 0) tc_commit(smem_u32(&bars->o_full));
-      if (ok && n > 0) ok = issue_S(0);
-      if (ok && n > 1) ok = issue_S(1);
-      for (int j = 0; j < n && ok && !SCORES_ONLY; ++j) {
+      auto issue_PV = [&](int t, int j) -> bool {
         const int it = vidx(j), s = it % C::NSLOT;
-        ok = wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
-        ok = wait_bar(smem_u32(&bars->p_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
         const uint64_t so = (uint64_t)(s * (C::SLOTB >> 4));
-        const uint32_t sfv = tbase + C::T_SFV + (j & 1) * 8, sfp = tbase + C::T_SFP + (j & 1) * 8;
-        const uint64_t po = (uint64_t)((j & 1) * (C::TILE >> 4)), pso = (uint64_t)((j & 1) * (C::SF >> 4));
-        tc_cp_sf(sfv, dSf0 + so);
-        tc_cp_sf(sfv + 4, dSf0 + so + (512 >> 4));
+        const uint32_t sfv = tbase + C::T_SFV + (j & 1) * 8;
+        const bool first = (t == 0) || (j >= n[0]);
+        const bool last = (t == 1) || (j >= n[1]);
+        if (first) {
+          if (!wait_bar(smem_u32(&bars->kv_full[s]), (it / C::NSLOT) & 1, abort_flag, p.timeout_ns)) return false;
+          tc_fence_after();
+          tc_cp_sf(sfv, dSf0 + so);
+          tc_cp_sf(sfv + 4, dSf0 + so + (512 >> 4));
+        }
+        if (!wait_bar(smem_u32(&bars->p_full[t][j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns)) return false;
+        tc_fence_after();
+        const int pb = t * 2 + (j & 1);
+        const uint32_t sfp = tbase + C::T_SFP + pb * 8;
+        const uint64_t pso = (uint64_t)(pb * (C::SF >> 4));
         tc_cp_sf(sfp, dPsf0 + pso);
         tc_cp_sf(sfp + 4, dPsf0 + pso + (512 >> 4));
+        const uint64_t po = (uint64_t)(pb * (C::TILE >> 4));
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          mma_nvf4(tbase + 256, dP0 + po + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID, sfp + ks * 4,
-                   sfv + ks * 4, (j > 0 || ks > 0) ? 1u : 0u);
-        tc_commit(smem_u32(&bars->pv_done));
-        tc_commit(smem_u32(&bars->kv_empty[s]));
-        if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
-        if (j + 2 < n) ok = issue_S(j + 2);
+          mma_nvf4(tbase + C::T_O + 128 * t, dP0 + po + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID,
+                   sfp + ks * 4, sfv + ks * 4, (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bars->pv_done[t]));
+        if (last) tc_commit(smem_u32(&bars->kv_empty[s]));
+        if (j == n[t] - 1) tc_commit(smem_u32(&bars->o_full[t]));
+        return true;
+      };
+      if (ok) {
+        for (int t = 0; t < 2; ++t)
+          if (!SCORES_ONLY && present[t] && n[t] == 0) tc_commit(smem_u32(&bars->o_full[t]));
       }
-      if (SCORES_ONLY) {
-        for (int j = 2; j < n && ok; ++j) {
-          ok = wait_bar(smem_u32(&bars->p_full[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns);
-          if (ok) ok = issue_S(j);
-        }
+      if (ok && n[0] > 0) ok = issue_S(0, 0);
+      if (ok && n[1] > 0) ok = issue_S(1, 0);
+      if (ok && n[0] > 1) ok = issue_S(0, 1);
+      for (int j = 0; j < nmax && ok; ++j) {
+        if (!SCORES_ONLY && j < n[0] && !(ok = issue_PV(0, j))) break;
+        if (j + 1 < n[1] && !(ok = issue_S(1, j + 1))) break;
+        if (!SCORES_ONLY && j < n[1] && !(ok = issue_PV(1, j))) break;
+        if (j + 2 < n[0] && !(ok = issue_S(0, j + 2))) break;
       }
       if (!ok) {
         tc_commit(smem_u32(&bars->drain));
@@ -293,35 +352,40 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
+   }
   } else {
+    reg_alloc<C::REG_HIGH>();
     // ================================================================ softmax
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;
-    const int row = r0 + rr;
+    const int row = r0[t] + rr;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tO = tbase + lane_off + 256;
+    const uint32_t tS = tbase + lane_off + C::T_S;
+    const uint32_t tO = tbase + lane_off + C::T_O + 128 * t;
     const int off = p.Nkv - p.Nq;
     const float sl2 = p.sl2;
     const bool direct = p.p_mode == 0;
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
+    bool ok = present[t];
     if (!SCORES_ONLY && direct) {
-      // Direct-P: every P block scale is 1.0 (0x38); both buffers, written once
-      for (int i = threadIdx.x - 64; i < 2 * C::SF / 4; i += 128)
-        *reinterpret_cast<uint32_t*>(smem + C::PSF_OFF + i * 4) = 0x38383838u;
+      // Direct-P: every P block scale is 1.0 (0x38); this tile's two buffers, written once
+      for (int i = threadIdx.x & 127; i < 2 * C::SF / 4; i += 128)
+        *reinterpret_cast<uint32_t*>(smem + C::PSF_OFF + t * 2 * C::SF + i * 4) = 0x38383838u;
     }
-    for (int j = 0; j < n && ok; ++j) {
+    for (int j = 0; j < n[t] && ok; ++j) {
       const int kb = j * 128;
-      ok = wait_bar(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns);
+      ok = wait_bar(smem_u32(&bars->s_full[t]), j & 1, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tS = tbase + lane_off + (j & 1) * 128;
       uint32_t s[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->s_free));  // the score buffer goes to the other tile
       if (SCORES_ONLY) {
         if (row < p.Nq) {
           float* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb;
@@ -331,12 +395,10 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < 32; ++i)
               if (kb + c * 32 + i < p.Nkv) dst[c * 32 + i] = __uint_as_float(s[c][i]);
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_full[j & 1]));
         continue;
       }
       const bool tail = kb + 128 > p.Nkv;
-      const bool diag = p.causal && (kb + 127 > r0 + off);
+      const bool diag = p.causal && (kb + 127 > r0[t] + off);
       if (tail || diag) {
         int lim = p.Nkv - 1 - kb;
         if (p.causal) lim = min(lim, row + off - kb);
@@ -364,9 +426,11 @@ __global__ void __launch_bounds__(192, 1)
         m_ref = m_blk;
       }
       const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      // ---- P codes (row rr of the P tile, 64 bytes, 64-byte swizzle) and scales
-      uint8_t* ptile = smem + C::P_OFF + (j & 1) * C::TILE + rr * 64;
-      uint8_t* psf = smem + C::PSF_OFF + (j & 1) * C::SF;
+      // ---- P codes (row rr of the P tile, 64 bytes, 64-byte swizzle) and scales.
+      // Buffer j % 2 was last read by P V_t(j-2), which finished before S_t(j)
+      // was computed (the S_t(j) commit covers every earlier MMA).
+      uint8_t* ptile = smem + C::P_OFF + (t * 2 + (j & 1)) * C::TILE + rr * 64;
+      uint8_t* psf = smem + C::PSF_OFF + (t * 2 + (j & 1)) * C::SF;
       float lsum = 0.f;
       // Direct-P: 6 * 2^(x - m) = 2^(x - m + log2 6), one exponential per score
       const float neg_arg = direct ? negm + 2.5849625007211562f : negm;
@@ -408,8 +472,8 @@ __global__ void __launch_bounds__(192, 1)
       }
       l += lsum;
       if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
-        // rescale O (P V of blocks < j) to the new reference
-        ok = wait_bar(smem_u32(&bars->pv_done), (j - 1) & 1, abort_flag, p.timeout_ns);
+        // rescale O_t (P V of blocks < j) to the new reference
+        ok = wait_bar(smem_u32(&bars->pv_done[t]), (j - 1) & 1, abort_flag, p.timeout_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -427,11 +491,11 @@ __global__ void __launch_bounds__(192, 1)
       }
       fence_proxy_async_smem();  // P tile and scales are read by the tensor core
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->p_full[j & 1]));
+      mbar_arrive(smem_u32(&bars->p_full[t][j & 1]));
     }
     // ---------------------------------------------------------- epilogue
     if (!SCORES_ONLY && ok) {
-      ok = wait_bar(smem_u32(&bars->o_full), 0, abort_flag, p.timeout_ns);
+      ok = wait_bar(smem_u32(&bars->o_full[t]), 0, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
