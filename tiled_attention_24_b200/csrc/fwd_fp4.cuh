@@ -35,7 +35,10 @@
 // to registers at once, then it is released to the other tile), O_0
 // [128,256), O_1 [256,384), scale factors from column 384.  The next block's
 // S of a tile is issued before that tile's current P V, so a softmax warp
-// finds its next scores ready when it finishes a block.  d = 128 only.
+// finds its next scores ready when it finishes a block.  The row sums l of
+// the P values are accumulated by the tensor core too: P times a 16-column
+// matrix of ones (e2m1 1.0, scale 1.0) into 16 TMEM columns per tile, so the
+// softmax threads never decode their own codes.  d = 128 only.
 #pragma once
 #include "ptx.cuh"
 #include "fwd_bf16.cuh"
@@ -72,19 +75,24 @@ struct FwdF4Cfg {
   static constexpr int SLOT_OFF = QSF_OFF + 2 * SF;    // 18 KB
   static constexpr int P_OFF = SLOT_OFF + NSLOT * SLOTB;  // [tile][buffer] P tiles
   static constexpr int PSF_OFF = P_OFF + 4 * TILE;        // [tile][buffer] P scales
-  static constexpr int BAR_OFF = PSF_OFF + 4 * SF;
+  static constexpr int ONES_OFF = PSF_OFF + 4 * SF;      // 16 x 128 e2m1 ones (0x22 bytes)
+  static constexpr int SF1_OFF = ONES_OFF + 1024;        // 512 bytes of scale 1.0 (0x38)
+  static constexpr int BAR_OFF = SF1_OFF + 512;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;
   static constexpr int THREADS = 384;
   // register split (launch: 384 threads x 168): warpgroup 0 drops to 72, the
   // two softmax warpgroups rise to 216: 128*72 + 256*216 = 64512 = 384*168
   static constexpr int REG_LOW = 72, REG_HIGH = 216;
   static constexpr uint32_t ID = idesc_nvf4(128, 128);
+  static constexpr uint32_t ID_L = idesc_nvf4(128, 16);  // P x ones: row sums
   // TMEM columns: S, O_t, and the scale factors (8 columns = 2 MMA steps x 4)
   static constexpr uint32_t T_S = 0, T_O = 128;
   static constexpr uint32_t T_SFQ = 384;  // + 8 t
   static constexpr uint32_t T_SFK = 400;  // + 8 (j % 2)
   static constexpr uint32_t T_SFV = 416;  // + 8 (j % 2)
   static constexpr uint32_t T_SFP = 432;  // + 16 t + 8 (j % 2)
+  static constexpr uint32_t T_SF1 = 464;  // scales of the ones matrix
+  static constexpr uint32_t T_L = 480;    // + 16 t: row sums of tile t (column 0 is read)
 };
 
 struct FwdF4Bars {
@@ -205,6 +213,10 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
+  // constant operands of the row-sum MMA: e2m1 ones (code 2) and their scales (1.0)
+  for (int i = threadIdx.x; i < (1024 + 512) / 4; i += C::THREADS)
+    *reinterpret_cast<uint32_t*>(smem + C::ONES_OFF + i * 4) = (i < 256) ? 0x22222222u : 0x38383838u;
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -269,7 +281,11 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dSf0 = smem_desc_l(sbase + C::SLOT_OFF + C::TILE, 16, 128, 0);
       const uint64_t dP0 = smem_desc_l(sbase + C::P_OFF, 16, 512, 4);
       const uint64_t dPsf0 = smem_desc_l(sbase + C::PSF_OFF, 16, 128, 0);
+      const uint64_t dOnes = smem_desc_l(sbase + C::ONES_OFF, 16, 512, 4);
       if (ok) {
+        const uint64_t dSf1 = smem_desc_l(sbase + C::SF1_OFF, 16, 128, 0);
+        tc_cp_sf(tbase + C::T_SF1, dSf1);
+        tc_cp_sf(tbase + C::T_SF1 + 4, dSf1);
         for (int t = 0; t < 2; ++t) {
           if (!present[t]) continue;
           const uint64_t dQsf = smem_desc_l(sbase + C::QSF_OFF + t * C::SF, 16, 128, 0);
@@ -328,6 +344,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int ks = 0; ks < 2; ++ks)
           mma_nvf4(tbase + C::T_O + 128 * t, dP0 + po + (uint64_t)(ks * 2), dSlot0 + so + (uint64_t)(ks * 2), C::ID,
                    sfp + ks * 4, sfv + ks * 4, (j > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)  // l_t += P~ 1
+          mma_nvf4(tbase + C::T_L + 16 * t, dP0 + po + (uint64_t)(ks * 2), dOnes + (uint64_t)(ks * 2), C::ID_L,
+                   sfp + ks * 4, tbase + C::T_SF1 + ks * 4, (j > 0 || ks > 0) ? 1u : 0u);
         tc_commit(smem_u32(&bars->pv_done[t]));
         if (last) tc_commit(smem_u32(&bars->kv_empty[s]));
         if (j == n[t] - 1) tc_commit(smem_u32(&bars->o_full[t]));
@@ -363,10 +383,11 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tbase + lane_off + C::T_S;
     const uint32_t tO = tbase + lane_off + C::T_O + 128 * t;
+    const uint32_t tL = tbase + lane_off + C::T_L + 16 * t;
     const int off = p.Nkv - p.Nq;
     const float sl2 = p.sl2;
     const bool direct = p.p_mode == 0;
-    float m_ref = -INFINITY, l = 0.f;
+    float m_ref = -INFINITY;  // l lives in TMEM (column tL), summed by the tensor core
     bool ok = present[t];
     if (!SCORES_ONLY && direct) {
       // Direct-P: every P block scale is 1.0 (0x38); this tile's two buffers, written once
@@ -422,7 +443,6 @@ __global__ void __launch_bounds__(384, 1)
       float factor = 1.f;
       if (grow) {
         factor = had ? ex2(m_ref - m_blk) : 0.f;
-        l *= factor;
         m_ref = m_blk;
       }
       const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
@@ -431,7 +451,6 @@ __global__ void __launch_bounds__(384, 1)
       // was computed (the S_t(j) commit covers every earlier MMA).
       uint8_t* ptile = smem + C::P_OFF + (t * 2 + (j & 1)) * C::TILE + rr * 64;
       uint8_t* psf = smem + C::PSF_OFF + (t * 2 + (j & 1)) * C::SF;
-      float lsum = 0.f;
       // Direct-P: 6 * 2^(x - m) = 2^(x - m + log2 6), one exponential per score
       const float neg_arg = direct ? negm + 2.5849625007211562f : negm;
 #pragma unroll
@@ -456,13 +475,8 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < 16; ++e) v[e] *= r;
         }
         uint32_t b[8];
-        uint32_t hs = 0u;  // f16x2 running sum of the decoded codes
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          b[e] = e2m1x2_pos(v[2 * e], v[2 * e + 1]);
-          hs = hadd2(hs, e2m1x2_f16x2(b[e]));
-        }
-        lsum += f16x2_sum(hs) * sc;  // l sums the P values the MMA multiplies into V
+        for (int e = 0; e < 8; ++e) b[e] = e2m1x2_pos(v[2 * e], v[2 * e + 1]);
         const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
         const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
         // 8 bytes = keys [16 blk, 16 blk + 16) -> chunk blk / 2, half blk % 2
@@ -470,9 +484,8 @@ __global__ void __launch_bounds__(384, 1)
         uint8_t* dst = ptile + ((chunk ^ ((rr >> 1) & 3)) << 4) + (blk & 1) * 8;
         *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
       }
-      l += lsum;
       if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
-        // rescale O_t (P V of blocks < j) to the new reference
+        // rescale O_t and l_t (blocks < j) to the new reference
         ok = wait_bar(smem_u32(&bars->pv_done[t]), (j - 1) & 1, abort_flag, p.timeout_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -487,6 +500,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
           tmem_st32(tO + cc * 32, o);
         }
+        uint32_t lv = tmem_ld1(tL);
+        tmem_ld_wait1(lv);
+        tmem_st1(tL, __float_as_uint(__uint_as_float(lv) * f));
         tmem_st_wait();
       }
       fence_proxy_async_smem();  // P tile and scales are read by the tensor core
@@ -499,6 +515,12 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
+        float l = 0.f;  // no block visible: no row-sum MMA ran, the column is stale
+        if (n[t] > 0) {
+          uint32_t lv = tmem_ld1(tL);
+          tmem_ld_wait1(lv);
+          l = __uint_as_float(lv);
+        }
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         float* orow = p.o + ((size_t)bh * p.Nq + row) * 128;
 #pragma unroll 1
