@@ -453,26 +453,50 @@ __global__ void __launch_bounds__(384, 1)
       uint8_t* psf = smem + C::PSF_OFF + (t * 2 + (j & 1)) * C::SF;
       // Direct-P: 6 * 2^(x - m) = 2^(x - m + log2 6), one exponential per score
       const float neg_arg = direct ? negm + 2.5849625007211562f : negm;
+      // p = 2^(x - m) (times 6 for Direct-P) for the whole row, in place
+      const uint64_t sl2x2 = f2(sl2, sl2), na2 = f2(neg_arg, neg_arg);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float a0, a1;
+          f2_split(ffma2(f2(__uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1])), sl2x2, na2), a0, a1);
+          s[c][i] = __float_as_uint(ex2(a0));
+          s[c][i + 1] = __float_as_uint(ex2(a1));
+        }
+      // quantise-after-exp: the 8 block scales of the row first (independent
+      // chains), then codes of p * (1 / sf): within an ulp of p / sf, so only a
+      // value on an e2m1 rounding boundary can round differently; a zero scale
+      // (an all-zero block) gives zero codes
+      float rs[8];
+      if (!direct) {
+#pragma unroll
+        for (int blk = 0; blk < 8; ++blk) {
+          const uint32_t* v = &s[blk >> 1][(blk & 1) * 16];
+          const float a0 = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+          const float a1 = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+          const float a2 = fmax3(__uint_as_float(v[6]), __uint_as_float(v[7]), __uint_as_float(v[8]));
+          const float a3 = fmax3(__uint_as_float(v[9]), __uint_as_float(v[10]), __uint_as_float(v[11]));
+          const float a4 = fmax3(__uint_as_float(v[12]), __uint_as_float(v[13]), __uint_as_float(v[14]));
+          const float amax = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, __uint_as_float(v[15])), 0.f);
+          const uint32_t sfc = (amax > 0.f) ? e4m3_rne(__fdiv_rn(fmaxf(amax, 1e-30f), 6.f)) : 0u;
+          const float sc = e4m3_value(sfc);
+          psf[sf_offset(rr, blk)] = (uint8_t)sfc;
+          rs[blk] = (sc > 0.f) ? __frcp_rn(sc) : 0.f;
+        }
+      }
 #pragma unroll
       for (int blk = 0; blk < 8; ++blk) {  // 16 keys per block
         const int c = blk >> 1, i0 = (blk & 1) * 16;
         float v[16];
+        if (direct) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = ex2(fmaf(__uint_as_float(s[c][i0 + e]), sl2, neg_arg));
-        float sc = 1.f;
-        if (!direct) {
-          float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]), a2 = fmax3(v[6], v[7], v[8]);
-          float a3 = fmax3(v[9], v[10], v[11]), a4 = fmax3(v[12], v[13], v[14]);
-          const float amax = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]), 0.f);
-          const uint32_t sfc = (amax > 0.f) ? e4m3_rne(__fdiv_rn(fmaxf(amax, 1e-30f), 6.f)) : 0u;
-          sc = e4m3_value(sfc);
-          psf[sf_offset(rr, blk)] = (uint8_t)sfc;
-          // codes from p * (1 / sf): within an ulp of p / sf, so only a value
-          // on an e2m1 rounding boundary can round differently; a zero scale
-          // (an all-zero block) gives zero codes
-          const float r = (sc > 0.f) ? __frcp_rn(sc) : 0.f;
+          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(s[c][i0 + e]);
+        } else {
+          const uint64_t r2 = f2(rs[blk], rs[blk]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] *= r;
+          for (int e = 0; e < 16; e += 2)
+            f2_split(fmul2(f2(__uint_as_float(s[c][i0 + e]), __uint_as_float(s[c][i0 + e + 1])), r2), v[e], v[e + 1]);
         }
         uint32_t b[8];
 #pragma unroll
