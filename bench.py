@@ -393,8 +393,11 @@ def run_ours(args):
                 "frac": pn["rate"] / peak_tc, "traffic": traffic.get("fwd_bf16_prefill_noncausal"),
                 "kernel": "fwd_bf16_kernel<128>, prefill B4 H16 N4096 d128 non-causal",
                 "peak_source": f"{peak_src} bf16 burst"}
-    if "decode" in out_parts:
-        out_parts["decode"]["traffic"] = traffic.get("decode_split")
+    for part, key in (("decode", "decode_split"), ("lowp_int8", "fwd_int8_lowp"),
+                      ("lowp_fp4_direct_p", "fwd_fp4_direct_p_lowp"),
+                      ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp")):
+        if part in out_parts:
+            out_parts[part]["traffic"] = traffic.get(key)
     for nm in ("lowp_int8", "lowp_fp4_direct_p", "lowp_fp4_quant_after_exp"):
         if nm in out_parts:
             out_parts[nm]["peak_source"] = lowp_peak_src
