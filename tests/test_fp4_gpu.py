@@ -125,7 +125,8 @@ def _check_fp4(ta, q, k, v, causal, scale, mode, rows=None, what=""):
 
 @pytest.mark.parametrize("mode", [0, 1], ids=["direct_p", "quant_after_exp"])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("shape", [(1, 2, 128, 128), (1, 1, 300, 333), (2, 1, 129, 1000), (1, 1, 1, 1)],
+@pytest.mark.parametrize("shape", [(1, 2, 128, 128), (1, 1, 300, 333), (2, 1, 129, 1000), (1, 1, 1, 1),
+                                   (1, 1, 640, 200), (2, 2, 513, 129)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_fp4_forward_small(cuda_lib, shape, causal, mode):
     B, H, Nq, Nkv = shape

@@ -28,7 +28,9 @@
 //
 // Shared memory (128-byte swizzled, the TMA and UMMA canonical layout): each
 // 128 x D bf16 tile is stored as D/64 column blocks of 128 rows x 128 bytes.
-// Q0, Q1, then NSLOT ring slots holding K_0, V_0, K_1, V_1, ... in load order.
+// Q0, Q1, then a ring of NSTAGE stages; stage i holds V_{i-1} (first tile)
+// and K_i (second tile), the two operands a KV step consumes together, so
+// the MMA thread waits on one barrier per step.
 #pragma once
 #include "ptx.cuh"
 
@@ -57,16 +59,17 @@ struct FwdCfg {
   static constexpr int BR = 128, BC = 128;
   static constexpr int TILE = 128 * D * 2;       // bytes of one 128 x D bf16 tile
   static constexpr int HALF = 128 * 128;         // one 64-column block (128 rows x 128 B)
-  static constexpr int NSLOT = (D == 128) ? 5 : 10;
+  static constexpr int NSTAGE = (D == 128) ? 2 : 5;
+  static constexpr int STAGE = 2 * TILE;
   static constexpr int Q_OFF = 0;
   static constexpr int SLOT_OFF = 2 * TILE;
-  static constexpr int BAR_OFF = SLOT_OFF + NSLOT * TILE;
+  static constexpr int BAR_OFF = SLOT_OFF + NSTAGE * STAGE;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
-  // register split (launch: 384 threads x 168): warpgroup 0 drops to 56,
-  // the two softmax warpgroups rise to 224: 128*56 + 256*224 = 64512 = 384*168
-  static constexpr int REG_LOW = 56, REG_HIGH = 224;
+  // register split (launch: 384 threads x 168): warpgroup 0 drops to 80,
+  // the two softmax warpgroups rise to 208: 128*80 + 256*208 = 63488 <= 384*168
+  static constexpr int REG_LOW = 80, REG_HIGH = 208;
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);
   static constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
   static constexpr float TAU = 8.0f;  // lazy-rescale threshold, log2 units
@@ -76,8 +79,8 @@ struct FwdCfg {
 
 struct FwdBars {
   uint64_t q_full;
-  uint64_t kv_full[10];
-  uint64_t kv_empty[10];
+  uint64_t kv_full[5];
+  uint64_t kv_empty[5];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
@@ -134,7 +137,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
-    for (int s = 0; s < C::NSLOT; ++s) {
+    for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
       mbar_init(smem_u32(&bars->kv_empty[s]), 1);
     }
@@ -172,26 +175,27 @@ __global__ void __launch_bounds__(384, 1)
         for (int h = 0; h < D / 64; ++h)
           tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
       }
+      // stage i (0..nmax): V_{i-1} at +0 (none for i = 0), K_i at +TILE (none for i = nmax)
       int it = 0, slot = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int j = 0; j < nmax && ok; ++j) {
-        for (int w = 0; w < 2 && ok; ++w, ++it, (++slot == C::NSLOT) ? (slot = 0, ph ^= 1u) : 0u) {
-          ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
-          if (!ok) break;
-          const uint32_t fb = smem_u32(&bars->kv_full[slot]);
-          mbar_arrive_expect_tx(fb, C::TILE);
-          const uint32_t dst = sbase + C::SLOT_OFF + slot * C::TILE;
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(dst + h * C::HALF, w == 0 ? &tmK : &tmV, fb, h * 64, j * 128, bh);
+      for (int i = 0; nmax > 0 && i <= nmax && ok; ++i, ++it, (++slot == C::NSTAGE) ? (slot = 0, ph ^= 1u) : 0u) {
+        ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+        mbar_arrive_expect_tx(fb, ((i > 0) + (i < nmax)) * C::TILE);
+        const uint32_t dst = sbase + C::SLOT_OFF + slot * C::STAGE;
+        for (int h = 0; h < D / 64; ++h) {
+          if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, (i - 1) * 128, bh);
+          if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, i * 128, bh);
         }
       }
-      // Never leave a copy in flight: wait for the last load of every slot.
+      // Never leave a copy in flight: wait for the last load of every stage.
       if (!ok) {
         wait_bar_drain(qbar, 0, p.timeout_ns);
-        for (int back = 1; back <= C::NSLOT && it - back >= 0; ++back) {
+        for (int back = 1; back <= C::NSTAGE && it - back >= 0; ++back) {
           const int i2 = it - back;
-          wait_bar_drain(smem_u32(&bars->kv_full[i2 % C::NSLOT]), (i2 / C::NSLOT) & 1, p.timeout_ns);
+          wait_bar_drain(smem_u32(&bars->kv_full[i2 % C::NSTAGE]), (i2 / C::NSTAGE) & 1, p.timeout_ns);
         }
       }
     }
@@ -209,20 +213,12 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const uint64_t dQ0 = smem_desc(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dQ1 = smem_desc(sbase + C::Q_OFF + C::TILE, 16, 1024);
-      const uint64_t dK0 = smem_desc(sbase + C::SLOT_OFF, 16, 1024);
       const uint64_t dV0 = smem_desc(sbase + C::SLOT_OFF, C::HALF, 1024);
-      // K_j is load number 2j, V_j number 2j+1 (slot = number % NSLOT,
-      // phase = (number / NSLOT) & 1)
-      int sK = 0, sV = 1 % C::NSLOT;
-      uint32_t pK = 0, pV = (1 >= C::NSLOT) ? 1u : 0u;
-      auto adv = [&](int& sl, uint32_t& ph) {
-        sl += 2;
-        if (sl >= C::NSLOT) { sl -= C::NSLOT; ph ^= 1u; }
-      };
-      // Issue one S group; before its last MMA, test barrier (nb, np).
-      auto issue_S = [&](int t, int sl, uint32_t nb, uint32_t np) -> bool {
+      const uint64_t dK0 = smem_desc(sbase + C::SLOT_OFF + C::TILE, 16, 1024);
+      // Issue one S group (K in stage st); before its last MMA, test barrier (nb, np).
+      auto issue_S = [&](int t, int st, uint32_t nb, uint32_t np) -> bool {
         const uint64_t dq = t ? dQ1 : dQ0;
-        const uint64_t dk = dK0 + (uint64_t)(sl * (C::TILE >> 4));
+        const uint64_t dk = dK0 + (uint64_t)(st * (C::STAGE >> 4));
         const uint32_t dS = tbase + t * 128;
         bool ready = true;
 #pragma unroll
@@ -234,8 +230,8 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(smem_u32(&bars->s_full[t]));
         return ready;
       };
-      auto issue_PV = [&](int t, int sl, int j, uint32_t nb, uint32_t np) -> bool {
-        const uint64_t dv = dV0 + (uint64_t)(sl * (C::TILE >> 4));
+      auto issue_PV = [&](int t, int st, int j, uint32_t nb, uint32_t np) -> bool {
+        const uint64_t dv = dV0 + (uint64_t)(st * (C::STAGE >> 4));
         const uint32_t dO = tbase + 256 + t * D, aP = tbase + t * 128;
         const uint32_t acc0 = (j > 0) ? 1u : 0u;
         bool ready = true;
@@ -253,55 +249,46 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       const uint32_t pf0 = smem_u32(&bars->p_full[0]), pf1 = smem_u32(&bars->p_full[1]);
+      int st = 0;        // stage of the current step (slot), its phase
+      uint32_t sp = 0;
       if (ok && nmax > 0) {
-        ok = wait_bar(smem_u32(&bars->kv_full[sK]), pK, abort_flag, p.timeout_ns);
+        ok = wait_bar(smem_u32(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns);
         tc_fence_after();
         if (ok) {
-          if (n[0] > 0) issue_S(0, sK, 0, 0);
-          if (n[1] > 0) issue_S(1, sK, 0, 0);
-          tc_commit(smem_u32(&bars->kv_empty[sK]));
+          if (n[0] > 0) issue_S(0, 0, 0, 0);
+          if (n[1] > 0) issue_S(1, 0, 0, 0);
+          tc_commit(smem_u32(&bars->kv_empty[0]));
         }
       }
       if (ok) {
         for (int t = 0; t < 2; ++t)
           if (present[t] && n[t] == 0) tc_commit(smem_u32(&bars->o_full[t]));
       }
-      bool seenV = false;
+      // step j uses stage j + 1: V_j for both P V groups, K_{j+1} for the next S
+      bool seenSt = false;
       for (int j = 0; j < nmax && ok; ++j) {
-        // V_j is needed by both P V groups of this step
-        if (!(ok = need(seenV, smem_u32(&bars->kv_full[sV]), pV))) break;
-        const bool nextK = j + 1 < nmax;
-        int sK1 = sK;
-        uint32_t pK1 = pK;
-        if (nextK) adv(sK1, pK1);
-        const uint32_t kbar = nextK ? smem_u32(&bars->kv_full[sK1]) : 0u;
-        bool seenK = !nextK;
+        if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
+        if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
+        int st1 = st + 1;
+        uint32_t sp1 = sp;
+        if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }
+        const uint32_t nbar = (j + 1 < nmax) ? smem_u32(&bars->kv_full[st1]) : 0u;
+        bool seenP1 = false;
         if (j < n[0]) {
           if (!(ok = need(false, pf0, j & 1))) break;
-          seenK = issue_PV(0, sV, j, kbar, pK1) || !nextK;
+          seenP1 = issue_PV(0, st, j, (j < n[1]) ? pf1 : 0u, j & 1);
           if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
         }
-        if (nextK) {
-          if (!(ok = need(seenK, kbar, pK1))) break;
-        }
-        bool seenP1 = false;
-        if (j + 1 < n[0]) seenP1 = issue_S(0, sK1, (j < n[1]) ? pf1 : 0u, j & 1);
+        if (j + 1 < n[0]) seenP1 = issue_S(0, st, (!seenP1 && j < n[1]) ? pf1 : 0u, j & 1) || seenP1;
+        seenSt = false;
         if (j < n[1]) {
           if (!(ok = need(seenP1, pf1, j & 1))) break;
-          issue_PV(1, sV, j, 0, 0);
+          seenSt = issue_PV(1, st, j, nbar, sp1);
           if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
         }
-        tc_commit(smem_u32(&bars->kv_empty[sV]));
-        int sV1 = sV;
-        uint32_t pV1 = pV;
-        adv(sV1, pV1);
-        seenV = false;
-        if (j + 1 < n[1]) seenV = issue_S(1, sK1, (j + 1 < nmax) ? smem_u32(&bars->kv_full[sV1]) : 0u, pV1);
-        if (nextK) tc_commit(smem_u32(&bars->kv_empty[sK1]));
-        sK = sK1;
-        pK = pK1;
-        sV = sV1;
-        pV = pV1;
+        if (j + 1 < n[1]) seenSt = issue_S(1, st, seenSt ? 0u : nbar, sp1) || seenSt;
+        seenSt = seenSt && nbar;
+        tc_commit(smem_u32(&bars->kv_empty[st]));
       }
       if (!ok) {
         // drain: every MMA issued so far must finish before TMEM is freed
