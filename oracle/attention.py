@@ -87,6 +87,25 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None,
     return O, LSE
 
 
+def kv_head_index(Hq: int, Hkv: int) -> np.ndarray:
+    """Key/value head of every query head under grouped-query attention:
+    query head h reads key/value head h // (Hq / Hkv) ([FA4-overview]
+    "Compatibility and current status": several attention heads share one
+    key/value projection; Hkv = 1 is multi-query attention, Hkv = Hq plain
+    multi-head attention)."""
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return np.arange(Hq) // (Hq // Hkv)
+
+
+def attention_gqa(q, k, v, causal: bool = False, scale: float | None = None, rows=None):
+    """Grouped-query attention: the plain definition with each query head's
+    key/value head substituted (q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    idx = kv_head_index(q.shape[1], k.shape[1])
+    return attention(q, k[:, idx], v[:, idx], causal, scale, rows=rows)
+
+
 def softmax_rows(q, k, causal: bool = False, scale: float | None = None):
     """The normalised probability matrix P [B,H,Nq,Nkv] (small inputs only)."""
     q, k = _f64(q), _f64(k)

@@ -190,3 +190,43 @@ def test_bf16_inputs_convert_exactly():
     O2, _ = A.attention(t.float().numpy().astype(np.float64), t.float().numpy(), t.float().numpy(),
                         False, 0.1)
     assert np.array_equal(O, O2)
+
+
+# ---------------------------------------------------------------- GQA / MQA
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 1), (6, 3), (3, 3)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_matches_torch_sdpa_enable_gqa(Hq, Hkv, causal):
+    """Pin against PyTorch's own grouped-query SDPA (fp64 on CPU), an
+    implementation independent of the head-index substitution."""
+    g = torch.Generator().manual_seed(Hq * 10 + Hkv)
+    B, Nq, Nkv, d = 2, 7, 11 if not causal else 7, 5
+    q = torch.randn(B, Hq, Nq, d, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, Nkv, d, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, Nkv, d, generator=g, dtype=torch.float64)
+    O, _ = A.attention_gqa(q, k, v, causal, 0.4)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=0.4,
+                                                           enable_gqa=True)
+    assert np.abs(O - ref.numpy()).max() < 1e-12
+
+
+def test_mqa_heads_share_one_kv_head():
+    """Hkv = 1: every query head attends to the same keys and values, so two
+    query heads with equal queries give equal outputs, and each head equals a
+    single-head call with that head's queries."""
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(1, 4, 6, 8, generator=g, dtype=torch.float64)
+    q[:, 3] = q[:, 1]
+    k = torch.randn(1, 1, 9, 8, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 1, 9, 8, generator=g, dtype=torch.float64)
+    O, L = A.attention_gqa(q, k, v, False, 0.3)
+    assert np.array_equal(O[:, 3], O[:, 1]) and np.array_equal(L[:, 3], L[:, 1])
+    for h in range(4):
+        Oh, Lh = A.attention(q[:, h:h + 1], k, v, False, 0.3)
+        assert np.array_equal(O[:, h:h + 1], Oh) and np.array_equal(L[:, h:h + 1], Lh)
+
+
+def test_kv_head_index_groups_and_rejects_uneven():
+    assert A.kv_head_index(8, 2).tolist() == [0, 0, 0, 0, 1, 1, 1, 1]
+    assert A.kv_head_index(4, 4).tolist() == [0, 1, 2, 3]
+    with pytest.raises(ValueError):
+        A.kv_head_index(6, 4)
