@@ -6,7 +6,9 @@ A step is one pass of the hot path over the seeded synthetic workloads:
   * prefill  B=4 H=16 N=4096 d=128 bf16: attn_fwd non-causal + attn_fwd causal
              (the headline: attention forward TFLOP/s, 4*B*H*N*N*d, halved
              for causal);
-  * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine
+  * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine; and
+             the same with grouped-query attention (8 cache heads, 4 query
+             heads each: 2.1 GB of cache);
              (KV-read GB/s against HBM);
   * longseq  B=1 H=12 N=23400 d=64 bf16, non-causal + causal;
   * lowp     B=2 H=24 N=8192 d=128 with outlier channels: bf16 forward, INT8
@@ -244,6 +246,11 @@ def run_ours(args):
                           dtype=torch.uint8, device=dev)
         seg("decode", lambda: ta.attn_decode(dq, dk, dv, do, dlse, wd.scale, wd.num_splits, dws, stream),
             2 * dk.numel() * dk.element_size(), "GB/s", peak_hbm, "hbm", 2)
+        # grouped-query decode: 4 query heads per cache head (the same queries,
+        # the first H/4 cache heads); GB/s counts the cache bytes it must read
+        gk, gv = dk[:, :wd.H // 4].contiguous(), dv[:, :wd.H // 4].contiguous()
+        seg("decode_gqa", lambda: ta.attn_decode_gqa(dq, gk, gv, do, dlse, wd.scale, wd.num_splits, dws, stream),
+            2 * gk.numel() * gk.element_size(), "GB/s", peak_hbm, "hbm", 2)
     wl = WORKLOADS["longseq"]
     if "longseq" in parts:
         lq, lk, lv = (t.to(dev) for t in make_qkv(wl, seed=0))

@@ -91,6 +91,21 @@ ATTN_API int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf1
              void* stream);
 
 /*
+ * attn_fwd_gqa -- attn_fwd with grouped-query / multi-query attention:
+ * Hq query heads share Hkv key/value heads, query head h reading key/value
+ * head h / (Hq / Hkv) ([FA4-overview] "Compatibility and current status":
+ * several attention heads use the same key/value projection, to save memory;
+ * Hkv = 1 is multi-query attention, Hkv = Hq is attn_fwd).
+ *
+ *   q [B][Hq][Nq][d] bf16, k, v [B][Hkv][Nkv][d] bf16, o [B][Hq][Nq][d] bf16
+ *   out, lse [B][Hq][Nq] fp32 out; Hkv >= 1 and Hq % Hkv == 0, else
+ *   ATTN_ERR_INVALID_ARG.  Everything else as attn_fwd.
+ */
+ATTN_API int attn_fwd_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                          float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                          void* stream);
+
+/*
  * attn_decode -- split-KV decode: ONE query row per (batch, head) against a
  * KV cache of Nkv keys; the key range is cut into num_splits equal chunks of
  * ceil(Nkv / num_splits) keys, each chunk gives a partial (O_c, LSE_c) in the
@@ -110,6 +125,21 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits)
 ATTN_API int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
                 float* lse, int B, int H, int Nkv, int d, float scale, int num_splits,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_decode_gqa -- attn_decode with Hq query heads sharing Hkv key/value
+ * heads (query head h reads cache head h / (Hq / Hkv), as attn_fwd_gqa).
+ * The query heads of a group are scheduled together, so the cache of a
+ * key/value head crosses HBM once for the whole group.
+ *
+ *   q [B][Hq][1][d], k, v [B][Hkv][Nkv][d], o [B][Hq][1][d], lse [B][Hq];
+ *   workspace: attn_decode_workspace_bytes(B, Hq, d, num_splits) bytes.
+ *   Hkv >= 1 and Hq % Hkv == 0, else ATTN_ERR_INVALID_ARG; everything else as
+ *   attn_decode.
+ */
+ATTN_API int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                             float* lse, int B, int Hq, int Hkv, int Nkv, int d, float scale, int num_splits,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * attn_decode_noalloc -- the same split-KV decode as attn_decode, for callers

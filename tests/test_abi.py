@@ -78,6 +78,19 @@ def test_decode_workspace_size_and_validation(lib):
     assert call(B=0) == 0
 
 
+@pytest.mark.parametrize("Hq,Hkv,code", [(8, 3, -1), (8, 0, -1), (4, 8, -1), (8, 2, None), (8, 8, None), (8, 1, None)])
+def test_gqa_head_validation(lib, Hq, Hkv, code):
+    """Uneven head groups are rejected before anything touches the device;
+    valid groups pass validation (checked with d = 96, which then fails as
+    unsupported, so nothing is launched)."""
+    rc = lib.attn_fwd_gqa(P, P, P, P, P, 1, Hq, Hkv, 8, 8, 64 if code else 96, 0, 0.125, None)
+    assert rc == (code if code else -2)
+    n = lib.attn_decode_workspace_bytes(1, Hq, 128, 4)
+    rc = lib.attn_decode_gqa(P, P, P, P, P, 1, Hq, Hkv, 100, 128 if code else 96, 0.1, 4,
+                             ctypes.c_void_p(16 * 4096), n, None)
+    assert rc == (code if code else -2)
+
+
 def test_product_path_never_imports_the_oracle():
     """The package must not reach the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "tiled_attention_24_b200")

@@ -11,7 +11,8 @@ import math
 import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
-                       attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores, attn_fwd,
+                       attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
+                       attn_fwd, attn_fwd_gqa,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
                        attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
                        attn_status_string, attn_version, attn_watchdog_selftest, load)
@@ -21,25 +22,30 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "AttnError", "forward", "decode", "quantize_int8", "forward_int8",
            "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc",
            "attn_quantize_nvfp4", "attn_fwd_fp4", "attn_fp4_scores", "quantize_nvfp4", "forward_fp4",
-           "DIRECT_P", "QUANT_AFTER_EXP"]
+           "attn_fwd_gqa", "attn_decode_gqa", "DIRECT_P", "QUANT_AFTER_EXP"]
 
 DIRECT_P, QUANT_AFTER_EXP = 0, 1
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
             scale: float | None = None, stream=None):
-    """Allocate O (bf16) and LSE (fp32) and run ``attn_fwd``."""
+    """Allocate O (bf16) and LSE (fp32) and run ``attn_fwd`` (``attn_fwd_gqa``
+    when k/v have fewer heads than q: grouped-query attention)."""
     B, H, Nq, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    attn_fwd(q, k, v, o, lse, causal, scale, stream)
+    if k.shape[1] != H:
+        attn_fwd_gqa(q, k, v, o, lse, causal, scale, stream)
+    else:
+        attn_fwd(q, k, v, o, lse, causal, scale, stream)
     return o, lse
 
 
 def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
            num_splits: int = 16, workspace: torch.Tensor | None = None, stream=None):
-    """Allocate O, LSE (and a workspace if none is given) and run ``attn_decode``."""
+    """Allocate O, LSE (and a workspace if none is given) and run ``attn_decode``
+    (``attn_decode_gqa`` when k/v have fewer heads than q)."""
     B, H, _, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if workspace is None:
@@ -47,7 +53,10 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | Non
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
-    attn_decode(q, k, v, o, lse, scale, num_splits, workspace, stream)
+    if k.shape[1] != H:
+        attn_decode_gqa(q, k, v, o, lse, scale, num_splits, workspace, stream)
+    else:
+        attn_decode(q, k, v, o, lse, scale, num_splits, workspace, stream)
     return o, lse
 
 

@@ -30,6 +30,8 @@ SIGNATURES = [
     ("attn_decode_workspace_bytes", _SZ, [_I, _I, _I, _I]),
     ("attn_decode", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_decode_noalloc", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP]),
+    ("attn_fwd_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    ("attn_decode_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_fwd_int8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_int8_scores", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
@@ -100,6 +102,27 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
     rc = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nkv, d, int(bool(causal)),
                          float(scale), _stream(stream))
     _check("attn_fwd", rc)
+
+
+def attn_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """Grouped-query forward: q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d] (Hq % Hkv == 0)."""
+    _need_cuda(q, k, v, o, lse)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    rc = load().attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nkv, d,
+                             int(bool(causal)), float(scale), _stream(stream))
+    _check("attn_fwd_gqa", rc)
+
+
+def attn_decode_gqa(q, k, v, o, lse, scale: float, num_splits: int, workspace, stream=None):
+    """Grouped-query split-KV decode: q [B,Hq,1,d], k/v [B,Hkv,Nkv,d]."""
+    _need_cuda(q, k, v, o, lse, workspace)
+    B, Hq, _, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    rc = load().attn_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nkv, d, float(scale),
+                                int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _check("attn_decode_gqa", rc)
 
 
 def attn_decode_workspace_bytes(B: int, H: int, d: int, num_splits: int) -> int:

@@ -168,15 +168,15 @@ int set_smem_attr(K kernel, int bytes) {
 }
 
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nkv,
-               int causal, float scale, cudaStream_t st) {
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int Nq,
+               int Nkv, int causal, float scale, cudaStream_t st) {
   using C = ta::FwdCfg<D>;
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
   int rc;
   if ((rc = make_tmap_bf16(&tq, q, D, Nq, BH)) != ATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&tk, k, D, Nkv, BH)) != ATTN_OK) return rc;
-  if ((rc = make_tmap_bf16(&tv, v, D, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, D, Nkv, B * Hkv)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, D, Nkv, B * Hkv)) != ATTN_OK) return rc;
   if ((rc = make_tmap_bf16(&to, o, D, Nq, BH)) != ATTN_OK) return rc;
   if ((rc = set_smem_attr(ta::fwd_bf16_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
   ta::FwdParams p;
@@ -185,6 +185,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.Nkv = Nkv;
   p.n_qp = (Nq + 255) / 256;
   p.Tc = (Nkv + 127) / 128;
+  p.group = H / Hkv;
   p.causal = causal ? 1 : 0;
   p.sl2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_ns;
@@ -260,9 +261,10 @@ const char* attn_version(void) { return "tiledattn 0.1 sm_100a"; }
 
 void attn_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
 
-int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
-             int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
+int attn_fwd_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+                 int B, int H, int Hkv, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
   if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv < 1 || (H > 0 && H % Hkv != 0) || Hkv > (H > 0 ? H : Hkv)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
@@ -279,8 +281,13 @@ int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, a
     ta::fill_empty_kernel<<<(unsigned)blocks, 256, 0, st>>>(o, lse, rows, d);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
-  return d == 128 ? launch_fwd<128>(q, k, v, o, lse, B, H, Nq, Nkv, causal, scale, st)
-                  : launch_fwd<64>(q, k, v, o, lse, B, H, Nq, Nkv, causal, scale, st);
+  return d == 128 ? launch_fwd<128>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, causal, scale, st)
+                  : launch_fwd<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, causal, scale, st);
+}
+
+int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+             int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
+  return attn_fwd_gqa(q, k, v, o, lse, B, H, H > 0 ? H : 1, Nq, Nkv, d, causal, scale, stream);
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
@@ -288,10 +295,11 @@ size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
   return decode_ws_bytes((long long)B * H, d, num_splits);
 }
 
-int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
-                int B, int H, int Nkv, int d, float scale, int num_splits, void* workspace,
-                size_t workspace_bytes, void* stream) {
+int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                    float* lse, int B, int H, int Hkv, int Nkv, int d, float scale, int num_splits,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 0 || H < 0 || Nkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hkv < 1 || (H > 0 && H % Hkv != 0) || Hkv > (H > 0 ? H : Hkv)) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -309,17 +317,41 @@ int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v
                                            (((size_t)BH * num_splits * d * sizeof(float) + 255) & ~size_t(255)));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float sl2 = scale * 1.4426950408889634f;
-  const unsigned grid = (unsigned)(BH * num_splits);
-  if (d == 128) {
-    ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                    chunk, sl2);
-    ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  // query heads per CTA: the largest of 8, 4, 2 dividing the group (each
+  // cache row then crosses memory once per G query heads); 1 = plain kernel
+  const int grp = H / Hkv;
+  const int G = (grp % 8 == 0) ? 8 : (grp % 4 == 0) ? 4 : (grp % 2 == 0) ? 2 : 1;
+  const unsigned grid = (unsigned)(BH / G * num_splits);
+  if (G == 1) {
+    if (d == 128)
+      ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits, chunk,
+                                                                      sl2, grp);
+    else
+      ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits, chunk,
+                                                                     sl2, grp);
   } else {
-    ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                   chunk, sl2);
-    ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
+#define TA_DECODE_GROUP(DD, GG)                                                                           \
+  ta::decode_split_group_kernel<DD, GG><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, \
+                                                                         num_splits, chunk, sl2, grp)
+    if (d == 128) {
+      if (G == 8) TA_DECODE_GROUP(128, 8); else if (G == 4) TA_DECODE_GROUP(128, 4); else TA_DECODE_GROUP(128, 2);
+    } else {
+      if (G == 8) TA_DECODE_GROUP(64, 8); else if (G == 4) TA_DECODE_GROUP(64, 4); else TA_DECODE_GROUP(64, 2);
+    }
+#undef TA_DECODE_GROUP
   }
+  if (d == 128)
+    ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
+  else
+    ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+                int B, int H, int Nkv, int d, float scale, int num_splits, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  return attn_decode_gqa(q, k, v, o, lse, B, H, H > 0 ? H : 1, Nkv, d, scale, num_splits, workspace,
+                         workspace_bytes, stream);
 }
 
 int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
@@ -347,11 +379,11 @@ int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_b
   const unsigned grid = (unsigned)(BH * num_splits);
   if (d == 128) {
     ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                    chunk, sl2);
+                                                                    chunk, sl2, 1);
     ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
   } else {
     ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                   chunk, sl2);
+                                                                   chunk, sl2, 1);
     ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -49,6 +49,7 @@ namespace ta {
 struct FwdParams {
   float* lse;
   int Nq, Nkv, n_qp, Tc;
+  int group;  // query heads per key/value head (grouped-query attention; 1 = plain)
   int causal;
   float sl2;  // scale * log2(e)
   unsigned long long timeout_ns;
@@ -175,6 +176,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int h = 0; h < D / 64; ++h)
           tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
       }
+      const int kvh = bh / p.group;  // key/value head of this query head
       // stage i (0..nmax): V_{i-1} at +0 (none for i = 0), K_i at +TILE (none for i = nmax)
       int it = 0, slot = 0;
       uint32_t ph = 0;
@@ -186,8 +188,8 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(fb, ((i > 0) + (i < nmax)) * C::TILE);
         const uint32_t dst = sbase + C::SLOT_OFF + slot * C::STAGE;
         for (int h = 0; h < D / 64; ++h) {
-          if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, (i - 1) * 128, bh);
-          if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, i * 128, bh);
+          if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, (i - 1) * 128, kvh);
+          if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, i * 128, kvh);
         }
       }
       // Never leave a copy in flight: wait for the last load of every stage.
