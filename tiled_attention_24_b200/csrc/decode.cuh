@@ -28,6 +28,9 @@ namespace ta {
 constexpr int DEC_THREADS = 128;
 constexpr int DEC_SB = 512;  // keys per sub-block
 constexpr int DEC_UNROLL = 8;
+// grouped kernel: loads in flight per lane, by heads per CTA (measured on
+// B200 with B64 Hq32 N_kv 8192: G = 4 is fastest with 4, G = 8 with 8)
+__host__ __device__ constexpr int dec_group_unroll(int G) { return G == 4 ? 4 : 8; }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
@@ -188,17 +191,17 @@ __global__ void __launch_bounds__(DEC_THREADS)
 // by G ([FA4-overview] "Compatibility and current status": several heads
 // share one key/value projection).  Same lane layout and sub-block online
 // softmax as decode_split_kernel, with G scores per key.
-template <int D, int G>
-__global__ void __launch_bounds__(DEC_THREADS)
+template <int D, int G, int NT = DEC_THREADS, int UNR = dec_group_unroll(G)>
+__global__ void __launch_bounds__(NT)
     decode_split_group_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                               const uint16_t* __restrict__ v, float* __restrict__ o_part,
                               float* __restrict__ lse_part, int Nkv, int S, int chunk, float sl2, int group) {
   constexpr int LPK = D / 8;
   constexpr int KPW = 32 / LPK;
-  constexpr int NW = DEC_THREADS / 32;
+  constexpr int NW = NT / 32;
   constexpr int PER_WARP = DEC_SB / NW;
-  constexpr int STEPS = PER_WARP / (KPW * DEC_UNROLL);
-  static_assert(PER_WARP % (KPW * DEC_UNROLL) == 0, "sub-block split");
+  constexpr int STEPS = PER_WARP / (KPW * UNR);
+  static_assert(PER_WARP % (KPW * UNR) == 0, "sub-block split");
 
   __shared__ float xs[G][DEC_SB];
   __shared__ float red[NW][D];
@@ -238,15 +241,15 @@ __global__ void __launch_bounds__(DEC_THREADS)
     // ---- 1. G scores per key of this sub-block
 #pragma unroll 1
     for (int st = 0; st < STEPS; ++st) {
-      uint4 kr[DEC_UNROLL];
+      uint4 kr[UNR];
 #pragma unroll
-      for (int u = 0; u < DEC_UNROLL; ++u) {
-        const int kk = warp * PER_WARP + (st * DEC_UNROLL + u) * KPW + sub;
+      for (int u = 0; u < UNR; ++u) {
+        const int kk = warp * PER_WARP + (st * UNR + u) * KPW + sub;
         kr[u] = (kk < ns) ? ldg_stream(kb + (size_t)(s0 + kk) * D) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < DEC_UNROLL; ++u) {
-        const int kk = warp * PER_WARP + (st * DEC_UNROLL + u) * KPW + sub;
+      for (int u = 0; u < UNR; ++u) {
+        const int kk = warp * PER_WARP + (st * UNR + u) * KPW + sub;
         const float k0 = bf_lo(kr[u].x), k1 = bf_hi(kr[u].x), k2 = bf_lo(kr[u].y), k3 = bf_hi(kr[u].y);
         const float k4 = bf_lo(kr[u].z), k5 = bf_hi(kr[u].z), k6 = bf_lo(kr[u].w), k7 = bf_hi(kr[u].w);
 #pragma unroll
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       mx[g] = -INFINITY;
-      for (int i = threadIdx.x; i < DEC_SB; i += DEC_THREADS) mx[g] = fmaxf(mx[g], xs[g][i]);
+      for (int i = threadIdx.x; i < DEC_SB; i += NT) mx[g] = fmaxf(mx[g], xs[g][i]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
       if (lane == 0) wred[warp][g] = mx[g];
@@ -287,7 +290,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       factor[g] = ex2(m_run[g] - m_new);           // 0 on the first sub-block
       m_run[g] = m_new;
       ps[g] = 0.f;
-      for (int i = threadIdx.x; i < DEC_SB; i += DEC_THREADS) {
+      for (int i = threadIdx.x; i < DEC_SB; i += NT) {
         const float pv = ex2(xs[g][i] - m_new);      // -inf -> 0
         xs[g][i] = pv;
         ps[g] += pv;
@@ -313,15 +316,15 @@ __global__ void __launch_bounds__(DEC_THREADS)
     // ---- 3. values: each V row once, for all G heads
 #pragma unroll 1
     for (int st = 0; st < STEPS; ++st) {
-      uint4 vr[DEC_UNROLL];
+      uint4 vr[UNR];
 #pragma unroll
-      for (int u = 0; u < DEC_UNROLL; ++u) {
-        const int kk = warp * PER_WARP + (st * DEC_UNROLL + u) * KPW + sub;
+      for (int u = 0; u < UNR; ++u) {
+        const int kk = warp * PER_WARP + (st * UNR + u) * KPW + sub;
         vr[u] = (kk < ns) ? ldg_stream(vb + (size_t)(s0 + kk) * D) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < DEC_UNROLL; ++u) {
-        const int kk = warp * PER_WARP + (st * DEC_UNROLL + u) * KPW + sub;
+      for (int u = 0; u < UNR; ++u) {
+        const int kk = warp * PER_WARP + (st * UNR + u) * KPW + sub;
         const float v0 = bf_lo(vr[u].x), v1 = bf_hi(vr[u].x), v2 = bf_lo(vr[u].y), v3 = bf_hi(vr[u].y);
         const float v4 = bf_lo(vr[u].z), v5 = bf_hi(vr[u].z), v6 = bf_lo(vr[u].w), v7 = bf_hi(vr[u].w);
 #pragma unroll
@@ -354,7 +357,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
     __syncthreads();
     const size_t part = (size_t)(bh0 + g) * S + c;
-    for (int e = threadIdx.x; e < D; e += DEC_THREADS) {
+    for (int e = threadIdx.x; e < D; e += NT) {
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < NW; ++w) sum += red[w][e];
