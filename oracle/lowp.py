@@ -70,6 +70,22 @@ def quantize_int8_rows(x):
     return q, s
 
 
+def quantize_int4_rows(x):
+    """Symmetric INT4 with one fp32 scale per row, the token-level scheme at 4
+    bits ([INT-FA]: the token-level quantisation carries over to lower
+    formats such as INT4): s = amax / 7 in fp32, q = clamp(rne(x / s), -7, 7)
+    with an IEEE fp32 divide, amax == 0 gives s = 1 and q = 0.  The codes are
+    returned in int8 containers (the INT8 forward consumes them unchanged).
+    Returns (q int8 in [-7, 7], s float32)."""
+    xf = _f64(x).astype(F32)
+    amax = np.abs(xf).max(axis=-1)
+    s = (amax / F32(7.0)).astype(F32)
+    s = np.where(amax == 0, F32(1.0), s).astype(F32)
+    qf = np.rint((xf / s[..., None]).astype(F32))
+    q = np.clip(qf, -7, 7).astype(np.int8)
+    return q, s
+
+
 def quantize_int8_heads(x):
     """Symmetric INT8 with one fp32 scale per (batch, head) of a [B,H,N,d]
     tensor (the V operand).  Same formula as ``quantize_int8_rows``."""

@@ -7,6 +7,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import attention as A
 from oracle import lowp as Q
@@ -280,3 +281,44 @@ def test_fp4_single_visible_key():
     for mode in (Q.DIRECT_P, Q.QUANT_AFTER_EXP):
         O, _ = Q.attention_fp4(qd, kd, vd, mode, True, 0.3)
         np.testing.assert_allclose(O[0, :, 0], vd[0, :, 0], atol=1e-12)
+
+
+# ---------------------------------------------------------------- INT4 Q/K
+def test_int4_rows_identity_on_integer_rows_with_amax_7():
+    """Rows of integers in [-7, 7] whose amax is 7: s = 7 / 7 = 1 exactly, so
+    quantisation is the identity."""
+    g = np.random.default_rng(4)
+    x = g.integers(-7, 8, size=(3, 5, 16)).astype(np.float32)
+    x[..., 0] = 7.0
+    q, s = Q.quantize_int4_rows(torch.tensor(x).to(torch.bfloat16))
+    assert (s == 1.0).all() and np.array_equal(q.astype(np.float32), x)
+
+
+def test_int4_rows_zero_row_error_bound_and_range():
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(2, 3, 40, 64, generator=g).to(torch.bfloat16)
+    x[0, 0, 3] = 0
+    q, s = Q.quantize_int4_rows(x)
+    assert q[0, 0, 3].tolist() == [0] * 64 and s[0, 0, 3] == 1.0
+    assert q.min() >= -7 and q.max() <= 7
+    xf = x.double().numpy()
+    err = np.abs(xf - q.astype(np.float64) * s[..., None].astype(np.float64))
+    assert (err <= 0.5 * s[..., None] * (1 + 1e-6)).all()
+    # every row uses the full range: its largest magnitude maps to +-7
+    assert (np.abs(q).max(axis=-1)[s != 1.0] == 7).all()
+
+
+def test_int4_emulation_drifts_more_than_int8_but_stays_close():
+    """The same emulated forward with INT4 Q/K: further from the exact
+    attention than with INT8 Q/K, still close on N(0,1) inputs."""
+    g = torch.Generator().manual_seed(9)
+    q, k, v = (torch.randn(1, 2, 96, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    Oe, _ = A.attention(q, k, v, False, 0.125)
+    vi, vs = Q.quantize_int8_heads(v)
+    errs = []
+    for quant in (Q.quantize_int8_rows, Q.quantize_int4_rows):
+        qi, qs = quant(q)
+        ki, ks = quant(k)
+        O, _ = Q.attention_int8(qi, qs, ki, ks, vi, vs, False, 0.125)
+        errs.append(np.abs(O - Oe).max())
+    assert errs[0] < errs[1] < 0.25
