@@ -188,6 +188,19 @@ ATTN_API int attn_quantize_int8(const attn_bf16_t* x, int8_t* xq, float* xs, int
                                 int per_head, void* stream);
 
 /*
+ * attn_quantize_int4 -- token-level INT4 quantisation of Q or K ([INT-FA]:
+ * the token-level scheme carries over to lower formats such as 4-bit
+ * integers): one scale per token row, s = amax / 7 (IEEE fp32 divide;
+ * amax == 0 gives s = 1), xq = clamp(rne(x / s), -7, 7), stored one code per
+ * byte (int8 containers: attn_fwd_int8 consumes them unchanged, with V
+ * quantised by attn_quantize_int8 per head).
+ *   x bf16 [B][H][N][d] 16-byte aligned, xq int8 [B][H][N][d] 16-byte aligned,
+ *   xs fp32 [B][H][N]; d in {64, 128}.
+ */
+ATTN_API int attn_quantize_int4(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H, int N, int d,
+                                void* stream);
+
+/*
  * attn_fwd_int8 -- INT8 attention forward ([INT-FA]: INT8 GEMMs for Q K^T and
  * P V inside the FlashAttention forward, int32 accumulation):
  *   S = q_i8 . k_i8 (int32, exact); x = S * q_scale[i] * k_scale[j] * scale;

@@ -50,16 +50,27 @@ def test_int8_scores_bit_exact(cuda_lib, Nq, Nkv):
     assert np.array_equal(_np(s), Q.int8_scores(qi.numpy(), ki.numpy()))
 
 
-def _check_int8(ta, q, k, v, causal, scale, rows=None, what=""):
-    qi, qs = ta.quantize_int8(q.cuda(), False)
-    ki, ks = ta.quantize_int8(k.cuda(), False)
+def _check_int8(ta, q, k, v, causal, scale, rows=None, what="", int4=False):
+    """The device quantises and runs the forward; the oracle quantises the same
+    bf16 inputs itself (its quantisers are bit-exact with the device's, checked
+    separately) and emulates the forward."""
+    if int4:
+        qi, qs = ta.quantize_int4(q.cuda())
+        ki, ks = ta.quantize_int4(k.cuda())
+    else:
+        qi, qs = ta.quantize_int8(q.cuda(), False)
+        ki, ks = ta.quantize_int8(k.cuda(), False)
     vi, vs = ta.quantize_int8(v.cuda(), True)
     B, H, Nq, d = q.shape
     o = torch.empty((B, H, Nq, d), dtype=torch.float32, device="cuda")
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
     ta.attn_fwd_int8(qi, qs, ki, ks, vi, vs, o, lse, causal, scale)
     assert ta.attn_check_status() == 0
-    O, L, FB, LB, flips = Q.attention_int8(_np(qi), _np(qs), _np(ki), _np(ks), _np(vi), _np(vs), causal, scale,
+    quant = Q.quantize_int4_rows if int4 else Q.quantize_int8_rows
+    rqi, rqs = quant(q)
+    rki, rks = quant(k)
+    rvi, rvs = Q.quantize_int8_heads(v)
+    O, L, FB, LB, flips = Q.attention_int8(rqi, rqs, rki, rks, rvi, rvs, causal, scale,
                                            with_flip_bound=True, rows=rows)
     og, lg = _np(o).astype(np.float64), _np(lse).astype(np.float64)
     if rows is not None:
@@ -97,3 +108,33 @@ def test_int8_full_lowp_workload_sampled_rows(cuda_lib):
     rows = np.array(sorted({0, 1, 127, 128, 4095, 8190, 8191} | set(np.random.default_rng(0).choice(8192, 24).tolist())))
     _, flips, cos = _check_int8(cuda_lib, q, k, v, False, w.scale, rows=rows, what="lowp full")
     assert cos > 0.99
+
+
+# ---------------------------------------------------------------- INT4 Q/K
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("name", ["prefill", "lowp"])
+def test_int4_quantiser_bit_exact(cuda_lib, name, d):
+    q, _, _ = make_qkv(name, seed=13, B=2, H=3, Nq=300, Nkv=1, d=d)
+    q[0, 1, 7] = 0
+    qi, qs = cuda_lib.quantize_int4(q.cuda())
+    assert cuda_lib.attn_check_status() == 0
+    rq, rs = Q.quantize_int4_rows(q)
+    assert np.array_equal(_np(qi), rq) and np.array_equal(_np(qs), rs)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 2, 128, 128), (1, 1, 300, 333), (1, 1, 640, 200)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_int4_forward_small(cuda_lib, shape, causal):
+    B, H, Nq, Nkv = shape
+    q, k, v = make_qkv("prefill", seed=19, B=B, H=H, Nq=Nq, Nkv=Nkv, d=128)
+    _, _, cos = _check_int8(cuda_lib, q, k, v, causal, 128 ** -0.5, what=f"int4 {shape} causal={causal}", int4=True)
+    print(f"int4 {shape} causal={causal}: cosine vs fp64 {cos:.4f}")
+
+
+def test_int4_full_lowp_workload_sampled_rows(cuda_lib):
+    w = WORKLOADS["lowp"]
+    q, k, v = make_qkv(w, seed=0)
+    rows = np.array(sorted({0, 1, 127, 128, 8191} | set(np.random.default_rng(2).choice(8192, 11).tolist())))
+    _, flips, cos = _check_int8(cuda_lib, q, k, v, False, w.scale, rows=rows, what="int4 lowp full", int4=True)
+    print(f"int4 lowp: cosine vs fp64 {cos:.4f}, boundary elements {flips}")

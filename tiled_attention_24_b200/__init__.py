@@ -12,7 +12,7 @@ import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
                        attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
-                       attn_fwd, attn_fwd_gqa,
+                       attn_fwd, attn_fwd_gqa, attn_quantize_int4,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
                        attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
                        attn_status_string, attn_version, attn_watchdog_selftest, load)
@@ -22,7 +22,8 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "AttnError", "forward", "decode", "quantize_int8", "forward_int8",
            "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc",
            "attn_quantize_nvfp4", "attn_fwd_fp4", "attn_fp4_scores", "quantize_nvfp4", "forward_fp4",
-           "attn_fwd_gqa", "attn_decode_gqa", "DIRECT_P", "QUANT_AFTER_EXP"]
+           "attn_fwd_gqa", "attn_decode_gqa", "attn_quantize_int4", "quantize_int4", "forward_int4",
+           "DIRECT_P", "QUANT_AFTER_EXP"]
 
 DIRECT_P, QUANT_AFTER_EXP = 0, 1
 
@@ -76,6 +77,29 @@ def forward_int8(q, k, v, causal: bool = False, scale: float | None = None, stre
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     qi, qs = quantize_int8(q, False, stream)
     ki, ks = quantize_int8(k, False, stream)
+    vi, vs = quantize_int8(v, True, stream)
+    o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    attn_fwd_int8(qi, qs, ki, ks, vi, vs, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def quantize_int4(x: torch.Tensor, stream=None):
+    """Token-level INT4 quantisation (codes in [-7, 7], int8 containers)."""
+    B, H, N, d = x.shape
+    xq = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    xs = torch.empty((B, H, N), dtype=torch.float32, device=x.device)
+    attn_quantize_int4(x, xq, xs, stream)
+    return xq, xs
+
+
+def forward_int4(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """INT4 q, k (per token), INT8 v (per head), through the INT8 forward.
+    Returns (o fp32, lse fp32)."""
+    B, H, Nq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    qi, qs = quantize_int4(q, stream)
+    ki, ks = quantize_int4(k, stream)
     vi, vs = quantize_int8(v, True, stream)
     o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)

@@ -33,6 +33,7 @@ SIGNATURES = [
     ("attn_fwd_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_decode_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    ("attn_quantize_int4", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     ("attn_fwd_int8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_int8_scores", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_nvfp4_codes_bytes", _SZ, [_I, _I, _I, _I, _I]),
@@ -157,6 +158,13 @@ def attn_quantize_int8(x, xq, xs, per_head: bool, stream=None):
     B, H, N, d = x.shape
     _check("attn_quantize_int8", load().attn_quantize_int8(_ptr(x), _ptr(xq), _ptr(xs), B, H, N, d,
                                                              int(bool(per_head)), _stream(stream)))
+
+
+def attn_quantize_int4(x, xq, xs, stream=None):
+    """bf16 [B,H,N,d] -> INT4 codes in int8 containers, fp32 per-token scales."""
+    _need_cuda(x, xq, xs)
+    B, H, N, d = x.shape
+    _check("attn_quantize_int4", load().attn_quantize_int4(_ptr(x), _ptr(xq), _ptr(xs), B, H, N, d, _stream(stream)))
 
 
 def attn_fwd_int8(q, qs, k, ks, v, vs, o, lse, causal: bool, scale: float, stream=None):

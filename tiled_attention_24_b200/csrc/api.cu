@@ -419,6 +419,23 @@ int attn_quantize_int8(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+int attn_quantize_int4(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H, int N, int d, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!x || !xq || !xs) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned4(xs)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long rows = (long long)B * H * N;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (d == 128)
+    ta::quant_int8_rows_kernel<128, 7><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
+  else
+    ta::quant_int8_rows_kernel<64, 7><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 int attn_fwd_int8(const int8_t* q, const float* q_scale, const int8_t* k, const float* k_scale, const int8_t* v,
                   const float* v_scale, float* o, float* lse, int B, int H, int Nq, int Nkv, int d, int causal,
                   float scale, void* stream) {

@@ -14,14 +14,16 @@ namespace ta {
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+template <int QMAX = 127>
 __device__ __forceinline__ int8_t q8(float x, float s) {
   int v = __float2int_rn(__fdiv_rn(x, s));
-  v = max(-127, min(127, v));
+  v = max(-QMAX, min(QMAX, v));
   return (int8_t)v;
 }
 
-// One warp per row of D bf16 values (D = 64 or 128).
-template <int D>
+// One warp per row of D bf16 values (D = 64 or 128).  QMAX = 127 (INT8) or 7
+// (INT4 codes in int8 containers: the same token-level scheme at 4 bits).
+template <int D, int QMAX = 127>
 __global__ void __launch_bounds__(256) quant_int8_rows_kernel(const uint16_t* __restrict__ x, int8_t* __restrict__ xq,
                                                              float* __restrict__ xs, long long rows) {
   constexpr int E = D / 32;  // elements per lane
@@ -46,10 +48,10 @@ __global__ void __launch_bounds__(256) quant_int8_rows_kernel(const uint16_t* __
   for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[e]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 127.f);
+  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, (float)QMAX);
   uint32_t packed = 0;
 #pragma unroll
-  for (int e = 0; e < E; ++e) packed |= (uint32_t)(uint8_t)q8(v[e], s) << (8 * e);
+  for (int e = 0; e < E; ++e) packed |= (uint32_t)(uint8_t)q8<QMAX>(v[e], s) << (8 * e);
   if constexpr (E == 4) {
     *reinterpret_cast<uint32_t*>(xq + row * D + lane * E) = packed;
   } else {
