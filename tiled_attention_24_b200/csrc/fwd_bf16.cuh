@@ -71,6 +71,11 @@ struct FwdCfg {
   // register split (launch: 384 threads x 168): warpgroup 0 drops to 80,
   // the two softmax warpgroups rise to 208: 128*80 + 256*208 = 63488 <= 384*168
   static constexpr int REG_LOW = 80, REG_HIGH = 208;
+  // d = 64: P gets its own TMEM columns (S_0, S_1 [0,256), P_0, P_1 [256,384),
+  // O_0, O_1 [384,512)), so a tile's next S is issued as soon as its softmax
+  // holds the current scores, not after its P V.  d = 128: no room; P aliases S.
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr uint32_t T_P = SEP_P ? 256 : 0, T_O = SEP_P ? 384 : 256;
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);
   static constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
   static constexpr float TAU = 8.0f;  // lazy-rescale threshold, log2 units
@@ -86,6 +91,8 @@ struct FwdBars {
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t epi[2];
+  uint64_t s_free[2];   // d = 64: scores of tile t are in registers
+  uint64_t pv_done[2];  // d = 64: P V_t(j) finished (P_t columns free, O_t settled)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -147,6 +154,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&bars->p_full[t]), 128);
       mbar_init(smem_u32(&bars->o_full[t]), 1);
       mbar_init(smem_u32(&bars->epi[t]), 128);
+      mbar_init(smem_u32(&bars->s_free[t]), 128);
+      mbar_init(smem_u32(&bars->pv_done[t]), 1);
     }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       auto issue_PV = [&](int t, int st, int j, uint32_t nb, uint32_t np) -> bool {
         const uint64_t dv = dV0 + (uint64_t)(st * (C::STAGE >> 4));
-        const uint32_t dO = tbase + 256 + t * D, aP = tbase + t * 128;
+        const uint32_t dO = tbase + C::T_O + t * D, aP = tbase + (C::SEP_P ? C::T_P + 64 * t : 128 * t);
         const uint32_t acc0 = (j > 0) ? 1u : 0u;
         bool ready = true;
 #pragma unroll
@@ -267,30 +276,67 @@ __global__ void __launch_bounds__(384, 1)
           if (present[t] && n[t] == 0) tc_commit(smem_u32(&bars->o_full[t]));
       }
       // step j uses stage j + 1: V_j for both P V groups, K_{j+1} for the next S
-      bool seenSt = false;
-      for (int j = 0; j < nmax && ok; ++j) {
-        if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
-        if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
-        int st1 = st + 1;
-        uint32_t sp1 = sp;
-        if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }
-        const uint32_t nbar = (j + 1 < nmax) ? smem_u32(&bars->kv_full[st1]) : 0u;
-        bool seenP1 = false;
-        if (j < n[0]) {
-          if (!(ok = need(false, pf0, j & 1))) break;
-          seenP1 = issue_PV(0, st, j, (j < n[1]) ? pf1 : 0u, j & 1);
-          if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
+      if constexpr (C::SEP_P) {
+        const uint32_t sf0 = smem_u32(&bars->s_free[0]), sf1 = smem_u32(&bars->s_free[1]);
+        bool seenSt = false;
+        for (int j = 0; j < nmax && ok; ++j) {
+          if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
+          if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
+          int st1 = st + 1;
+          uint32_t sp1 = sp;
+          if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }
+          const uint32_t nbar = (j + 1 < nmax) ? smem_u32(&bars->kv_full[st1]) : 0u;
+          // each tile's next S as soon as its softmax holds the current scores
+          if (j + 1 < n[0]) {
+            if (!(ok = need(false, sf0, j & 1))) break;
+            issue_S(0, st, 0, 0);
+          }
+          if (j + 1 < n[1]) {
+            if (!(ok = need(false, sf1, j & 1))) break;
+            issue_S(1, st, 0, 0);
+          }
+          if (j < n[0]) {
+            if (!(ok = need(false, pf0, j & 1))) break;
+            issue_PV(0, st, j, 0, 0);
+            tc_commit(smem_u32(&bars->pv_done[0]));
+            if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
+          }
+          seenSt = false;
+          if (j < n[1]) {
+            if (!(ok = need(false, pf1, j & 1))) break;
+            seenSt = issue_PV(1, st, j, nbar, sp1);
+            tc_commit(smem_u32(&bars->pv_done[1]));
+            if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
+          }
+          seenSt = seenSt && nbar;
+          tc_commit(smem_u32(&bars->kv_empty[st]));
         }
-        if (j + 1 < n[0]) seenP1 = issue_S(0, st, (!seenP1 && j < n[1]) ? pf1 : 0u, j & 1) || seenP1;
-        seenSt = false;
-        if (j < n[1]) {
-          if (!(ok = need(seenP1, pf1, j & 1))) break;
-          seenSt = issue_PV(1, st, j, nbar, sp1);
-          if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
+      } else {
+        bool seenSt = false;
+        for (int j = 0; j < nmax && ok; ++j) {
+          if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
+          if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
+          int st1 = st + 1;
+          uint32_t sp1 = sp;
+          if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }
+          const uint32_t nbar = (j + 1 < nmax) ? smem_u32(&bars->kv_full[st1]) : 0u;
+          bool seenP1 = false;
+          if (j < n[0]) {
+            if (!(ok = need(false, pf0, j & 1))) break;
+            seenP1 = issue_PV(0, st, j, (j < n[1]) ? pf1 : 0u, j & 1);
+            if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
+          }
+          if (j + 1 < n[0]) seenP1 = issue_S(0, st, (!seenP1 && j < n[1]) ? pf1 : 0u, j & 1) || seenP1;
+          seenSt = false;
+          if (j < n[1]) {
+            if (!(ok = need(seenP1, pf1, j & 1))) break;
+            seenSt = issue_PV(1, st, j, nbar, sp1);
+            if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
+          }
+          if (j + 1 < n[1]) seenSt = issue_S(1, st, seenSt ? 0u : nbar, sp1) || seenSt;
+          seenSt = seenSt && nbar;
+          tc_commit(smem_u32(&bars->kv_empty[st]));
         }
-        if (j + 1 < n[1]) seenSt = issue_S(1, st, seenSt ? 0u : nbar, sp1) || seenSt;
-        seenSt = seenSt && nbar;
-        tc_commit(smem_u32(&bars->kv_empty[st]));
       }
       if (!ok) {
         // drain: every MMA issued so far must finish before TMEM is freed
@@ -309,7 +355,8 @@ __global__ void __launch_bounds__(384, 1)
     const int row = r0[t] + rr;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tbase + lane_off + t * 128;
-    const uint32_t tO = tbase + lane_off + 256 + t * D;
+    const uint32_t tO = tbase + lane_off + C::T_O + t * D;
+    const uint32_t tP = C::SEP_P ? tbase + lane_off + C::T_P + 64 * t : tS;
     const float sl2 = p.sl2;
     const int off = p.Nkv - p.Nq;
     float m_ref = -INFINITY, l = 0.f;
@@ -324,6 +371,10 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+      if constexpr (C::SEP_P) {
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->s_free[t]));  // the MMA may now compute S_t(j+1) here
+      }
       const int kb = j * 128;
       const bool tail = kb + 128 > p.Nkv;
       const bool diag = p.causal && (kb + 127 > r0[t] + off);
@@ -354,6 +405,14 @@ __global__ void __launch_bounds__(384, 1)
         m_ref = m_blk;
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if constexpr (C::SEP_P) {
+          // P V_t(j-1) must be done with O_t (with P aliasing S, the S_t(j)
+          // commit already implied it)
+          ok = wait_bar(smem_u32(&bars->pv_done[t]), (j - 1) & 1, abort_flag, p.timeout_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -404,8 +463,16 @@ __global__ void __launch_bounds__(384, 1)
       float ls0, ls1;
       f2_split(fadd2(lsA, lsB), ls0, ls1);
       l += ls0 + ls1;
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+      if constexpr (C::SEP_P) {
+        if (j > 0) {  // P V_t(j-1) has read the P_t columns
+          ok = wait_bar(smem_u32(&bars->pv_done[t]), (j - 1) & 1, abort_flag, p.timeout_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
+      tmem_st32(tP, pk[0]);
+      tmem_st32(tP + 32, pk[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full[t]));
