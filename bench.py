@@ -400,7 +400,8 @@ def run_ours(args):
                 "frac": pn["rate"] / peak_tc, "traffic": traffic.get("fwd_bf16_prefill_noncausal"),
                 "kernel": "fwd_bf16_kernel<128>, prefill B4 H16 N4096 d128 non-causal",
                 "peak_source": f"{peak_src} bf16 burst"}
-    for part, key in (("decode", "decode_split"), ("lowp_int8", "fwd_int8_lowp"),
+    for part, key in (("decode", "decode_split"), ("longseq_noncausal", "fwd_bf16_longseq_noncausal"),
+                      ("prefill_causal", "fwd_bf16_prefill_causal"), ("lowp_int8", "fwd_int8_lowp"),
                       ("lowp_fp4_direct_p", "fwd_fp4_direct_p_lowp"),
                       ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp")):
         if part in out_parts:
