@@ -87,6 +87,43 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None,
     return O, LSE
 
 
+def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = None):
+    """Gradients of O = softmax(scale * Q K^T, masked) V with respect to Q, K
+    and V for an upstream gradient dO, in float64 -- the calculus of the
+    definition, with P materialised (the quantity [FA-trading] "Backward:
+    recompute instead of store" says the tiled method recomputes from Q, K and
+    the stored softmax statistics instead of keeping it):
+
+        dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik),
+        dQ = scale dS K,  dK = scale dS^T Q.
+
+    sum_k P_ik dP_ik equals sum_c dO_ic O_ic (O = P V).  Rows that see no key
+    have P = 0 and contribute nothing.  Returns (dQ, dK, dV) float64."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    vis = visible_mask(Nq, Nkv, causal)
+    for b in range(B):
+        for h in range(H):
+            S = np.where(vis, (q[b, h] @ k[b, h].T) * scale, -np.inf)
+            m = S.max(axis=1)
+            alive = np.isfinite(m)
+            P = np.exp(S - np.where(alive, m, 0.0)[:, None])
+            P /= np.where(alive, P.sum(axis=1), 1.0)[:, None]
+            P = np.where(alive[:, None], P, 0.0)
+            dP = do[b, h] @ v[b, h].T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dv[b, h] = P.T @ do[b, h]
+            dq[b, h] = scale * (dS @ k[b, h])
+            dk[b, h] = scale * (dS.T @ q[b, h])
+    return dq, dk, dv
+
+
 def kv_head_index(Hq: int, Hkv: int) -> np.ndarray:
     """Key/value head of every query head under grouped-query attention:
     query head h reads key/value head h // (Hq / Hkv) ([FA4-overview]

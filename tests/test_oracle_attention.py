@@ -230,3 +230,51 @@ def test_kv_head_index_groups_and_rejects_uneven():
     assert A.kv_head_index(4, 4).tolist() == [0, 1, 2, 3]
     with pytest.raises(ValueError):
         A.kv_head_index(6, 4)
+
+
+# ---------------------------------------------------------------- backward
+@pytest.mark.parametrize("causal,Nq,Nkv", [(False, 7, 9), (True, 8, 8), (True, 5, 9), (True, 9, 4)])
+def test_backward_matches_torch_autograd_fp64(causal, Nq, Nkv):
+    """Pin against PyTorch autograd through its own fp64 attention (explicit
+    scores, masked_fill, softmax, matmul): an implementation of the gradient
+    independent of the closed-form expressions."""
+    g = torch.Generator().manual_seed(Nq * 31 + Nkv)
+    q, k, v, do = (torch.randn(2, 2, n, 5, generator=g, dtype=torch.float64) for n in (Nq, Nkv, Nkv, Nq))
+    qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
+    S = (qr @ kr.transpose(-1, -2)) * 0.35
+    vis = torch.tensor(A.visible_mask(Nq, Nkv, causal))
+    S = S.masked_fill(~vis, float("-inf"))
+    P = torch.softmax(S, dim=-1).nan_to_num(0.0)      # rows with no visible key: P = 0
+    (P @ vr).backward(do)
+    dq, dk, dv = A.attention_backward(q, k, v, do, causal, 0.35)
+    for got, ref in ((dq, qr.grad), (dk, kr.grad), (dv, vr.grad)):
+        assert np.abs(got - ref.numpy()).max() < 1e-12
+
+
+def test_backward_finite_differences_tiny():
+    """Central differences of sum(O * dO) on a 1 x 1 x 3 x 2 problem."""
+    g = np.random.default_rng(12)
+    q, k, v, do = (g.standard_normal((1, 1, 3, 2)) for _ in range(4))
+    dq, dk, dv = A.attention_backward(q, k, v, do, True, 0.7)
+    f = lambda qq, kk, vv: float((A.attention(qq, kk, vv, True, 0.7)[0] * do).sum())
+    eps = 1e-6
+    for arr, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += eps
+            args_m[which][idx] -= eps
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * eps)
+        assert np.abs(num - grad).max() < 1e-7
+
+
+def test_backward_row_statistic_identity():
+    """sum_k P_ik dP_ik = sum_c dO_ic O_ic, the per-row quantity the tiled
+    backward computes from the stored O instead of from P."""
+    g = torch.Generator().manual_seed(2)
+    q, k, v, do = (torch.randn(1, 1, 6, 4, generator=g, dtype=torch.float64) for _ in range(4))
+    O, _ = A.attention(q, k, v, False, 0.5)
+    P = A.softmax_rows(q, k, False, 0.5)
+    dP = do.numpy() @ v.numpy().transpose(0, 1, 3, 2)
+    assert np.abs((P * dP).sum(-1) - (do.numpy() * O).sum(-1)).max() < 1e-12
