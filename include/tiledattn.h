@@ -106,6 +106,28 @@ ATTN_API int attn_fwd_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn
                           void* stream);
 
 /*
+ * attn_bwd -- bf16 attention backward by recomputation ([FA-trading]
+ * "Backward: recompute instead of store": P is never stored by the forward;
+ * it is recomputed tile by tile from Q, K and the forward's softmax
+ * statistics, here the LSE).  With S = scale Q K^T (masked as attn_fwd) and
+ * P = exp(S - LSE):
+ *   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - rowsum(dO o O)),
+ *   dQ = scale dS K,  dK = scale dS^T Q   (fp32 accumulation, bf16 out).
+ *
+ *   q, o, dout, dq [B][H][Nq][d] bf16; k, v, dk, dv [B][H][Nkv][d] bf16;
+ *   lse [B][H][Nq] fp32 (attn_fwd's output for the same q, k, v, causal,
+ *   scale); o = attn_fwd's O.  d in {64, 128}.  workspace: device scratch of
+ *   at least attn_bwd_workspace_bytes(B, H, Nq) bytes, 16-byte aligned,
+ *   owned by the caller (holds rowsum(dO o O)).  Nq == 0 or Nkv == 0: the
+ *   gradients that exist are set to zero.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int Nq);
+ATTN_API int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+                      const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv,
+                      int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode -- split-KV decode: ONE query row per (batch, head) against a
  * KV cache of Nkv keys; the key range is cut into num_splits equal chunks of
  * ceil(Nkv / num_splits) keys, each chunk gives a partial (O_c, LSE_c) in the

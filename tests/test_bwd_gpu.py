@@ -1,0 +1,72 @@
+"""GPU parity of attn_bwd (bf16 backward by recomputation) against the fp64
+oracle's gradients, through the C ABI.
+
+The device computes with bf16 operands: O from the device forward, P and dS
+rounded to bf16 before their MMAs, bf16 outputs.  Each rounding is a relative
+2^-9; the tolerance is 2^-7 of the largest reference magnitude of the tensor
+(max-abs) and 2^-9 of its mean magnitude plus that (mean-abs), per gradient.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from workloads import WORKLOADS, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def _grads(ta, q, k, v, do, causal, scale):
+    q, k, v, do = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = ta.forward(q, k, v, causal, scale)
+    dq, dk, dv = ta.backward(q, k, v, o, lse, do, causal, scale)
+    assert ta.attn_check_status() == 0
+    return [t.double().cpu().numpy() for t in (dq, dk, dv)]
+
+
+def _check(got, ref, what):
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(g).all(), f"{what} {name}: non-finite"
+        err = np.abs(g - r)
+        big = float(np.abs(r).max(initial=0.0))
+        mean = float(np.abs(r).mean()) if r.size else 0.0
+        print(f"{what} {name}: max err {err.max(initial=0):.3e} (ref max {big:.3e}), "
+              f"mean err {err.mean() if err.size else 0:.3e} (ref mean {mean:.3e})")
+        assert err.max(initial=0.0) <= 2.0 ** -7 * big + 1e-6, f"{what} {name}"
+        assert (err.mean() if err.size else 0.0) <= 2.0 ** -9 * mean + 2.0 ** -7 * big / 64 + 1e-7, f"{what} {name}"
+
+
+SHAPES = [
+    # B, H, Nq, Nkv, d
+    (1, 2, 128, 128, 64),
+    (1, 1, 300, 333, 128),
+    (2, 1, 129, 1000, 64),
+    (1, 1, 640, 200, 128),     # causal: the first rows see no key
+    (1, 2, 384, 384, 128),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_backward_small(cuda_lib, shape, causal):
+    B, H, Nq, Nkv, d = shape
+    q, k, v = make_qkv("prefill", seed=41, B=B, H=H, Nq=Nq, Nkv=Nkv, d=d)
+    do = make_qkv("prefill", seed=42, B=B, H=H, Nq=Nq, Nkv=1, d=d)[0]
+    scale = d ** -0.5
+    got = _grads(cuda_lib, q, k, v, do, causal, scale)
+    ref = A.attention_backward(q, k, v, do, causal, scale)
+    _check(got, ref, f"{shape} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_prefill_workload_sampled_heads(cuda_lib, causal):
+    """The prefill workload shape (B4 H16 N4096 d128); the oracle checks two
+    (batch, head) slices (heads are independent)."""
+    w = WORKLOADS["prefill"]
+    q, k, v = make_qkv(w, seed=0)
+    do = make_qkv(w, seed=1, Nkv=1)[0]
+    got = _grads(cuda_lib, q, k, v, do, causal, w.scale)
+    for b, h in [(0, 0), (3, 15)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = A.attention_backward(q[sl], k[sl], v[sl], do[sl], causal, w.scale)
+        _check([g[sl] for g in got], ref, f"prefill b={b} h={h} causal={causal}")

@@ -31,6 +31,8 @@ SIGNATURES = [
     ("attn_decode", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_decode_noalloc", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP]),
     ("attn_fwd_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    ("attn_bwd_workspace_bytes", _SZ, [_I, _I, _I]),
+    ("attn_bwd", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     ("attn_decode_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_quantize_int4", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP]),
@@ -124,6 +126,21 @@ def attn_decode_gqa(q, k, v, o, lse, scale: float, num_splits: int, workspace, s
                                 int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream))
     _check("attn_decode_gqa", rc)
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, Nq: int) -> int:
+    return int(load().attn_bwd_workspace_bytes(B, H, Nq))
+
+
+def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None):
+    """bf16 backward: gradients dq, dk, dv of the forward (o, lse) for upstream dout."""
+    _need_cuda(q, k, v, o, dout, lse, dq, dk, dv, workspace)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                         B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_bwd", rc)
 
 
 def attn_decode_workspace_bytes(B: int, H: int, d: int, num_splits: int) -> int:

@@ -17,6 +17,7 @@
 #include "quant.cuh"
 #include "fwd_int8.cuh"
 #include "fwd_fp4.cuh"
+#include "bwd_bf16.cuh"
 
 namespace {
 
@@ -195,6 +196,45 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, float* rowdot, int B, int H, int Nq, int Nkv, int causal, float scale,
+               cudaStream_t st) {
+  using C = ta::BwdCfg<D>;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if ((rc = make_tmap_bf16(&tq, q, D, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, D, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, D, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tdo, dout, D, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::bwd_dkdv_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::bwd_dq_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
+  ta::BwdParams p;
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.rowdot = rowdot;
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.nqt = (Nq + 127) / 128;
+  p.nkt = (Nkv + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_ns;
+  const long long rows = (long long)BH * Nq;
+  const long long gk = (long long)BH * p.nkt, gq = (long long)BH * p.nqt;
+  if ((rows + 7) / 8 > 0x7fffffffLL || gk > 0x7fffffffLL || gq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  ta::bwd_rowdot_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.o, p.dout, rowdot, rows);
+  ta::bwd_dkdv_kernel<D><<<(unsigned)gk, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tdo, p);
+  ta::bwd_dq_kernel<D><<<(unsigned)gq, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 size_t decode_ws_bytes(long long BH, int d, int S) {
   const size_t o_bytes = (size_t)BH * S * d * sizeof(float);
   const size_t l_bytes = (size_t)BH * S * sizeof(float);
@@ -288,6 +328,42 @@ int attn_fwd_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* 
 int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
              int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
   return attn_fwd_gqa(q, k, v, o, lse, B, H, H > 0 ? H : 1, Nq, Nkv, d, causal, scale, stream);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int Nq) {
+  if (B <= 0 || H <= 0 || Nq <= 0) return 0;
+  return ((size_t)B * H * Nq * sizeof(float) + 255) & ~size_t(255);
+}
+
+int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+             const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv, int B,
+             int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+             void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return ATTN_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t kv_bytes = (size_t)B * H * Nkv * d * 2, q_bytes = (size_t)B * H * Nq * d * 2;
+  if (Nq == 0 || Nkv == 0) {
+    // no query or no key: every gradient that exists is zero
+    if (Nkv > 0 && (!dk || !dv)) return ATTN_ERR_INVALID_ARG;
+    if (Nq > 0 && !dq) return ATTN_ERR_INVALID_ARG;
+    if (Nkv > 0 && (cudaMemsetAsync(dk, 0, kv_bytes, st) != cudaSuccess ||
+                    cudaMemsetAsync(dv, 0, kv_bytes, st) != cudaSuccess))
+      return ATTN_ERR_CUDA;
+    if (Nq > 0 && cudaMemsetAsync(dq, 0, q_bytes, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned4(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
+  float* rowdot = static_cast<float*>(workspace);
+  return d == 128 ? launch_bwd<128>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st)
+                  : launch_bwd<64>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st);
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
