@@ -5,7 +5,8 @@
 A step is one pass of the hot path over the seeded synthetic workloads:
   * prefill  B=4 H=16 N=4096 d=128 bf16: attn_fwd non-causal + attn_fwd causal
              (the headline: attention forward TFLOP/s, 4*B*H*N*N*d, halved
-             for causal);
+             for causal); and attn_bwd on the same shapes (reported as a part,
+             2.5 x the forward's FLOPs, not in the headline);
   * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine; and
              the same with grouped-query attention (8 cache heads, 4 query
              heads each: 2.1 GB of cache);
@@ -237,6 +238,20 @@ def run_ours(args):
             wp.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
         seg("prefill_causal", lambda: ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream),
             wp.flops(True), "TFLOP/s", peak_tc, "tensor", 1)
+        # backward by recomputation (from the causal forward's O and LSE above):
+        # algorithmic work = 5 matmuls (S, dP, dV, dK, dQ) = 2.5 x the forward's
+        bo, blse = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        ta.attn_fwd(q, k, v, bo, blse, True, wp.scale, stream)
+        bo_n, blse_n = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        ta.attn_fwd(q, k, v, bo_n, blse_n, False, wp.scale, stream)
+        dout = make_qkv(wp, seed=1, device=dev, Nkv=1)[0]
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(ta.attn_bwd_workspace_bytes(wp.B, wp.H, wp.Nq), dtype=torch.uint8, device=dev)
+        seg("prefill_bwd_noncausal",
+            lambda: ta.attn_bwd(q, k, v, bo_n, dout, blse_n, dq, dk, dv, False, wp.scale, bws, stream),
+            2.5 * wp.flops(False), "TFLOP/s", peak_tc, "tensor", 3)
+        seg("prefill_bwd_causal", lambda: ta.attn_bwd(q, k, v, bo, dout, blse, dq, dk, dv, True, wp.scale, bws, stream),
+            2.5 * wp.flops(True), "TFLOP/s", peak_tc, "tensor", 3)
     wd = WORKLOADS["decode"]
     if "decode" in parts:
         dq, dk, dv = make_qkv(wd, seed=0, device=dev, B=args.decode_batch or wd.B)
@@ -344,7 +359,7 @@ def run_ours(args):
         rate = work / (avg * 1e-3) / scale
         out_parts[name] = {"ms": avg, "rate": rate, "unit": unit, "bound": bound, "peak": peak,
                            "frac": rate / peak}
-    pre = [i for i, sg in enumerate(segs) if sg[0].startswith("prefill_")]
+    pre = [i for i, sg in enumerate(segs) if sg[0] in ("prefill_noncausal", "prefill_causal")]
     if pre:
         value = job_throughput(ws, args.steps, sum(segs[i][2] for i in pre), sum(seg_ms[i] for i in pre)) / 1e12
     else:
