@@ -91,6 +91,20 @@ def test_gqa_head_validation(lib, Hq, Hkv, code):
     assert rc == (code if code else -2)
 
 
+def test_bwd_workspace_and_validation(lib):
+    n = lib.attn_bwd_workspace_bytes(2, 3, 100)
+    assert n >= 2 * 3 * 100 * 4 and n % 256 == 0
+    assert lib.attn_bwd_workspace_bytes(0, 3, 100) == 0
+    ws = ctypes.c_void_p(16 * 4096)
+    def call(**kw):
+        a = dict(B=1, H=2, Nq=64, Nkv=64, d=128, causal=0, scale=0.1, ws_bytes=n)
+        a.update(kw)
+        return lib.attn_bwd(P, P, P, P, P, P, P, P, P, a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
+                            a["scale"], ws, a["ws_bytes"], None)
+    assert call(d=96) == -2 and call(scale=0.0) == -1 and call(B=-1) == -1 and call(Nkv=-2) == -1
+    assert call(ws_bytes=16) == -1 and call(B=0) == 0
+
+
 def test_product_path_never_imports_the_oracle():
     """The package must not reach the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "tiled_attention_24_b200")
