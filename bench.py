@@ -14,7 +14,8 @@ A step is one pass of the hot path over the seeded synthetic workloads:
   * longseq  B=1 H=12 N=23400 d=64 bf16, non-causal + causal;
   * lowp     B=2 H=24 N=8192 d=128 with outlier channels: bf16 forward, INT8
              quantisers + INT8 forward, NVFP4 quantisers + FP4 forward with
-             Direct-P and with quantise-after-exp.
+             Direct-P and with quantise-after-exp, FP8 quantisers (Hadamard
+             rotation of Q, K) + FP8 forward.
 Inputs are resident in HBM before timing starts and are larger than the
 126 MB L2 (prefill Q+K+V = 201 MB, decode K+V = 8.6 GB), so no L2 flush is
 needed between steps.  Every launch is bracketed by CUDA events on the
@@ -47,7 +48,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, make_qkv  # noqa: E402
+from workloads import WORKLOADS, make_qkv, rotation_signs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -221,6 +222,7 @@ def run_ours(args):
     ratio = peak_tc / 2250.0
     peak_i8 = float(peaks.get("int8_tops", 4500.0 * ratio))
     peak_f4 = float(peaks.get("fp4_tflops", 9000.0 * ratio))
+    peak_f8 = float(peaks.get("fp8_tflops", 4500.0 * ratio))
     lowp_peak_src = "measured" if "int8_tops" in peaks else "nominal x (measured/nominal bf16)"
 
     segs = []   # (name, fn, work, unit, peak, bound, launches)
@@ -310,6 +312,19 @@ def run_ours(args):
             seg(nm, (lambda mode=mode: ta.attn_fwd_fp4(c4[0], f4[0], c4[1], f4[1], c4[2], f4[2], of, lf, B5, H5,
                                                         N5, N5, False, wq.scale, mode, stream)),
                 wq.flops(False), "TFLOP/s", peak_f4, "tensor", 1)
+        c8 = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (xq, xk, xv)]
+        s8f = [torch.empty((B5, H5, N5), dtype=torch.float32, device=dev) for _ in range(2)]
+        s8f.append(torch.empty((B5, H5, D5), dtype=torch.float32, device=dev))
+        signs = rotation_signs(D5, 0).to(dev)
+
+        def qf8():
+            ta.attn_quantize_fp8(xq, c8[0], s8f[0], 0, signs, stream)
+            ta.attn_quantize_fp8(xk, c8[1], s8f[1], 0, signs, stream)
+            ta.attn_quantize_fp8(xv, c8[2], s8f[2], 1, None, stream)
+        seg("lowp_fp8_quantise", qf8, 3 * xq.numel() * 2 + 3 * xq.numel(), "GB/s", peak_hbm, "hbm", 3)
+        seg("lowp_fp8", lambda: ta.attn_fwd_fp8(c8[0], s8f[0], c8[1], s8f[1], c8[2], s8f[2], of, lf, False,
+                                                wq.scale, True, stream),
+            wq.flops(False), "TFLOP/s", peak_f8, "tensor", 1)
 
     nseg = len(segs)
 
@@ -421,7 +436,7 @@ def run_ours(args):
                       ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp")):
         if part in out_parts:
             out_parts[part]["traffic"] = traffic.get(key)
-    for nm in ("lowp_int8", "lowp_fp4_direct_p", "lowp_fp4_quant_after_exp"):
+    for nm in ("lowp_int8", "lowp_fp4_direct_p", "lowp_fp4_quant_after_exp", "lowp_fp8"):
         if nm in out_parts:
             out_parts[nm]["peak_source"] = lowp_peak_src
     line = {

@@ -294,6 +294,47 @@ ATTN_API int attn_fp4_scores(const uint8_t* q, const uint8_t* q_sf, const uint8_
                              int B, int H, int Nq, int Nkv, int d, void* stream);
 
 /*
+ * FP8 (e4m3) operands with incoherent processing ([FA-trading] "FA2"/"FA3"
+ * list, item 3: FP8 doubles the matmul rate; Q and K are rotated by a random
+ * Hadamard transform before quantisation so that outliers spread over the
+ * coordinates).  e4m3: OCP E4M3 (bias 7, largest finite 448), round to
+ * nearest even, saturating; codes stored one per byte.
+ * attn_quantize_fp8
+ *   mode 0 (Q, K): one fp32 scale per token row.  If `signs` (fp32 [d], each
+ *     +1 or -1, device) is given, the row is first rotated, y = H_d (signs o x)
+ *     with H_d the unnormalised Sylvester Hadamard matrix, evaluated as the
+ *     fast Walsh-Hadamard transform in fp32 (stages h = 1, 2, ..., d/2, pair
+ *     (a, b) -> (a + b, a - b)); signs = NULL quantises x unrotated.
+ *     s = amax(|y|) / 448 (IEEE fp32 divide; amax == 0 gives s = 1), codes
+ *     e4m3(y / s); scales [B][H][N].
+ *   mode 1 (V): one scale per (batch, head, channel) over the N tokens, no
+ *     rotation; scales [B][H][d].
+ *   x bf16 [B][H][N][d], codes [B][H][N][d] bytes (both 16-byte aligned);
+ *   d in {64, 128}.
+ */
+ATTN_API int attn_quantize_fp8(const attn_bf16_t* x, uint8_t* codes, float* scales, int B, int H, int N, int d,
+                               int mode, const float* signs, void* stream);
+
+/*
+ * attn_fwd_fp8 -- FP8 attention forward on the FP8 tensor cores
+ * ([FA-trading] FA3 list item 3; tiling and online softmax as attn_fwd):
+ *   S = codes(q) codes(k)^T (fp32 accumulation of exact e4m3 products);
+ *   x = S * q_scale[i] * k_scale[j] * scale * log2(e) / r, r = d when q and k
+ *   were rotated (rotated != 0: the rotation multiplies q k^T by d), else 1;
+ *   per block of 128 keys the running row max m moves on every increase,
+ *   P~ = e4m3(2^(x - m)) (values in [0, 1], unit scale), l = l 2^(m_old - m) +
+ *   sum P~, acc = acc 2^(m_old - m) + P~ codes(v);
+ *   O[i][c] = acc[i][c] * v_scale[c] / l (fp32), LSE = ln 2 (m + log2 l).
+ *   q [B][H][Nq][128] codes + q_scale [B][H][Nq]; k [B][H][Nkv][128] codes +
+ *   k_scale [B][H][Nkv]; v [B][H][Nkv][128] codes + v_scale [B][H][128]
+ *   (16-byte aligned); o [B][H][Nq][128] fp32 out, lse [B][H][Nq] fp32 out.
+ *   d must be 128; Nkv >= 1.
+ */
+ATTN_API int attn_fwd_fp8(const uint8_t* q, const float* q_scale, const uint8_t* k, const float* k_scale,
+                          const uint8_t* v, const float* v_scale, float* o, float* lse, int B, int H, int Nq,
+                          int Nkv, int d, int causal, float scale, int rotated, void* stream);
+
+/*
  * attn_check_status -- synchronise `stream`, read the device status word
  * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT), clear it and
  * return it; also returns ATTN_ERR_CUDA if the synchronisation itself fails.

@@ -144,7 +144,8 @@ def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=
                 m_new = np.maximum(m, xb.max(axis=1))
                 grow = np.isfinite(m) & (m_new > m)
                 f = np.ones_like(m)
-                np.exp2(m - m_new, out=f, where=grow)
+                with np.errstate(invalid="ignore"):  # -inf - -inf where not grow (not used)
+                    np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
                 m = m_new

@@ -105,6 +105,23 @@ def test_bwd_workspace_and_validation(lib):
     assert call(ws_bytes=16) == -1 and call(B=0) == 0
 
 
+def test_fp8_host_validation(lib):
+    def quant(**kw):
+        a = dict(B=1, H=2, N=64, d=128, mode=0, signs=None)
+        a.update(kw)
+        return lib.attn_quantize_fp8(P, P, P, a["B"], a["H"], a["N"], a["d"], a["mode"], a["signs"], None)
+    assert quant(d=96) == -2 and quant(mode=2) == -1 and quant(N=-1) == -1
+    assert quant(mode=1, signs=P) == -1 and quant(signs=ctypes.c_void_p(16 * 1000 + 2)) == -3
+    assert quant(B=0) == 0
+    def fwd(**kw):
+        a = dict(B=1, H=2, Nq=64, Nkv=64, d=128, causal=0, scale=0.1, rot=1, vs=P)
+        a.update(kw)
+        return lib.attn_fwd_fp8(P, P, P, P, P, a["vs"], P, P, a["B"], a["H"], a["Nq"], a["Nkv"], a["d"],
+                                a["causal"], a["scale"], a["rot"], None)
+    assert fwd(d=64) == -2 and fwd(scale=0.0) == -1 and fwd(Nkv=0) == -2 and fwd(Nq=-1) == -1
+    assert fwd(vs=ctypes.c_void_p(16 * 1000 + 4)) == -3 and fwd(Nq=0) == 0
+
+
 def test_product_path_never_imports_the_oracle():
     """The package must not reach the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "tiled_attention_24_b200")

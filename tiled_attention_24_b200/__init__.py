@@ -12,7 +12,7 @@ import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
                        attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
-                       attn_fwd, attn_fwd_gqa, attn_quantize_int4, attn_bwd, attn_bwd_workspace_bytes,
+                       attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_workspace_bytes,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
                        attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
                        attn_status_string, attn_version, attn_watchdog_selftest, load)
@@ -24,6 +24,7 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "attn_quantize_nvfp4", "attn_fwd_fp4", "attn_fp4_scores", "quantize_nvfp4", "forward_fp4",
            "attn_fwd_gqa", "attn_decode_gqa", "attn_quantize_int4", "quantize_int4", "forward_int4",
            "attn_bwd", "attn_bwd_workspace_bytes", "backward",
+           "attn_quantize_fp8", "attn_fwd_fp8", "quantize_fp8", "forward_fp8", "hadamard_signs",
            "DIRECT_P", "QUANT_AFTER_EXP"]
 
 DIRECT_P, QUANT_AFTER_EXP = 0, 1
@@ -116,6 +117,42 @@ def forward_int4(q, k, v, causal: bool = False, scale: float | None = None, stre
     o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     attn_fwd_int8(qi, qs, ki, ks, vi, vs, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def hadamard_signs(d: int, seed: int = 0, device="cuda"):
+    """Seeded random sign vector (fp32, +-1) of the FP8 rotation H_d diag(signs)."""
+    g = torch.Generator().manual_seed(int(seed))
+    s = torch.randint(0, 2, (d,), generator=g, dtype=torch.int64) * 2 - 1
+    return s.to(torch.float32).to(device)
+
+
+def quantize_fp8(x: torch.Tensor, mode: int, signs: torch.Tensor | None = None, stream=None):
+    """e4m3 codes (uint8) and fp32 scales of a bf16 [B,H,N,d] tensor: mode 0 per
+    token row (rotated first when ``signs`` is given), mode 1 per channel."""
+    B, H, N, d = x.shape
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((B, H, N) if mode == 0 else (B, H, d), dtype=torch.float32, device=x.device)
+    attn_quantize_fp8(x, codes, scales, mode, signs, stream)
+    return codes, scales
+
+
+def forward_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotate: bool = True,
+                signs: torch.Tensor | None = None, stream=None):
+    """Quantise bf16 q, k (per token, rotated by H_d diag(signs) unless
+    ``rotate`` is False) and v (per channel) to e4m3 and run the FP8 forward.
+    Returns (o fp32, lse fp32)."""
+    B, H, Nq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if rotate and signs is None:
+        signs = hadamard_signs(d, 0, q.device)
+    sg = signs if rotate else None
+    qc, qs = quantize_fp8(q, 0, sg, stream)
+    kc, ks = quantize_fp8(k, 0, sg, stream)
+    vc, vs = quantize_fp8(v, 1, None, stream)
+    o = torch.empty((B, H, Nq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    attn_fwd_fp8(qc, qs, kc, ks, vc, vs, o, lse, causal, scale, rotate, stream)
     return o, lse
 
 

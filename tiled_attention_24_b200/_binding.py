@@ -43,6 +43,8 @@ SIGNATURES = [
     ("attn_quantize_nvfp4", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_fwd_fp4", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
     ("attn_fp4_scores", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    ("attn_quantize_fp8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
+    ("attn_fwd_fp8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
     ("attn_check_status", _I, [_VP]),
     ("attn_set_wait_limit_ns", None, [_ULL]),
     ("attn_watchdog_selftest", _I, [_ULL, _VP]),
@@ -232,6 +234,29 @@ def attn_fp4_scores(q, qsf, k, ksf, s, B, H, Nq, Nkv, stream=None):
     _need_cuda(q, qsf, k, ksf, s)
     _check("attn_fp4_scores", load().attn_fp4_scores(_ptr(q), _ptr(qsf), _ptr(k), _ptr(ksf), _ptr(s), B, H, Nq, Nkv,
                                                        128, _stream(stream)))
+
+
+def attn_quantize_fp8(x, codes, scales, mode: int, signs=None, stream=None):
+    """bf16 [B,H,N,d] -> e4m3 codes (uint8) + fp32 scales; mode 0: per row
+    ([B,H,N]; rotated by H_d diag(signs) when signs is given), 1: per channel ([B,H,d])."""
+    _need_cuda(x, codes, scales)
+    if signs is not None:
+        _need_cuda(signs)
+    B, H, N, d = x.shape
+    _check("attn_quantize_fp8", load().attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(scales), B, H, N, d, int(mode),
+                                                           None if signs is None else _ptr(signs),
+                                                           _stream(stream)))
+
+
+def attn_fwd_fp8(q, qs, k, ks, v, vs, o, lse, causal: bool, scale: float, rotated: bool, stream=None):
+    """FP8 forward: e4m3 codes [B,H,N,128] with scales -> o fp32, lse fp32."""
+    _need_cuda(q, qs, k, ks, v, vs, o, lse)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_fwd_fp8(_ptr(q), _ptr(qs), _ptr(k), _ptr(ks), _ptr(v), _ptr(vs), _ptr(o), _ptr(lse),
+                             B, H, Nq, Nkv, d, int(bool(causal)), float(scale), int(bool(rotated)),
+                             _stream(stream))
+    _check("attn_fwd_fp8", rc)
 
 
 def attn_check_status(stream=None) -> int:

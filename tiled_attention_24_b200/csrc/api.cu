@@ -18,6 +18,7 @@
 #include "fwd_int8.cuh"
 #include "fwd_fp4.cuh"
 #include "bwd_bf16.cuh"
+#include "fwd_fp8.cuh"
 
 namespace {
 
@@ -538,6 +539,77 @@ int attn_int8_scores(const int8_t* q, const int8_t* k, int32_t* s, int B, int H,
   if (!aligned16(q) || !aligned16(k) || !aligned4(s)) return ATTN_ERR_MISALIGNED;
   return launch_int8<true>(q, nullptr, k, nullptr, nullptr, nullptr, nullptr, nullptr, s, B, H, Nq, Nkv, 0, 1.f,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_quantize_fp8(const attn_bf16_t* x, uint8_t* codes, float* scales, int B, int H, int N, int d, int mode,
+                      const float* signs, void* stream) {
+  if (B < 0 || H < 0 || N < 0 || (mode != 0 && mode != 1)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (mode == 1 && signs != nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!x || !codes || !scales) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned4(scales) || (signs && !aligned4(signs)))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long BH = (long long)B * H;
+  if (mode == 0) {
+    const long long rows = BH * N;
+    const long long blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (d == 128)
+      ta::quant_fp8_rows_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(x, signs, codes, scales, rows);
+    else
+      ta::quant_fp8_rows_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(x, signs, codes, scales, rows);
+  } else {
+    if (BH > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (d == 128)
+      ta::quant_fp8_channels_kernel<128><<<(unsigned)BH, 128, 0, st>>>(x, codes, scales, N);
+    else
+      ta::quant_fp8_channels_kernel<64><<<(unsigned)BH, 64, 0, st>>>(x, codes, scales, N);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_fwd_fp8(const uint8_t* q, const float* q_scale, const uint8_t* k, const float* k_scale, const uint8_t* v,
+                 const float* v_scale, float* o, float* lse, int B, int H, int Nq, int Nkv, int d, int causal,
+                 float scale, int rotated, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;
+  if (Nkv == 0) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !q_scale || !k || !k_scale || !v || !v_scale || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(v_scale) ||
+      !aligned4(q_scale) || !aligned4(k_scale) || !aligned4(lse))
+    return ATTN_ERR_MISALIGNED;
+  using C = ta::FwdF8Cfg;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_i8(&tq, q, Nq, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_i8(&tk, k, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_i8(&tv, v, Nkv, BH)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::fwd_fp8_kernel, C::SMEM)) != ATTN_OK) return rc;
+  ta::FwdF8Params p;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.o = o;
+  p.lse = lse;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.n_qp = (Nq + 255) / 256;
+  p.Tc = (Nkv + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.ks_vec = (Nkv % 4 == 0) && aligned16(k_scale);
+  p.sl2 = scale * 1.4426950408889634f / (rotated ? 128.f : 1.f);
+  p.timeout_ns = g_wait_ns;
+  const long long grid = (long long)BH * p.n_qp;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  ta::fwd_fp8_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv,
+                                                                                                     p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 size_t attn_nvfp4_codes_bytes(int B, int H, int N, int d, int mode) {

@@ -226,4 +226,93 @@ __global__ void __launch_bounds__(256) quant_nvfp4_cols_kernel(const uint16_t* _
   sf[((bh * KT + tb / 8) * 1024) + sf_offset(c, tb & 7)] = (uint8_t)sfc;
 }
 
+// ---------------------------------------------------------------------------
+// FP8 e4m3 with incoherent processing ("Can a full-day context beat one
+// minute? ..." page, FA3 list item 3: rotate the vectors before quantising so
+// that outliers spread over the coordinates).  Q, K rows: optional rotation
+// y = H_d (sigma o x) by the unnormalised fast Walsh-Hadamard transform in
+// fp32 (stages h = 1, 2, ..., d/2; (a, b) -> (a + b, a - b)), then one scale
+// per row s = amax / 448 and codes e4m3_rne_satfinite(y / s) (IEEE divides).
+// V: one scale per (batch, head, channel) over the head's tokens.
+__device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {  // lo -> low byte
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One warp per row; D / 32 values per lane (element e = lane * E + i).
+template <int D>
+__global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const uint16_t* __restrict__ x,
+                                                             const float* __restrict__ signs,
+                                                             uint8_t* __restrict__ codes, float* __restrict__ xs,
+                                                             long long rows) {
+  constexpr int E = D / 32;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint16_t* src = x + row * D + lane * E;
+  float v[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) v[i] = bf16_to_f32(src[i]);
+  if (signs != nullptr) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) v[i] *= signs[lane * E + i];
+    // stages inside a lane
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if ((i & h) == 0) {
+          const float a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+      }
+    }
+    // stages across lanes: partner lane differs in bit h / E
+#pragma unroll
+    for (int h = E; h < D; h <<= 1) {
+      const int lm = h / E;
+      const bool upper = (lane & lm) != 0;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[i], lm);
+        v[i] = upper ? (o - v[i]) : (v[i] + o);
+      }
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < E; i += 2)
+    packed |= e4m3x2_bits(__fdiv_rn(v[i], s), __fdiv_rn(v[i + 1], s)) << (8 * i);
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint32_t*>(codes + row * D + lane * E) = packed;
+  } else {
+    *reinterpret_cast<uint16_t*>(codes + row * D + lane * E) = (uint16_t)packed;
+  }
+  if (lane == 0) xs[row] = s;
+}
+
+// V: one CTA per (batch, head), thread = channel: amax over the tokens, then codes.
+template <int D>
+__global__ void __launch_bounds__(D) quant_fp8_channels_kernel(const uint16_t* __restrict__ x,
+                                                                uint8_t* __restrict__ codes,
+                                                                float* __restrict__ xs, int N) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  const uint16_t* src = x + (size_t)bh * N * D + c;
+  float amax = 0.f;
+  for (int n = 0; n < N; ++n) amax = fmaxf(amax, fabsf(bf16_to_f32(src[(size_t)n * D])));
+  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+  uint8_t* dst = codes + (size_t)bh * N * D + c;
+  for (int n = 0; n < N; ++n)
+    dst[(size_t)n * D] = (uint8_t)(e4m3x2_bits(__fdiv_rn(bf16_to_f32(src[(size_t)n * D]), s), 0.f) & 0xFFu);
+  xs[(size_t)bh * D + c] = s;
+}
+
 }  // namespace ta

@@ -29,7 +29,7 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "normal_bf16", "make_qkv", "outlier_channels"]
+__all__ = ["Workload", "WORKLOADS", "normal_bf16", "make_qkv", "outlier_channels", "rotation_signs"]
 
 
 @dataclass(frozen=True)
@@ -134,3 +134,12 @@ def make_qkv(w: Workload | str, seed: int = 0, device="cpu", B: int | None = Non
     k = normal_bf16((B, H, Nkv, d), gen, dev, w.input_scale, gain)
     v = normal_bf16((B, H, Nkv, d), gen, dev, w.input_scale, gain)
     return q, k, v
+
+
+def rotation_signs(d: int, seed: int = 0) -> torch.Tensor:
+    """Seeded random sign vector (fp32 +-1, CPU) for the FP8 path's rotation:
+    d Bernoulli(1/2) draws of a torch CPU generator, mapped {0, 1} -> {-1, +1}.
+    The rotation draws these numbers; both implementations receive them."""
+    g = torch.Generator()
+    g.manual_seed(seed + 7_000_003)
+    return (torch.randint(0, 2, (d,), generator=g, dtype=torch.int64) * 2 - 1).to(torch.float32)
