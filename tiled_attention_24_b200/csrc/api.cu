@@ -561,11 +561,18 @@ int attn_quantize_fp8(const attn_bf16_t* x, uint8_t* codes, float* scales, int B
     else
       ta::quant_fp8_rows_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(x, signs, codes, scales, rows);
   } else {
-    if (BH > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    if (d == 128)
-      ta::quant_fp8_channels_kernel<128><<<(unsigned)BH, 128, 0, st>>>(x, codes, scales, N);
-    else
-      ta::quant_fp8_channels_kernel<64><<<(unsigned)BH, 64, 0, st>>>(x, codes, scales, N);
+    if (BH > 65535 || BH * d > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    unsigned* amax = reinterpret_cast<unsigned*>(scales);  // amax bits first, scales at the end
+    if (cudaMemsetAsync(amax, 0, BH * d * sizeof(float), st) != cudaSuccess) return ATTN_ERR_CUDA;
+    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)BH);
+    if (d == 128) {
+      ta::channel_amax_kernel<128><<<grid, 256, 0, st>>>(x, amax, N);
+      ta::channel_codes_kernel<128><<<grid, 256, 0, st>>>(x, amax, codes, N);
+    } else {
+      ta::channel_amax_kernel<64><<<grid, 256, 0, st>>>(x, amax, N);
+      ta::channel_codes_kernel<64><<<grid, 256, 0, st>>>(x, amax, codes, N);
+    }
+    ta::channel_scale_kernel<<<(unsigned)((BH * d + 255) / 256), 256, 0, st>>>(amax, (int)(BH * d));
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -10,7 +10,8 @@
 //   S  = codes(Q) codes(K_j)^T                 fp32 in TMEM
 //   x  = S * s_Q[row] * s_K[key] * scale * log2(e) / rot_d     (rot_d = d when
 //        Q and K were rotated: the rotation multiplies Q K^T by d)
-//   P~ = e4m3_rne(2^(x - m))   (unit scale),   l += sum P~
+//   P~ = e4m3_rne(2^(x - m))   (unit scale),   l += sum P~ (by the tensor
+//        core: P~ times a 128 x 16 matrix of ones, into TMEM)
 //   O += P~ codes(V_j)                          fp32 in TMEM, corrected in
 //        place by 2^(m_old - m) when the max grows
 //   O_c = O_c * s_V[c] / l (fp32 output), LSE = ln2 * (m + log2 l).
@@ -19,11 +20,14 @@
 // 1 MMA issuer, 2-3 idle (registers given to the softmax warps), 4-7 and 8-11
 // softmax / correction / epilogue of tiles 0 and 1 (thread = row).  One TMEM
 // score buffer shared by the tiles (moved to registers at once, then released
-// to the other tile), O_0 [128,256), O_1 [256,384), P~ tiles (A operand of
-// P V, 128 keys = 32 columns) [384 + 64 t + 32 (j % 2), +32).  MMA order as
-// the FP4 kernel: S_0(0), S_1(0), S_0(1), then per block P V_0(j), S_1(j+1),
-// P V_1(j), S_0(j+2).  Shared memory: Q tiles and a ring of K / V tiles
-// (128 x 128 bytes, 128-byte swizzle), per-warp key constants.  d = 128 only.
+// to the other tile), O_0 [128,256), O_1 [256,384), P~ of tile t (A operand
+// of P V, 128 keys = 32 columns) [384 + 32 t, +32), row sums l_t
+// [448 + 16 t, +16) (column 0 read).  One P~ buffer per tile: the softmax
+// waits for P V_t(j-1) before it stores P~_t(j) (its exps are already in
+// registers by then).  MMA order as the FP4 kernel: S_0(0), S_1(0), S_0(1),
+// then per block P V_0(j), S_1(j+1), P V_1(j), S_0(j+2).  Shared memory: Q
+// tiles and a ring of K / V tiles (128 x 128 bytes, 128-byte swizzle), the
+// ones matrix, per-warp key constants.  d = 128 only.
 #pragma once
 #include "ptx.cuh"
 #include "fwd_bf16.cuh"  // fwd_tile_kv_count, wait_bar_drain
@@ -54,7 +58,8 @@ struct FwdF8Cfg {
   static constexpr int NSLOT = 8;
   static constexpr int Q_OFF = 0;                         // Q_0, Q_1
   static constexpr int SLOT_OFF = 2 * TILE;
-  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;  // [8 warps][2 bufs][128] floats
+  static constexpr int ONES_OFF = SLOT_OFF + NSLOT * TILE;  // 16 x 128 e4m3 ones (0x38)
+  static constexpr int KC_OFF = ONES_OFF + 2048;            // [8 warps][2 bufs][128] floats
   static constexpr int BAR_OFF = KC_OFF + 8 * 2 * 128 * 4;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
   static constexpr int THREADS = 384;
@@ -63,7 +68,8 @@ struct FwdF8Cfg {
   static constexpr int REG_LOW = 72, REG_HIGH = 216;
   static constexpr uint32_t ID_S = idesc_f8(128, false);
   static constexpr uint32_t ID_PV = idesc_f8(128, true);  // V is MN-major
-  static constexpr uint32_t T_S = 0, T_O = 128, T_P8 = 384;
+  static constexpr uint32_t ID_L = idesc_f8(16, false);   // P~ x ones: row sums
+  static constexpr uint32_t T_S = 0, T_O = 128, T_P8 = 384, T_L = 448;
 };
 
 struct FwdF8Bars {
@@ -72,7 +78,7 @@ struct FwdF8Bars {
   uint64_t kv_empty[8];
   uint64_t s_full[2];     // MMA -> softmax of tile t: S_t(j) in the score buffer
   uint64_t s_free;        // softmax -> MMA: the score buffer's scores are in registers
-  uint64_t p_full[2][2];  // [tile][j % 2]: P~_t(j) in TMEM, O_t corrected
+  uint64_t p_full[2][2];  // [tile][j % 2]: P~_t(j) in TMEM, O_t and l_t corrected
   uint64_t pv_done[2];    // [tile]: P V_t(j) finished
   uint64_t o_full[2];
   uint64_t drain;
@@ -97,28 +103,10 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// two e4m3 codes (one 16-bit pair, low byte first) -> f16x2 values
-__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t pair) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(pair));
-  return r;
-}
 __device__ __forceinline__ uint32_t e4m3x2_pair(float lo, float hi) {  // non-negative inputs
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
-}
-__device__ __forceinline__ uint32_t hadd2_f8(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-__device__ __forceinline__ float f16x2_sum_f8(uint32_t v) {
-  float lo, hi;
-  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(v));
-  return lo + hi;
 }
 
 __global__ void __launch_bounds__(384, 1)
@@ -168,6 +156,11 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
+  // constant B operand of the row-sum MMA: e4m3 ones (every byte 0x38, so the
+  // swizzle does not matter)
+  for (int i = threadIdx.x; i < 2048 / 16; i += C::THREADS)
+    *reinterpret_cast<uint4*>(smem + C::ONES_OFF + i * 16) = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -214,6 +207,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dQ0 = smem_desc(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dK0 = smem_desc(sbase + C::SLOT_OFF, 16, 1024);
       const uint64_t dV0 = smem_desc(sbase + C::SLOT_OFF, C::TILE, 1024);
+      const uint64_t dOnes = smem_desc(sbase + C::ONES_OFF, 16, 1024);
       int n_s = 0;  // S MMAs issued so far (the score buffer's uses)
       auto issue_S = [&](int t, int j) -> bool {
         if (n_s > 0) {
@@ -247,10 +241,14 @@ __global__ void __launch_bounds__(384, 1)
         if (!wait_bar(smem_u32(&bars->p_full[t][j & 1]), (j >> 1) & 1, abort_flag, p.timeout_ns)) return false;
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)(s * (C::TILE >> 4));
-        const uint32_t aP = tbase + C::T_P8 + 64 * t + 32 * (j & 1);
+        const uint32_t aP = tbase + C::T_P8 + 32 * t;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 keys per MMA: 8 P~ columns / 32 rows x 128 B of V
           mma_f8_ts(tbase + C::T_O + 128 * t, aP + kk * 8, dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // l_t += P~ 1
+          mma_f8_ts(tbase + C::T_L + 16 * t, aP + kk * 8, dOnes + (uint64_t)(kk * 2), C::ID_L,
                     (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(smem_u32(&bars->pv_done[t]));
         if (last) tc_commit(smem_u32(&bars->kv_empty[s]));
@@ -287,6 +285,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tbase + lane_off + C::T_S;
     const uint32_t tO = tbase + lane_off + C::T_O + 128 * t;
+    const uint32_t tL = tbase + lane_off + C::T_L + 16 * t;
     const int off = p.Nkv - p.Nq;
     const float qs_row = (present[t] && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] : 0.f;
     const float* ksrow = p.k_scale + (size_t)bh * p.Nkv;
@@ -310,7 +309,7 @@ __global__ void __launch_bounds__(384, 1)
       *reinterpret_cast<float4*>(kcbuf + (jj & 1) * 128 + lane * 4) =
           make_float4(ks_next.x * p.sl2, ks_next.y * p.sl2, ks_next.z * p.sl2, ks_next.w * p.sl2);
     };
-    float m_ref = -INFINITY, l = 0.f;
+    float m_ref = -INFINITY;  // l lives in TMEM (column tL), summed by the tensor core
     bool ok = present[t];
     if (ok && n[t] > 0) {
       load_ks(0);
@@ -377,13 +376,11 @@ __global__ void __launch_bounds__(384, 1)
       float factor = 1.f;
       if (grow) {
         factor = had ? ex2(m_ref - m_blk) : 0.f;
-        l *= factor;
         m_ref = m_blk;
       }
       const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const uint64_t qs2 = f2(qs_row, qs_row), nm2 = f2(negm, negm);
-      // P~ = e4m3(2^(x - m)); l sums the values the MMA multiplies (f16 sums
-      // of 4 values <= 4 on the 2^-9 grid are exact)
+      // P~ = e4m3(2^(x - m))
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -395,18 +392,18 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t lo = e4m3x2_pair(ex2(a0), ex2(a1));
           const uint32_t hi = e4m3x2_pair(ex2(a2), ex2(a3));
           pk[c * 8 + i / 4] = lo | (hi << 16);
-          l += f16x2_sum_f8(hadd2_f8(e4m3x2_f16x2(lo), e4m3x2_f16x2(hi)));
         }
       }
-      // P~_t(j) -> its TMEM tile; P V_t(j-2) read it last and finished
-      // before S_t(j) was computed (the S_t(j) commit covers earlier MMAs)
-      tmem_st32(tbase + lane_off + C::T_P8 + 64 * t + 32 * (j & 1), pk);
-      if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
-        // rescale O_t (blocks < j) to the new reference
+      if (j > 0) {
+        // P V_t(j-1) and its row sum have read the P~ buffer and finished
         ok = wait_bar(smem_u32(&bars->pv_done[t]), (j - 1) & 1, abort_flag, p.timeout_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
+      }
+      tmem_st32(tbase + lane_off + C::T_P8 + 32 * t, pk);
+      if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
+        // rescale O_t and l_t (blocks < j) to the new reference
         const float f = (grow && had) ? factor : 1.f;
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -417,6 +414,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
           tmem_st32(tO + cc * 32, o);
         }
+        uint32_t lv = tmem_ld1(tL);
+        tmem_ld_wait1(lv);
+        tmem_st1(tL, __float_as_uint(__uint_as_float(lv) * f));
       }
       tmem_st_wait();
       __syncwarp();  // the staged key constants of block j + 1 are visible to the warp
@@ -430,6 +430,12 @@ __global__ void __launch_bounds__(384, 1)
       if (ok) tc_fence_after();
     }
     if (ok) {
+      float l = 0.f;  // no block visible: no row-sum MMA ran, the column is stale
+      if (n[t] > 0) {
+        uint32_t lv = tmem_ld1(tL);
+        tmem_ld_wait1(lv);
+        l = __uint_as_float(lv);
+      }
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const float* vs = p.v_scale + (size_t)bh * 128;
       float* orow = p.o + ((size_t)bh * p.Nq + row) * 128;

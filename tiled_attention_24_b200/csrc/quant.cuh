@@ -299,20 +299,76 @@ __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const uint16_t* __r
   if (lane == 0) xs[row] = s;
 }
 
-// V: one CTA per (batch, head), thread = channel: amax over the tokens, then codes.
+// V: one scale per (batch, head, channel) over the head's tokens.  Three
+// passes over chunks of 128 tokens (grid: chunks x BH): per-channel amax
+// (atomicMax on the bit patterns of non-negative floats, into the scale
+// buffer), codes (each block derives the scales from the amax), then the
+// amax words become the scales in place.  A thread covers 8 channels (16 B).
 template <int D>
-__global__ void __launch_bounds__(D) quant_fp8_channels_kernel(const uint16_t* __restrict__ x,
-                                                                uint8_t* __restrict__ codes,
-                                                                float* __restrict__ xs, int N) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  const uint16_t* src = x + (size_t)bh * N * D + c;
-  float amax = 0.f;
-  for (int n = 0; n < N; ++n) amax = fmaxf(amax, fabsf(bf16_to_f32(src[(size_t)n * D])));
-  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
-  uint8_t* dst = codes + (size_t)bh * N * D + c;
-  for (int n = 0; n < N; ++n)
-    dst[(size_t)n * D] = (uint8_t)(e4m3x2_bits(__fdiv_rn(bf16_to_f32(src[(size_t)n * D]), s), 0.f) & 0xFFu);
-  xs[(size_t)bh * D + c] = s;
+__global__ void __launch_bounds__(256) channel_amax_kernel(const uint16_t* __restrict__ x,
+                                                           unsigned* __restrict__ amax_bits, int N) {
+  constexpr int G = D / 8, R = 256 / G;  // channel groups, token rows per pass
+  const int bh = blockIdx.y, g = threadIdx.x % G, r = threadIdx.x / G;
+  const int n0 = blockIdx.x * 128, n1 = min(N, n0 + 128);
+  const uint16_t* src = x + ((size_t)bh * N) * D + g * 8;
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int n = n0 + r; n < n1; n += R) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src + (size_t)n * D);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(u[i] << 16)));
+      m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
+    }
+  }
+  __shared__ float part[R][D];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[r][g * 8 + i] = m[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float a = 0.f;
+    for (int k = 0; k < R; ++k) a = fmaxf(a, part[k][threadIdx.x]);
+    atomicMax(amax_bits + (size_t)bh * D + threadIdx.x, __float_as_uint(a));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) channel_codes_kernel(const uint16_t* __restrict__ x,
+                                                            const unsigned* __restrict__ amax_bits,
+                                                            uint8_t* __restrict__ codes, int N) {
+  constexpr int G = D / 8, R = 256 / G;
+  const int bh = blockIdx.y, g = threadIdx.x % G, r = threadIdx.x / G;
+  const int n0 = blockIdx.x * 128, n1 = min(N, n0 + 128);
+  float sc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = __uint_as_float(amax_bits[(size_t)bh * D + g * 8 + i]);
+    sc[i] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
+  }
+  const uint16_t* src = x + ((size_t)bh * N) * D + g * 8;
+  uint8_t* dst = codes + ((size_t)bh * N) * D + g * 8;
+  for (int n = n0 + r; n < n1; n += R) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src + (size_t)n * D);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    uint32_t out[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t pr = e4m3x2_bits(__fdiv_rn(__uint_as_float(u[i] << 16), sc[2 * i]),
+                                      __fdiv_rn(__uint_as_float(u[i] & 0xFFFF0000u), sc[2 * i + 1]));
+      if (i & 1)
+        out[i >> 1] |= pr << 16;
+      else
+        out[i >> 1] = pr;
+    }
+    *reinterpret_cast<uint2*>(dst + (size_t)n * D) = make_uint2(out[0], out[1]);
+  }
+}
+
+__global__ void channel_scale_kernel(unsigned* amax_bits, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float amax = __uint_as_float(amax_bits[i]);
+  amax_bits[i] = __float_as_uint((amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f));
 }
 
 }  // namespace ta
