@@ -321,9 +321,11 @@ ATTN_API int attn_quantize_fp8(const attn_bf16_t* x, uint8_t* codes, float* scal
  *   S = codes(q) codes(k)^T (fp32 accumulation of exact e4m3 products);
  *   x = S * q_scale[i] * k_scale[j] * scale * log2(e) / r, r = d when q and k
  *   were rotated (rotated != 0: the rotation multiplies q k^T by d), else 1;
- *   per block of 128 keys the running row max m moves on every increase,
- *   P~ = e4m3(2^(x - m)) (values in [0, 1], unit scale), l = l 2^(m_old - m) +
- *   sum P~, acc = acc 2^(m_old - m) + P~ codes(v);
+ *   per block of 128 keys a reference row max m moves to the block max only
+ *   when that exceeds it by more than 8 (lazy rescaling, [FA4-overview]
+ *   "Smarter online softmax rescaling"), P~ = e4m3(2^(x - m)) (values in
+ *   [0, 256], unit scale), l = l 2^(m_old - m) + sum P~,
+ *   acc = acc 2^(m_old - m) + P~ codes(v);
  *   O[i][c] = acc[i][c] * v_scale[c] / l (fp32), LSE = ln 2 (m + log2 l).
  *   q [B][H][Nq][128] codes + q_scale [B][H][Nq]; k [B][H][Nkv][128] codes +
  *   k_scale [B][H][Nkv]; v [B][H][Nkv][128] codes + v_scale [B][H][128]

@@ -26,9 +26,13 @@ not the formulas; the readings taken here:
   3. S = sum_c deq(Q)_ic deq(K)_jc without the scales (exact e4m3 products,
      fp64 sum), rounded once to fp32; x = S * s_Q[i] * s_K[j] * scale *
      log2(e) / d, masked.
-  4. blockwise over B_c = 128 keys, the running max moved on every increase
-     (tau = 0, so P <= 1): P~ = e4m3(2^(x - m)) with unit scale,
-     l = l * 2^(m_old - m) + sum P~,  acc = acc * 2^(m_old - m) + P~ . codes(V).
+  4. blockwise over B_c = 128 keys with a reference max m that moves to the
+     block max only when that exceeds it by more than tau ([FA4-overview]
+     "Smarter online softmax rescaling"; tau = 0 moves it on every increase):
+     P~ = e4m3(2^(x - m)) with unit scale, l = l * 2^(m_old - m) + sum P~,
+     acc = acc * 2^(m_old - m) + P~ . codes(V).  The FP8 kernel takes tau = 8:
+     P~ <= 2^8 = 256 stays inside e4m3's finite range (448), and the precision
+     of e4m3 is the same in every binade of its normal range.
   5. O_c = acc_c * s_V[c] / l, LSE = ln2 (m + log2 l).
 """
 from __future__ import annotations
@@ -106,7 +110,7 @@ def quantize_fp8_channels(v):
 
 
 def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=128,
-                  with_flip_bound=False, rows=None):
+                  with_flip_bound=False, rows=None, tau=0.0):
     """Emulated FP8 forward (steps 3-5 of the module docstring) from code values
     and scales; ``rot_d`` = d when Q and K were rotated (the product is then d
     times Q K^T), 1 otherwise.  Returns (O, LSE) float64 and, with
@@ -126,9 +130,9 @@ def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=
     LB = np.zeros((B, H, Nq))
     flips = 0
     vis = visible_mask(Nq_all, Nkv, causal, ridx)
-    # e4m3 rounding midpoints in (0, 1]: the value between two neighbours
+    # e4m3 rounding midpoints up to the largest P~ (2^tau): the value between two neighbours
     mids = (UE4M3_VALUES[:-1] + UE4M3_VALUES[1:]) / 2.0
-    mids = mids[mids <= 1.0]
+    mids = mids[mids <= 2.0 ** tau * 1.07]
     for b in range(B):
         for h in range(H):
             S = (qv[b, h, ridx] @ kv[b, h].T).astype(F32).astype(np.float64)
@@ -142,13 +146,14 @@ def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=
                 cols = slice(j0, min(Nkv, j0 + Bc))
                 xb = x[:, cols]
                 m_new = np.maximum(m, xb.max(axis=1))
-                grow = np.isfinite(m) & (m_new > m)
+                move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
+                grow = move & np.isfinite(m)
                 f = np.ones_like(m)
                 with np.errstate(invalid="ignore"):  # -inf - -inf where not grow (not used)
                     np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
-                m = m_new
+                m = np.where(move, m_new, m)
                 ms = np.where(np.isfinite(m), m, 0.0)
                 fin = np.isfinite(xb) & np.isfinite(m)[:, None]
                 p = np.zeros_like(xb)

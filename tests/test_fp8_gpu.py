@@ -3,7 +3,8 @@ oracle, through the C ABI.
 
 * quantisers (rotation by the fast Walsh-Hadamard transform, per-row and
   per-channel e4m3): bit-exact codes and fp32 scales;
-* forward: within 5e-3 max-abs of the oracle's step-by-step FP8 emulation plus,
+* forward: within 5e-3 max-abs of the oracle's step-by-step FP8 emulation
+  (lazy rescale threshold 8, as the kernel) plus,
   for rows where a P element sat within fp32 evaluation error of an e4m3
   rounding midpoint, the oracle's bound on what that rounding can change.
 """
@@ -76,7 +77,8 @@ def _check_fp8(ta, q, k, v, causal, scale, rotate, rows=None, what="", seed=0):
     rkv, rks = F.quantize_fp8_rows(k, sn)
     rvv, rvs = F.quantize_fp8_channels(v)
     O, L, FB, LB, flips = F.attention_fp8(rqv, rqs, rkv, rks, rvv, rvs, causal, scale,
-                                          rot_d=d if rotate else 1, with_flip_bound=True, rows=rows)
+                                          rot_d=d if rotate else 1, with_flip_bound=True, rows=rows,
+                                          tau=8.0)
     og, lg = _np(o).astype(np.float64), _np(lse).astype(np.float64)
     if rows is not None:
         og, lg = og[:, :, rows], lg[:, :, rows]

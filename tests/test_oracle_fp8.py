@@ -111,3 +111,40 @@ def test_fp8_emulation_close_to_exact_attention():
     cos = (O * Oe).sum() / (np.linalg.norm(O) * np.linalg.norm(Oe))
     # P in e4m3 (3 mantissa bits) moves l, hence LSE, by a few per cent at most
     assert cos > 0.995 and np.abs(L - Le).max() < 0.1
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_integer_scores_are_exact_for_every_tau(tau):
+    """Base-2 scores that are integers: every P~ = 2^(x - m) the recurrence
+    forms (x - m in [-9, 8]) is an e4m3 value, so the blockwise emulation with
+    either threshold must equal the softmax definition 2^S / sum 2^S exactly
+    (up to fp64 rounding).  The patterns make the reference move inside later
+    blocks, stay stale by up to 7 (tau = 8), and jump past the threshold."""
+    pat = np.array([[0, 1, 0, 2, 3, 9, 1, 0, 11, 2, 4, 9, 5, 6, 3, 10],
+                    [10, 9, 8, 7, 6, 5, 4, 3, 2, 1, 4, 8, 12, 3, 11, 9]], dtype=np.float64)
+    N = pat.shape[1]
+    qv = np.eye(2)[None, None]                      # row c picks pattern c
+    kv = pat.T[None, None]                          # S[c, j] = pat[c, j]
+    g = np.random.default_rng(3)
+    vv = F.UE4M3_VALUES[g.integers(0, 100, size=(1, 1, N, 2))] * np.where(g.random((1, 1, N, 2)) < 0.5, -1, 1)
+    one = np.ones((1, 1, 2), np.float32)
+    O, L = F.attention_fp8(qv, one, kv, np.ones((1, 1, N), np.float32), vv, one, False, math.log(2.0),
+                           rot_d=1, Bc=4, tau=tau)
+    w = 2.0 ** pat
+    Oe = (w @ vv[0, 0]) / w.sum(axis=1)[:, None]
+    np.testing.assert_allclose(O[0, 0], Oe, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(L[0, 0], np.log(w.sum(axis=1)), rtol=0, atol=1e-13)
+
+
+def test_lazy_threshold_changes_only_the_rounding():
+    """On random rotated inputs tau = 8 and tau = 0 differ only through where
+    P~ is rounded: both stay within the e4m3 error of each other."""
+    g = np.random.default_rng(5)
+    q = g.standard_normal((1, 2, 64, 128)).astype(np.float32)
+    k = g.standard_normal((1, 2, 512, 128)).astype(np.float32)
+    v = g.standard_normal((1, 2, 512, 128)).astype(np.float32)
+    sg = np.where(g.random(128) < 0.5, -1.0, 1.0)
+    a = F.quantize_fp8_rows(q, sg) + F.quantize_fp8_rows(k, sg) + F.quantize_fp8_channels(v)
+    O0, L0 = F.attention_fp8(*a, False, 128 ** -0.5, rot_d=128, tau=0.0)
+    O8, L8 = F.attention_fp8(*a, False, 128 ** -0.5, rot_d=128, tau=8.0)
+    assert np.abs(O0 - O8).max() < 0.02 and np.abs(L0 - L8).max() < 0.01

@@ -6,12 +6,15 @@
 // (randomised Hadamard, see the FP8 quantisers) before the quantisation.
 // Operands: e4m3 codes with one fp32 scale per Q / K token row and one per V
 // channel.  Steps per 128-key block j (tiling, masking, online softmax as the
-// bf16 kernel; the running max moves on every increase, so P <= 1):
+// bf16 kernel):
 //   S  = codes(Q) codes(K_j)^T                 fp32 in TMEM
 //   x  = S * s_Q[row] * s_K[key] * scale * log2(e) / rot_d     (rot_d = d when
 //        Q and K were rotated: the rotation multiplies Q K^T by d)
 //   P~ = e4m3_rne(2^(x - m))   (unit scale),   l += sum P~ (by the tensor
 //        core: P~ times a 128 x 16 matrix of ones, into TMEM)
+//   m: lazy reference max ("FlashAttention 4" page, smarter online softmax
+//        rescaling): it moves to the block max only when that exceeds it by
+//        more than TAU = 8, so P~ <= 2^8 = 256 stays inside e4m3's range (448)
 //   O += P~ codes(V_j)                          fp32 in TMEM, corrected in
 //        place by 2^(m_old - m) when the max grows
 //   O_c = O_c * s_V[c] / l (fp32 output), LSE = ln2 * (m + log2 l).
@@ -66,6 +69,7 @@ struct FwdF8Cfg {
   // register split (launch: 384 threads x 168): warpgroup 0 drops to 72, the
   // two softmax warpgroups rise to 216: 128*72 + 256*216 = 64512 = 384*168
   static constexpr int REG_LOW = 72, REG_HIGH = 216;
+  static constexpr float TAU = 8.f;  // lazy-rescale threshold (log2 units)
   static constexpr uint32_t ID_S = idesc_f8(128, false);
   static constexpr uint32_t ID_PV = idesc_f8(128, true);  // V is MN-major
   static constexpr uint32_t ID_L = idesc_f8(16, false);   // P~ x ones: row sums
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       // s_Q > 0, so max(y) * s_Q is the row max of x
       const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * qs_row;
-      const bool grow = m_blk > m_ref;  // tau = 0
+      const bool grow = m_blk > m_ref + C::TAU;  // -inf + TAU = -inf: the first finite block moves it
       const bool had = m_ref != -INFINITY;
       float factor = 1.f;
       if (grow) {
