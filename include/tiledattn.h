@@ -164,6 +164,42 @@ ATTN_API int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const a
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_varlen -- attn_fwd over a batch of sequences of different lengths
+ * packed without padding ([FA4-overview] "Compatibility and current status":
+ * variable-length batches).  Sequence b owns query rows
+ * [cu_seqlens_q[b], cu_seqlens_q[b+1]) and keys [cu_seqlens_k[b],
+ * cu_seqlens_k[b+1]); it attends only to its own keys, with the causal rule
+ * of this header applied per sequence (N_q, N_kv = its own lengths).
+ *   q, o  bf16 [total_q][H][d]   (token-major packing, 16-byte aligned)
+ *   k, v  bf16 [total_k][Hkv][d] (grouped-query when Hkv < H; H % Hkv == 0)
+ *   lse   fp32 [H][total_q]
+ *   cu_seqlens_q, cu_seqlens_k  int32 [B + 1] DEVICE arrays, non-decreasing,
+ *         starting at 0 (offsets are clamped to [0, total] on the device).
+ *   max_seqlen_q  >= every sequence's query length (sets the grid; rows of a
+ *         longer sequence past it are not written).
+ *   Rows outside every sequence are not written.  A sequence with no keys
+ *   gets O = 0, LSE = -inf.  d in {64, 128}.
+ */
+ATTN_API int attn_fwd_varlen(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                             float* lse, const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int Hkv,
+                             int total_q, int total_k, int max_seqlen_q, int d, int causal, float scale,
+                             void* stream);
+
+/*
+ * attn_decode_varlen -- attn_decode_gqa with a cache length per batch entry
+ * (variable-length batches, as attn_fwd_varlen): batch b attends to keys
+ * [0, seqlens_k[b]) of its cache (clamped to [0, Nkv_max]); each entry's
+ * keys are split into num_splits chunks of its own length.  An entry with no
+ * keys gets O = 0, LSE = -inf.
+ *   q [B][H][1][d], k/v [B][Hkv][Nkv_max][d] bf16, seqlens_k int32 [B] DEVICE
+ *   array; o, lse, workspace as attn_decode.
+ */
+ATTN_API int attn_decode_varlen(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                                float* lse, const int* seqlens_k, int B, int H, int Hkv, int Nkv_max, int d,
+                                float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * attn_decode_noalloc -- the same split-KV decode as attn_decode, for callers
  * that cannot allocate device memory: code that runs where cudaMalloc is not
  * allowed or not wanted (inside a caller's own memory pool or allocator hook,

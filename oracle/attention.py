@@ -324,3 +324,49 @@ def decode(q, k, v, scale: float | None = None):
     """Decode reference: one (or a few) query rows against the whole cache,
     which is the plain definition (non-causal over all cached keys)."""
     return attention(q, k, v, causal=False, scale=scale)
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, causal: bool = False, scale: float | None = None):
+    """Variable-length batch packed without padding ([FA4-overview]
+    "Compatibility and current status": variable-length sequences): q
+    [total_q][Hq][d], k/v [total_k][Hkv][d] token-major; sequence b owns rows
+    [cu_q[b], cu_q[b+1]) and keys [cu_k[b], cu_k[b+1]) and is the plain
+    definition on its own rows and keys (causal alignment per sequence).
+    Returns O [total_q][Hq][d] (rows outside every sequence are 0) and LSE
+    [Hq][total_q] (-inf there)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu_q, cu_k = np.asarray(cu_q, dtype=np.int64), np.asarray(cu_k, dtype=np.int64)
+    total_q, Hq, d = q.shape
+    O = np.zeros((total_q, Hq, v.shape[2]))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        if q1 <= q0:
+            continue
+        qb = q[q0:q1].transpose(1, 0, 2)[None]          # [1][Hq][n][d]
+        if k1 <= k0:
+            LSE[:, q0:q1] = -np.inf                       # no key: O = 0
+            continue
+        kb = k[k0:k1].transpose(1, 0, 2)[None]
+        vb = v[k0:k1].transpose(1, 0, 2)[None]
+        Ob, Lb = attention_gqa(qb, kb, vb, causal, scale)
+        O[q0:q1] = Ob[0].transpose(1, 0, 2)
+        LSE[:, q0:q1] = Lb[0]
+    return O, LSE
+
+
+def decode_varlen(q, k, v, seqlens, scale: float | None = None):
+    """Decode with a cache length per batch entry: entry b attends to keys
+    [0, seqlens[b]) of k/v [B][Hkv][Nmax][d] (grouped-query when Hkv < Hq);
+    an entry with no keys gets O = 0, LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    O = np.zeros((B, Hq, Nq, v.shape[3]))
+    LSE = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        n = int(seqlens[b])
+        if n <= 0:
+            continue
+        Ob, Lb = attention_gqa(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], False, scale)
+        O[b], LSE[b] = Ob[0], Lb[0]
+    return O, LSE

@@ -122,6 +122,25 @@ def test_fp8_host_validation(lib):
     assert fwd(vs=ctypes.c_void_p(16 * 1000 + 4)) == -3 and fwd(Nq=0) == 0
 
 
+def test_varlen_host_validation(lib):
+    def fwd(**kw):
+        a = dict(cuq=P, cuk=P, B=2, H=4, Hkv=2, tq=100, tk=100, mq=64, d=128, scale=0.1, q=P)
+        a.update(kw)
+        return lib.attn_fwd_varlen(a["q"], P, P, P, P, a["cuq"], a["cuk"], a["B"], a["H"], a["Hkv"], a["tq"],
+                                   a["tk"], a["mq"], a["d"], 0, a["scale"], None)
+    assert fwd(d=96) == -2 and fwd(Hkv=3) == -1 and fwd(cuq=None) == -1 and fwd(tq=-1) == -1
+    assert fwd(scale=0.0) == -1 and fwd(q=ctypes.c_void_p(16 * 1000 + 8)) == -3
+    assert fwd(cuk=ctypes.c_void_p(16 * 1000 + 2)) == -3 and fwd(tq=0) == 0 and fwd(B=0) == 0
+    n = lib.attn_decode_workspace_bytes(2, 4, 128, 4)
+    def dec(**kw):
+        a = dict(lens=P, B=2, H=4, Hkv=2, N=100, d=128, S=4)
+        a.update(kw)
+        return lib.attn_decode_varlen(P, P, P, P, P, a["lens"], a["B"], a["H"], a["Hkv"], a["N"], a["d"], 0.1,
+                                      a["S"], ctypes.c_void_p(16 * 4096), n, None)
+    assert dec(lens=None) == -1 and dec(lens=ctypes.c_void_p(16 * 1000 + 2)) == -3 and dec(d=80) == -2
+    assert dec(S=0) == -1 and dec(N=0) == -1 and dec(B=0) == 0
+
+
 def test_product_path_never_imports_the_oracle():
     """The package must not reach the oracle (no CPU fallback)."""
     pkg = os.path.join(ROOT, "tiled_attention_24_b200")

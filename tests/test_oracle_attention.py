@@ -278,3 +278,73 @@ def test_backward_row_statistic_identity():
     P = A.softmax_rows(q, k, False, 0.5)
     dP = do.numpy() @ v.numpy().transpose(0, 1, 3, 2)
     assert np.abs((P * dP).sum(-1) - (do.numpy() * O).sum(-1)).max() < 1e-12
+
+
+def _packed_mask(cu_q, cu_k, causal):
+    """Boolean [total_q][total_k]: query row i sees key j iff both belong to the
+    same sequence (and, causal, j - k0 <= (i - q0) + (nk - nq))."""
+    tq, tk = cu_q[-1], cu_k[-1]
+    m = torch.zeros(tq, tk, dtype=torch.bool)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        i = torch.arange(q0, q1)[:, None] - q0
+        j = torch.arange(k0, k1)[None, :] - k0
+        vis = torch.ones(q1 - q0, k1 - k0, dtype=torch.bool)
+        if causal:
+            vis = j <= i + ((k1 - k0) - (q1 - q0))
+        m[q0:q1, k0:k1] = vis
+    return m
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
+def test_varlen_matches_block_diagonal_sdpa(causal, Hq, Hkv):
+    """The packed batch equals one attention over the concatenation with a
+    block-diagonal mask (PyTorch SDPA, fp64), and LSE equals the masked
+    log-sum-exp; rows that see no key (empty key set, or causal with fewer
+    keys than queries) get O = 0, LSE = -inf."""
+    lq = [5, 0, 17, 3, 9]
+    lk = [7, 4, 17, 0, 4]
+    cu_q = np.concatenate([[0], np.cumsum(lq)])
+    cu_k = np.concatenate([[0], np.cumsum(lk)])
+    g = torch.Generator().manual_seed(11)
+    d = 8
+    q = torch.randn(cu_q[-1], Hq, d, generator=g, dtype=torch.float64)
+    k = torch.randn(cu_k[-1], Hkv, d, generator=g, dtype=torch.float64)
+    v = torch.randn(cu_k[-1], Hkv, d, generator=g, dtype=torch.float64)
+    O, L = A.attention_varlen(q, k, v, cu_q, cu_k, causal, 0.3)
+    mask = _packed_mask(cu_q, cu_k, causal)
+    rep = Hq // Hkv
+    kh, vh = k.repeat_interleave(rep, dim=1), v.repeat_interleave(rep, dim=1)
+    s = torch.einsum("ihd,jhd->hij", q, kh) * 0.3
+    s = s.masked_fill(~mask[None], float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)                        # [H][total_q]
+    seen = mask.any(dim=1).numpy()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(0, 1)[None], kh.transpose(0, 1)[None], vh.transpose(0, 1)[None],
+        attn_mask=mask[None, None], scale=0.3)[0].transpose(0, 1).numpy()
+    np.testing.assert_allclose(O[seen], ref[seen], rtol=0, atol=1e-12)
+    assert (O[~seen] == 0).all() and np.isneginf(L[:, ~seen]).all()
+    np.testing.assert_allclose(L[:, seen], lse.numpy()[:, seen], rtol=0, atol=1e-12)
+    assert (~seen).sum() > 0                                 # the case is covered
+
+
+def test_decode_varlen_matches_masked_sdpa():
+    B, Hq, Hkv, N, d = 4, 4, 2, 23, 8
+    lens = [23, 0, 1, 11]
+    g = torch.Generator().manual_seed(12)
+    q = torch.randn(B, Hq, 1, d, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64)
+    O, L = A.decode_varlen(q, k, v, lens, 0.5)
+    keep = torch.arange(N)[None, :] < torch.tensor(lens)[:, None]          # [B][N]
+    kh, vh = k.repeat_interleave(2, dim=1), v.repeat_interleave(2, dim=1)
+    for b in range(B):
+        if lens[b] == 0:
+            assert (O[b] == 0).all() and np.isneginf(L[b]).all()
+            continue
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[b:b + 1], kh[b:b + 1], vh[b:b + 1], attn_mask=keep[b][None, None, None], scale=0.5)
+        np.testing.assert_allclose(O[b], ref[0].numpy(), rtol=0, atol=1e-12)
+        s = (q[b] @ kh[b].transpose(-1, -2) * 0.5)[..., : lens[b]]
+        np.testing.assert_allclose(L[b], torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)

@@ -12,7 +12,7 @@ import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
                        attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
-                       attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_workspace_bytes,
+                       attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_fwd_varlen, attn_decode_varlen, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_workspace_bytes,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
                        attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
                        attn_status_string, attn_version, attn_watchdog_selftest, load)
@@ -25,6 +25,7 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "attn_fwd_gqa", "attn_decode_gqa", "attn_quantize_int4", "quantize_int4", "forward_int4",
            "attn_bwd", "attn_bwd_workspace_bytes", "backward",
            "attn_quantize_fp8", "attn_fwd_fp8", "quantize_fp8", "forward_fp8", "hadamard_signs",
+           "attn_fwd_varlen", "attn_decode_varlen", "forward_varlen", "decode_varlen",
            "DIRECT_P", "QUANT_AFTER_EXP"]
 
 DIRECT_P, QUANT_AFTER_EXP = 0, 1
@@ -71,6 +72,29 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | Non
         attn_decode_gqa(q, k, v, o, lse, scale, num_splits, workspace, stream)
     else:
         attn_decode(q, k, v, o, lse, scale, num_splits, workspace, stream)
+    return o, lse
+
+
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool = False,
+                   scale: float | None = None, stream=None):
+    """Packed variable-length forward (q [total_q,H,d], k/v [total_k,Hkv,d],
+    cu_seqlens int32 [B+1] on the device).  Returns (o [total_q,H,d], lse [H,total_q])."""
+    total_q, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.zeros_like(q)
+    lse = torch.full((H, total_q), float("-inf"), dtype=torch.float32, device=q.device)
+    attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal, scale, stream)
+    return o, lse
+
+
+def decode_varlen(q, k, v, seqlens_k, scale: float | None = None, num_splits: int = 16, stream=None):
+    """Decode with a cache length per batch entry (seqlens_k int32 [B] on the device)."""
+    B, H, _, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    ws = torch.empty(attn_decode_workspace_bytes(B, H, d, num_splits), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    attn_decode_varlen(q, k, v, o, lse, seqlens_k, scale, num_splits, ws, stream)
     return o, lse
 
 

@@ -34,6 +34,8 @@ SIGNATURES = [
     ("attn_bwd_workspace_bytes", _SZ, [_I, _I, _I]),
     ("attn_bwd", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     ("attn_decode_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
+    ("attn_fwd_varlen", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    ("attn_decode_varlen", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_quantize_int8", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     ("attn_quantize_int4", _I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     ("attn_fwd_int8", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
@@ -169,6 +171,31 @@ def attn_decode_noalloc(q, k, v, o, lse, scale: float, num_splits: int, stream=N
     rc = load().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
                                     int(num_splits), _stream(stream))
     _check("attn_decode_noalloc", rc)
+
+
+def attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, max_seqlen_q: int, causal: bool, scale: float, stream=None):
+    """Packed variable-length forward: q/o [total_q,H,d], k/v [total_k,Hkv,d] bf16,
+    lse [H,total_q] fp32, cu_q/cu_k int32 [B+1] on the device."""
+    _need_cuda(q, k, v, o, lse, cu_q, cu_k)
+    total_q, H, d = q.shape
+    total_k, Hkv, _ = k.shape
+    B = cu_q.shape[0] - 1
+    rc = load().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q), _ptr(cu_k), B, H, Hkv,
+                                total_q, total_k, int(max_seqlen_q), d, int(bool(causal)), float(scale),
+                                _stream(stream))
+    _check("attn_fwd_varlen", rc)
+
+
+def attn_decode_varlen(q, k, v, o, lse, seqlens_k, scale: float, num_splits: int, workspace, stream=None):
+    """Decode with a cache length per batch entry: q [B,H,1,d], k/v [B,Hkv,Nkv_max,d],
+    seqlens_k int32 [B] on the device."""
+    _need_cuda(q, k, v, o, lse, seqlens_k, workspace)
+    B, H, _, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    rc = load().attn_decode_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, Hkv, Nkv,
+                                   d, float(scale), int(num_splits), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_decode_varlen", rc)
 
 
 def attn_quantize_int8(x, xq, xs, per_head: bool, stream=None):

@@ -56,6 +56,22 @@ int make_tmap_bf16(CUtensorMap* m, const void* ptr, int d, int N, int BH) {
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Packed token-major bf16 [total][heads][d] viewed as (d, heads, total);
+// boxes of 64 x 1 x 128 (the same 128-row x 128-byte smem tile as
+// make_tmap_bf16's boxes) with 128-byte swizzle.  Rows past total read as zero.
+int make_tmap_tok(CUtensorMap* m, const void* ptr, int d, int heads, int total) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)total};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // [BH][N][128] int8 viewed as (128, N, BH); boxes of 128 x 128 x 1 bytes with
 // 128-byte swizzle.
 int make_tmap_i8(CUtensorMap* m, const void* ptr, int N, int BH) {
@@ -198,6 +214,41 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 }
 
 template <int D>
+int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q,
+                      const int* cu_k, int B, int H, int Hkv, int total_q, int total_k, int max_q, int causal,
+                      float scale, cudaStream_t st) {
+  using C = ta::FwdCfg<D>;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_tok(&tq, q, D, H, total_q)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_tok(&tk, k, D, Hkv, total_k)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_tok(&tv, v, D, Hkv, total_k)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::fwd_bf16_kernel<D, true>, C::SMEM)) != ATTN_OK) return rc;
+  ta::FwdParams p;
+  p.lse = lse;
+  p.Nq = 0;
+  p.Nkv = 0;
+  p.n_qp = (max_q + 255) / 256;
+  p.Tc = 0;
+  p.group = H / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_ns;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.o = static_cast<uint16_t*>(o);
+  p.nb = B;
+  p.H = H;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  const long long grid = (long long)B * H * p.n_qp;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  // tmO is not used by the variable-length epilogue (direct stores); any valid map will do
+  ta::fwd_bf16_kernel<D, true><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tq, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                void* dq, void* dk, void* dv, float* rowdot, int B, int H, int Nq, int Nkv, int causal, float scale,
                cudaStream_t st) {
@@ -326,6 +377,33 @@ int attn_fwd_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* 
                   : launch_fwd<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, causal, scale, st);
 }
 
+int attn_fwd_varlen(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int Hkv, int total_q,
+                    int total_k, int max_seqlen_q, int d, int causal, float scale, void* stream) {
+  if (B < 0 || H < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv < 1 || (H > 0 && H % Hkv != 0) || Hkv > (H > 0 ? H : Hkv)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || total_q == 0) return ATTN_OK;
+  if (!q || !o || !lse || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned4(lse) || !aligned4(cu_seqlens_q) || !aligned4(cu_seqlens_k) ||
+      (total_k > 0 && (!aligned16(k) || !aligned16(v))))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (total_k == 0) {  // no keys anywhere: every row gets O = 0, LSE = -inf
+    const long long rows = (long long)total_q * H;
+    const long long blocks = (rows * d + 255) / 256;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    ta::fill_empty_kernel<<<(unsigned)blocks, 256, 0, st>>>(o, lse, rows, d);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (max_seqlen_q == 0) return ATTN_OK;
+  return d == 128 ? launch_fwd_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, Hkv, total_q, total_k,
+                                           max_seqlen_q, causal, scale, st)
+                  : launch_fwd_varlen<64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, Hkv, total_q, total_k,
+                                          max_seqlen_q, causal, scale, st);
+}
+
 int attn_fwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
              int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
   return attn_fwd_gqa(q, k, v, o, lse, B, H, H > 0 ? H : 1, Nq, Nkv, d, causal, scale, stream);
@@ -372,9 +450,9 @@ size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
   return decode_ws_bytes((long long)B * H, d, num_splits);
 }
 
-int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
-                    float* lse, int B, int H, int Hkv, int Nkv, int d, float scale, int num_splits,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+static int decode_impl(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                       float* lse, const int* seqlens, int B, int H, int Hkv, int Nkv, int d, float scale,
+                       int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 0 || H < 0 || Nkv < 1) return ATTN_ERR_INVALID_ARG;
   if (Hkv < 1 || (H > 0 && H % Hkv != 0) || Hkv > (H > 0 ? H : Hkv)) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
@@ -402,14 +480,14 @@ int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_
   if (G == 1) {
     if (d == 128)
       ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits, chunk,
-                                                                      sl2, grp);
+                                                                      sl2, grp, seqlens, H);
     else
       ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits, chunk,
-                                                                     sl2, grp);
+                                                                     sl2, grp, seqlens, H);
   } else {
 #define TA_DECODE_GROUP(DD, GG)                                                                           \
   ta::decode_split_group_kernel<DD, GG><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, \
-                                                                         num_splits, chunk, sl2, grp)
+                                                                         num_splits, chunk, sl2, grp, seqlens, H)
     if (d == 128) {
       if (G == 8) TA_DECODE_GROUP(128, 8); else if (G == 4) TA_DECODE_GROUP(128, 4); else TA_DECODE_GROUP(128, 2);
     } else {
@@ -422,6 +500,22 @@ int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_
   else
     ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode_gqa(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                    float* lse, int B, int H, int Hkv, int Nkv, int d, float scale, int num_splits,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k, v, o, lse, nullptr, B, H, Hkv, Nkv, d, scale, num_splits, workspace, workspace_bytes,
+                     stream);
+}
+
+int attn_decode_varlen(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o,
+                       float* lse, const int* seqlens_k, int B, int H, int Hkv, int Nkv_max, int d, float scale,
+                       int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B > 0 && H > 0 && !seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (seqlens_k && !aligned4(seqlens_k)) return ATTN_ERR_MISALIGNED;
+  return decode_impl(q, k, v, o, lse, seqlens_k, B, H, Hkv, Nkv_max, d, scale, num_splits, workspace,
+                     workspace_bytes, stream);
 }
 
 int attn_decode(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, attn_bf16_t* o, float* lse,
@@ -456,11 +550,11 @@ int attn_decode_noalloc(const attn_bf16_t* q, const attn_bf16_t* k, const attn_b
   const unsigned grid = (unsigned)(BH * num_splits);
   if (d == 128) {
     ta::decode_split_kernel<128><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                    chunk, sl2, 1);
+                                                                    chunk, sl2, 1, nullptr, H);
     ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
   } else {
     ta::decode_split_kernel<64><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, num_splits,
-                                                                   chunk, sl2, 1);
+                                                                   chunk, sl2, 1, nullptr, H);
     ta::decode_combine_kernel<64><<<(unsigned)BH, 64, 0, st>>>(o_part, l_part, o, lse, num_splits);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -46,7 +46,8 @@ template <int D>
 __global__ void __launch_bounds__(DEC_THREADS)
     decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                         const uint16_t* __restrict__ v, float* __restrict__ o_part,
-                        float* __restrict__ lse_part, int Nkv, int S, int chunk, float sl2, int group) {
+                        float* __restrict__ lse_part, int Nkv, int S, int chunk, float sl2, int group,
+                        const int* __restrict__ seqlens, int Hq) {
   constexpr int LPK = D / 8;          // lanes per key row (16 bytes each)
   constexpr int KPW = 32 / LPK;       // key rows per warp step
   constexpr int NW = DEC_THREADS / 32;
@@ -62,8 +63,11 @@ __global__ void __launch_bounds__(DEC_THREADS)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LPK;                    // which key of the warp step
   const int e0 = (lane % LPK) * 8;               // first channel of this lane
+  // per-batch cache length (seqlens != null): keys [0, len) of the Nkv rows
+  const int len = seqlens ? min(max(seqlens[bh / Hq], 0), Nkv) : Nkv;
+  if (seqlens) chunk = (len + S - 1) / S;
   const long long key0 = (long long)c * chunk;
-  const int nk = (int)max(0LL, min((long long)Nkv, key0 + chunk) - key0);
+  const int nk = (int)max(0LL, min((long long)len, key0 + chunk) - key0);
 
   float qv[8];
   {
@@ -195,7 +199,8 @@ template <int D, int G, int NT = DEC_THREADS, int UNR = dec_group_unroll(G)>
 __global__ void __launch_bounds__(NT)
     decode_split_group_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                               const uint16_t* __restrict__ v, float* __restrict__ o_part,
-                              float* __restrict__ lse_part, int Nkv, int S, int chunk, float sl2, int group) {
+                              float* __restrict__ lse_part, int Nkv, int S, int chunk, float sl2, int group,
+                              const int* __restrict__ seqlens, int Hq) {
   constexpr int LPK = D / 8;
   constexpr int KPW = 32 / LPK;
   constexpr int NW = NT / 32;
@@ -213,8 +218,10 @@ __global__ void __launch_bounds__(NT)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LPK;
   const int e0 = (lane % LPK) * 8;
+  const int len = seqlens ? min(max(seqlens[bh0 / Hq], 0), Nkv) : Nkv;  // per-batch cache length
+  if (seqlens) chunk = (len + S - 1) / S;
   const long long key0 = (long long)c * chunk;
-  const int nk = (int)max(0LL, min((long long)Nkv, key0 + chunk) - key0);
+  const int nk = (int)max(0LL, min((long long)len, key0 + chunk) - key0);
 
   float qv[G][8];
 #pragma unroll

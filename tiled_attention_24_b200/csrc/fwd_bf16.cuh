@@ -26,6 +26,17 @@
 //   P_t  : columns [128 t, 128 t + 64)    bf16x2 probabilities, aliasing S_t
 //   O_t  : columns [256 + D t, 256 + D t + D)   fp32 accumulator of tile t
 //
+// Variable-length batches (VARLEN = true; "FlashAttention 4" page, what is
+// missing: varlen): sequences packed token-major, Q/O [total_q][H][D],
+// K/V [total_k][H_kv][D], sequence b holding rows [cu_q[b], cu_q[b+1]) and
+// keys [cu_k[b], cu_k[b+1]); LSE [H][total_q].  The TMA maps view the packed
+// tensors as (D, heads, tokens) with boxes of 64 x 1 x 128, which land in
+// shared memory exactly like the dense (D, N, B*H) boxes of 64 x 128 x 1.
+// Rows of a tile past the sequence's end belong to the next sequence (or read
+// as zero past the tensor): their keys are masked like a ragged tail, their
+// query rows are not stored (the epilogue writes rows directly instead of a
+// TMA store, which would overwrite the next sequence).
+//
 // Shared memory (128-byte swizzled, the TMA and UMMA canonical layout): each
 // 128 x D bf16 tile is stored as D/64 column blocks of 128 rows x 128 bytes.
 // Q0, Q1, then a ring of NSTAGE stages; stage i holds V_{i-1} (first tile)
@@ -53,6 +64,11 @@ struct FwdParams {
   int causal;
   float sl2;  // scale * log2(e)
   unsigned long long timeout_ns;
+  // variable-length batches only
+  const int* cu_q;  // [nb + 1] row offsets of the sequences in the packed Q / O
+  const int* cu_k;  // [nb + 1] key offsets in the packed K / V
+  uint16_t* o;      // packed O [total_q][H][D]
+  int nb, H, total_q, total_k;
 };
 
 template <int D>
@@ -114,7 +130,7 @@ __device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, ui
   return wait_bar(bar, parity, &dummy, limit_ns);
 }
 
-template <int D>
+template <int D, bool VARLEN = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -132,13 +148,27 @@ __global__ void __launch_bounds__(384, 1)
   const int BH = gridDim.x / p.n_qp;
   const int bh = p.causal ? (int)(blockIdx.x % BH) : (int)(blockIdx.x / p.n_qp);
   const int qp = p.causal ? p.n_qp - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x % p.n_qp);
+  int Nq = p.Nq, Nkv = p.Nkv, Tc = p.Tc;
+  int qstart = 0, kstart = 0, head = bh;  // varlen: first row / key of the sequence, query head
+  if constexpr (VARLEN) {
+    const int b = bh / p.H;
+    head = bh % p.H;
+    // offsets clamped to the tensors, so that a bad offset array cannot
+    // move a store out of the packed O
+    qstart = min(max(p.cu_q[b], 0), p.total_q);
+    Nq = min(max(p.cu_q[b + 1], qstart), p.total_q) - qstart;
+    kstart = min(max(p.cu_k[b], 0), p.total_k);
+    Nkv = min(max(p.cu_k[b + 1], kstart), p.total_k) - kstart;
+    Tc = (Nkv + 127) / 128;
+    if (qp * 256 >= Nq) return;  // the whole CTA: nothing initialised yet
+  }
   int r0[2], n[2];
   bool present[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     r0[t] = qp * 256 + t * 128;
-    present[t] = r0[t] < p.Nq;
-    n[t] = fwd_tile_kv_count(r0[t], p.Nq, p.Nkv, p.Tc, p.causal);
+    present[t] = r0[t] < Nq;
+    n[t] = fwd_tile_kv_count(r0[t], Nq, Nkv, Tc, p.causal);
   }
   const int nmax = max(n[0], n[1]);
   volatile int* abort_flag = &bars->abort;
@@ -182,10 +212,14 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive_expect_tx(qbar, (present[0] + present[1]) * C::TILE);
       for (int t = 0; t < 2; ++t) {
         if (!present[t]) continue;
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
+        for (int h = 0; h < D / 64; ++h) {
+          if constexpr (VARLEN)
+            tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, head, qstart + r0[t]);
+          else
+            tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
+        }
       }
-      const int kvh = bh / p.group;  // key/value head of this query head
+      const int kvh = head / p.group;  // key/value head of this query head
       // stage i (0..nmax): V_{i-1} at +0 (none for i = 0), K_i at +TILE (none for i = nmax)
       int it = 0, slot = 0;
       uint32_t ph = 0;
@@ -197,8 +231,13 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(fb, ((i > 0) + (i < nmax)) * C::TILE);
         const uint32_t dst = sbase + C::SLOT_OFF + slot * C::STAGE;
         for (int h = 0; h < D / 64; ++h) {
-          if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, (i - 1) * 128, kvh);
-          if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, i * 128, kvh);
+          if constexpr (VARLEN) {
+            if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, kvh, kstart + (i - 1) * 128);
+            if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, kvh, kstart + i * 128);
+          } else {
+            if (i > 0) tma_load_3d(dst + h * C::HALF, &tmV, fb, h * 64, (i - 1) * 128, kvh);
+            if (i < nmax) tma_load_3d(dst + C::TILE + h * C::HALF, &tmK, fb, h * 64, i * 128, kvh);
+          }
         }
       }
       // Never leave a copy in flight: wait for the last load of every stage.
@@ -358,7 +397,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tbase + lane_off + C::T_O + t * D;
     const uint32_t tP = C::SEP_P ? tbase + lane_off + C::T_P + 64 * t : tS;
     const float sl2 = p.sl2;
-    const int off = p.Nkv - p.Nq;
+    const int off = Nkv - Nq;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = present[t];
     for (int j = 0; j < n[t] && ok; ++j) {
@@ -376,10 +415,10 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(smem_u32(&bars->s_free[t]));  // the MMA may now compute S_t(j+1) here
       }
       const int kb = j * 128;
-      const bool tail = kb + 128 > p.Nkv;
+      const bool tail = kb + 128 > Nkv;
       const bool diag = p.causal && (kb + 127 > r0[t] + off);
       if (tail || diag) {
-        int lim = p.Nkv - 1 - kb;                       // last visible column of this row
+        int lim = Nkv - 1 - kb;                         // last visible column of this row
         if (p.causal) lim = min(lim, row + off - kb);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -485,6 +524,32 @@ __global__ void __launch_bounds__(384, 1)
     if (present[t] && ok) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      if constexpr (VARLEN) {
+        // direct row stores (a tile may end inside the sequence)
+        uint16_t* orow = p.o + ((size_t)(qstart + row) * p.H + head) * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+          if (row < Nq) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float a = (l > 0.f) ? __uint_as_float(o[g * 8 + 2 * e]) * inv : 0.f;
+                const float b = (l > 0.f) ? __uint_as_float(o[g * 8 + 2 * e + 1]) * inv : 0.f;
+                w[e] = pack_bf16(a, b);
+              }
+              *reinterpret_cast<uint4*>(orow + cc * 32 + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        if (row < Nq)
+          p.lse[(size_t)head * p.total_q + qstart + row] =
+              (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      } else {
       uint8_t* stage = smem + C::Q_OFF + t * C::TILE;  // Q_t is no longer read
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -506,8 +571,8 @@ __global__ void __launch_bounds__(384, 1)
           *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      if (row < p.Nq)
-        p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (row < Nq)
+        p.lse[(size_t)bh * Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&bars->epi[t]));
       if (warp == 4 + 4 * t && lane == 0) {
@@ -519,6 +584,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
+      }
     }
   }
 

@@ -29,7 +29,7 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "normal_bf16", "make_qkv", "outlier_channels", "rotation_signs"]
+__all__ = ["Workload", "WORKLOADS", "normal_bf16", "make_qkv", "outlier_channels", "rotation_signs", "make_varlen"]
 
 
 @dataclass(frozen=True)
@@ -143,3 +143,19 @@ def rotation_signs(d: int, seed: int = 0) -> torch.Tensor:
     g = torch.Generator()
     g.manual_seed(seed + 7_000_003)
     return (torch.randint(0, 2, (d,), generator=g, dtype=torch.int64) * 2 - 1).to(torch.float32)
+
+
+def make_varlen(lens_q, lens_k, H: int, Hkv: int, d: int, seed: int = 0, input_scale: float = 1.0):
+    """A variable-length batch packed without padding: q [sum(lens_q)][H][d],
+    k, v [sum(lens_k)][Hkv][d] (bf16, drawn like ``normal_bf16``, in that
+    order) and the int32 offset arrays cu_q, cu_k ([B + 1], starting at 0).
+    Returns (q, k, v, cu_q, cu_k) on the CPU."""
+    gen = torch.Generator()
+    gen.manual_seed(seed + 9_000_011)
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    q = normal_bf16((tq, H, d), gen, "cpu", input_scale)
+    k = normal_bf16((tk, Hkv, d), gen, "cpu", input_scale)
+    v = normal_bf16((tk, Hkv, d), gen, "cpu", input_scale)
+    cu_q = torch.tensor([0] + list(torch.cumsum(torch.tensor(lens_q), 0).tolist()), dtype=torch.int32)
+    cu_k = torch.tensor([0] + list(torch.cumsum(torch.tensor(lens_k), 0).tolist()), dtype=torch.int32)
+    return q, k, v, cu_q, cu_k
