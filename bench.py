@@ -6,7 +6,9 @@ A step is one pass of the hot path over the seeded synthetic workloads:
   * prefill  B=4 H=16 N=4096 d=128 bf16: attn_fwd non-causal + attn_fwd causal
              (the headline: attention forward TFLOP/s, 4*B*H*N*N*d, halved
              for causal); and attn_bwd on the same shapes (reported as a part,
-             2.5 x the forward's FLOPs, not in the headline);
+             2.5 x the forward's FLOPs, not in the headline), the FP8-P
+             backward (causal), and the same token count as a packed
+             variable-length batch of 6 sequences (causal forward);
   * decode   B=64 H=32 one query, N_kv=8192 d=128, 16 splits + combine; and
              the same with grouped-query attention (8 cache heads, 4 query
              heads each: 2.1 GB of cache);
@@ -48,7 +50,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, make_qkv, rotation_signs  # noqa: E402
+from workloads import WORKLOADS, make_qkv, make_varlen, rotation_signs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -254,6 +256,19 @@ def run_ours(args):
             2.5 * wp.flops(False), "TFLOP/s", peak_tc, "tensor", 3)
         seg("prefill_bwd_causal", lambda: ta.attn_bwd(q, k, v, bo, dout, blse, dq, dk, dv, True, wp.scale, bws, stream),
             2.5 * wp.flops(True), "TFLOP/s", peak_tc, "tensor", 3)
+        # FP8-P backward (P rounded to e4m3 for dV), causal
+        seg("prefill_bwd_fp8p_causal",
+            lambda: ta.attn_bwd_fp8p(q, k, v, bo, dout, blse, dq, dk, dv, True, wp.scale, bws, stream),
+            2.5 * wp.flops(True), "TFLOP/s", peak_tc, "tensor", 3)
+        # the same tokens as a packed variable-length batch (causal, per sequence)
+        vl = [4096, 2048, 1024, 3000, 5000, 1216]
+        vq, vk, vv, vcu, _ = make_varlen(vl, vl, wp.H, wp.H, wp.d, seed=0)
+        vq, vk, vv, vcu = vq.to(dev), vk.to(dev), vv.to(dev), vcu.to(dev)
+        vo = torch.empty_like(vq)
+        vlse = torch.empty((wp.H, vq.shape[0]), dtype=torch.float32, device=dev)
+        seg("prefill_varlen_causal",
+            lambda: ta.attn_fwd_varlen(vq, vk, vv, vo, vlse, vcu, vcu, max(vl), True, wp.scale, stream),
+            sum(2.0 * wp.H * n * n * wp.d for n in vl), "TFLOP/s", peak_tc, "tensor", 1)
     wd = WORKLOADS["decode"]
     if "decode" in parts:
         dq, dk, dv = make_qkv(wd, seed=0, device=dev, B=args.decode_batch or wd.B)

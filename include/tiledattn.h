@@ -128,6 +128,19 @@ ATTN_API int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf1
                       size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd_fp8p -- attn_bwd with the recomputed probabilities in 8-bit
+ * floating point for the dV product ([FP4-FA4]: in training, 4-bit P made the
+ * backward diverge, 8-bit P kept it stable): P = exp(S - LSE) is rounded to
+ * e4m3 (round to nearest even, unit scale; P <= 1) before dV = P^T dO.
+ * dS = P o (dP - Dr) uses P unrounded, so dQ and dK equal attn_bwd's.  Same
+ * arguments, layouts and workspace as attn_bwd.
+ */
+ATTN_API int attn_bwd_fp8p(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+                           const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk,
+                           attn_bf16_t* dv, int B, int H, int Nq, int Nkv, int d, int causal, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode -- split-KV decode: ONE query row per (batch, head) against a
  * KV cache of Nkv keys; the key range is cut into num_splits equal chunks of
  * ceil(Nkv / num_splits) keys, each chunk gives a partial (O_c, LSE_c) in the

@@ -87,7 +87,8 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None,
     return O, LSE
 
 
-def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = None):
+def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = None, p_round=None,
+                       flip_band=None):
     """Gradients of O = softmax(scale * Q K^T, masked) V with respect to Q, K
     and V for an upstream gradient dO, in float64 -- the calculus of the
     definition, with P materialised (the quantity [FA-trading] "Backward:
@@ -98,7 +99,15 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
         dQ = scale dS K,  dK = scale dS^T Q.
 
     sum_k P_ik dP_ik equals sum_c dO_ic O_ic (O = P V).  Rows that see no key
-    have P = 0 and contribute nothing.  Returns (dQ, dK, dV) float64."""
+    have P = 0 and contribute nothing.  Returns (dQ, dK, dV) float64.
+
+    ``p_round`` (a function on arrays) rounds P where it is the operand of
+    dV = round(P)^T dO only (the FP8-P backward of [FP4-FA4]: 8-bit
+    probabilities in the backward); dS keeps P unrounded.  With ``flip_band``
+    = (midpoints, step, rel) it also returns, per dV element, a bound on what
+    P elements within ``rel`` (relative) of a rounding midpoint change if
+    they round to the other neighbour (``step(P)`` = that neighbour's
+    distance): sum_i flip_ij |dO_ic|."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
@@ -107,6 +116,7 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
+    fb = np.zeros_like(v)
     vis = visible_mask(Nq, Nkv, causal)
     for b in range(B):
         for h in range(H):
@@ -118,9 +128,18 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
             P = np.where(alive[:, None], P, 0.0)
             dP = do[b, h] @ v[b, h].T
             dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
-            dv[b, h] = P.T @ do[b, h]
+            Pv = P if p_round is None else p_round(P)
+            dv[b, h] = Pv.T @ do[b, h]
             dq[b, h] = scale * (dS @ k[b, h])
             dk[b, h] = scale * (dS.T @ q[b, h])
+            if flip_band is not None:
+                mids, step, rel = flip_band
+                near = np.zeros(P.shape, dtype=bool)
+                for t in mids:
+                    near |= np.abs(P - t) <= rel * t
+                fb[b, h] = np.where(near & (P > 0), step(P), 0.0).T @ np.abs(do[b, h])
+    if flip_band is not None:
+        return dq, dk, dv, fb
     return dq, dk, dv
 
 

@@ -70,3 +70,37 @@ def test_backward_prefill_workload_sampled_heads(cuda_lib, causal):
         sl = (slice(b, b + 1), slice(h, h + 1))
         ref = A.attention_backward(q[sl], k[sl], v[sl], do[sl], causal, w.scale)
         _check([g[sl] for g in got], ref, f"prefill b={b} h={h} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 2, 128, 128, 64), (1, 1, 300, 333, 128), (1, 1, 640, 200, 128),
+                                   (1, 2, 384, 384, 128)], ids=lambda s: "x".join(map(str, s)))
+def test_backward_fp8_p(cuda_lib, shape, causal):
+    """FP8-P backward: dQ, dK as the bf16 backward; dV against the oracle with
+    P rounded to e4m3, plus the bound on P elements that sat within fp32
+    evaluation error of an e4m3 midpoint.  O and LSE are the oracle's
+    (rounded to bf16 / fp32), so the device recomputes P from the same
+    statistics."""
+    from oracle import fp8 as F
+    B, H, Nq, Nkv, d = shape
+    q, k, v = make_qkv("prefill", seed=51, B=B, H=H, Nq=Nq, Nkv=Nkv, d=d)
+    do = make_qkv("prefill", seed=52, B=B, H=H, Nq=Nq, Nkv=1, d=d)[0]
+    scale = d ** -0.5
+    O, L = A.attention(q, k, v, causal, scale)
+    o = torch.from_numpy(O).to(torch.bfloat16).cuda()
+    lse = torch.from_numpy(L).to(torch.float32).cuda()
+    dq, dk, dv = cuda_lib.backward(q.cuda(), k.cuda(), v.cuda(), o, lse, do.cuda(), causal, scale, p_fp8=True)
+    assert cuda_lib.attn_check_status() == 0
+    got = [t.double().cpu().numpy() for t in (dq, dk, dv)]
+    vals = F.UE4M3_VALUES
+    mids = ((vals[:-1] + vals[1:]) / 2)[vals[1:] <= 1.0]
+    rq, rk, rv, fb = A.attention_backward(q, k, v, do, causal, scale, p_round=F.e4m3_encode_value,
+                                          flip_band=(mids, lambda p: np.maximum(p * 0.125, 2.0 ** -9), 2e-5))
+    _check(got[:2], (rq, rk), f"fp8p {shape} causal={causal}")
+    err = np.abs(got[2] - rv)
+    big = float(np.abs(rv).max())
+    print(f"fp8p {shape} causal={causal} dv: max err {err.max():.3e} (ref max {big:.3e}), flip bound max {fb.max():.3e}")
+    assert (err <= 2.0 ** -7 * big + 1e-6 + fb).all()
+    # the 8-bit P moves dV away from the exact gradient by far more than the bf16 path does
+    _, _, dv_exact = A.attention_backward(q, k, v, do, causal, scale)
+    assert np.abs(rv - dv_exact).max() > 0

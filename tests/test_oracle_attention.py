@@ -348,3 +348,26 @@ def test_decode_varlen_matches_masked_sdpa():
         np.testing.assert_allclose(O[b], ref[0].numpy(), rtol=0, atol=1e-12)
         s = (q[b] @ kh[b].transpose(-1, -2) * 0.5)[..., : lens[b]]
         np.testing.assert_allclose(L[b], torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_fp8_p_closed_form():
+    """Keys with identical scores give P = 1/n on every visible key.  For
+    n = 2, 4 the value is an e4m3 value and rounding changes nothing; for
+    n = 3, e4m3(1/3) = 0.34375 (the nearer of 0.3125 and 0.34375), so
+    dV_j = 0.34375 * sum of dO over the rows that see key j, while dQ and
+    dK are those of the unrounded backward."""
+    from oracle import fp8 as F
+    g = np.random.default_rng(21)
+    d = 4
+    for n, p8 in ((2, 0.5), (4, 0.25), (3, 0.34375)):
+        q = g.standard_normal((1, 1, 5, d))
+        k = np.tile(g.standard_normal(d), (n, 1))[None, None]      # identical keys
+        v = g.standard_normal((1, 1, n, d))
+        do = g.standard_normal((1, 1, 5, d))
+        dq0, dk0, dv0 = A.attention_backward(q, k, v, do, False, 0.7)
+        dq8, dk8, dv8 = A.attention_backward(q, k, v, do, False, 0.7, p_round=F.e4m3_encode_value)
+        np.testing.assert_allclose(dv8[0, 0], np.tile(p8 * do[0, 0].sum(axis=0), (n, 1)), rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(dq8, dq0)
+        np.testing.assert_array_equal(dk8, dk0)
+        if n != 3:
+            np.testing.assert_allclose(dv8, dv0, rtol=0, atol=1e-12)

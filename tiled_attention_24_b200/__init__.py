@@ -12,7 +12,7 @@ import torch
 
 from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
                        attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
-                       attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_fwd_varlen, attn_decode_varlen, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_workspace_bytes,
+                       attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_fwd_varlen, attn_decode_varlen, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_fp8p, attn_bwd_workspace_bytes,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
                        attn_nvfp4_sf_bytes, attn_quantize_int8, attn_quantize_nvfp4, attn_set_wait_limit_ns,
                        attn_status_string, attn_version, attn_watchdog_selftest, load)
@@ -23,7 +23,7 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "attn_quantize_int8", "attn_fwd_int8", "attn_int8_scores", "attn_decode_noalloc",
            "attn_quantize_nvfp4", "attn_fwd_fp4", "attn_fp4_scores", "quantize_nvfp4", "forward_fp4",
            "attn_fwd_gqa", "attn_decode_gqa", "attn_quantize_int4", "quantize_int4", "forward_int4",
-           "attn_bwd", "attn_bwd_workspace_bytes", "backward",
+           "attn_bwd", "attn_bwd_fp8p", "attn_bwd_workspace_bytes", "backward",
            "attn_quantize_fp8", "attn_fwd_fp8", "quantize_fp8", "forward_fp8", "hadamard_signs",
            "attn_fwd_varlen", "attn_decode_varlen", "forward_varlen", "decode_varlen",
            "DIRECT_P", "QUANT_AFTER_EXP"]
@@ -46,14 +46,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
     return o, lse
 
 
-def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, stream=None):
+def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, stream=None,
+             p_fp8: bool = False):
     """Allocate dq, dk, dv (bf16) and the row-statistic workspace, run ``attn_bwd``
-    (o, lse: the forward's outputs for the same arguments)."""
+    (``attn_bwd_fp8p`` with ``p_fp8``: P in e4m3 for dV) (o, lse: the
+    forward's outputs for the same arguments)."""
     B, H, Nq, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(16, attn_bwd_workspace_bytes(B, H, Nq)), dtype=torch.uint8, device=q.device)
-    attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, ws, stream)
+    (attn_bwd_fp8p if p_fp8 else attn_bwd)(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, ws, stream)
     return dq, dk, dv
 
 

@@ -33,6 +33,7 @@ SIGNATURES = [
     ("attn_fwd_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_bwd_workspace_bytes", _SZ, [_I, _I, _I]),
     ("attn_bwd", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
+    ("attn_bwd_fp8p", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     ("attn_decode_gqa", _I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     ("attn_fwd_varlen", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
     ("attn_decode_varlen", _I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
@@ -145,6 +146,17 @@ def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, work
                          B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream))
     _check("attn_bwd", rc)
+
+
+def attn_bwd_fp8p(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None):
+    """attn_bwd with P rounded to e4m3 before dV = P^T dO (the FP8-P backward)."""
+    _need_cuda(q, k, v, o, dout, lse, dq, dk, dv, workspace)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    rc = load().attn_bwd_fp8p(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                              _ptr(dv), B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_bwd_fp8p", rc)
 
 
 def attn_decode_workspace_bytes(B: int, H: int, d: int, num_splits: int) -> int:

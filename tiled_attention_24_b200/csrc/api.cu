@@ -248,7 +248,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool P8>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                void* dq, void* dk, void* dv, float* rowdot, int B, int H, int Nq, int Nkv, int causal, float scale,
                cudaStream_t st) {
@@ -260,7 +260,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if ((rc = make_tmap_bf16(&tk, k, D, Nkv, BH)) != ATTN_OK) return rc;
   if ((rc = make_tmap_bf16(&tv, v, D, Nkv, BH)) != ATTN_OK) return rc;
   if ((rc = make_tmap_bf16(&tdo, dout, D, Nq, BH)) != ATTN_OK) return rc;
-  if ((rc = set_smem_attr(ta::bwd_dkdv_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
+  if ((rc = set_smem_attr(ta::bwd_dkdv_kernel<D, P8>, C::SMEM)) != ATTN_OK) return rc;
   if ((rc = set_smem_attr(ta::bwd_dq_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
   ta::BwdParams p;
   p.o = static_cast<const uint16_t*>(o);
@@ -282,7 +282,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const long long gk = (long long)BH * p.nkt, gq = (long long)BH * p.nqt;
   if ((rows + 7) / 8 > 0x7fffffffLL || gk > 0x7fffffffLL || gq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   ta::bwd_rowdot_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.o, p.dout, rowdot, rows);
-  ta::bwd_dkdv_kernel<D><<<(unsigned)gk, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tdo, p);
+  ta::bwd_dkdv_kernel<D, P8><<<(unsigned)gk, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tdo, p);
   ta::bwd_dq_kernel<D><<<(unsigned)gq, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -414,10 +414,10 @@ size_t attn_bwd_workspace_bytes(int B, int H, int Nq) {
   return ((size_t)B * H * Nq * sizeof(float) + 255) & ~size_t(255);
 }
 
-int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
-             const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv, int B,
-             int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
-             void* stream) {
+static int bwd_impl(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+                    const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv,
+                    int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream, bool p8) {
   if (B < 0 || H < 0 || Nq < 0 || Nkv < 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -441,8 +441,27 @@ int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, c
     return ATTN_ERR_MISALIGNED;
   if (workspace_bytes < attn_bwd_workspace_bytes(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
   float* rowdot = static_cast<float*>(workspace);
-  return d == 128 ? launch_bwd<128>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st)
-                  : launch_bwd<64>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st);
+  if (p8)
+    return d == 128 ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st)
+                    : launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st);
+  return d == 128 ? launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st)
+                  : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, rowdot, B, H, Nq, Nkv, causal, scale, st);
+}
+
+int attn_bwd(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+             const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv, int B,
+             int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+             void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nkv, d, causal, scale, workspace, workspace_bytes,
+                  stream, false);
+}
+
+int attn_bwd_fp8p(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf16_t* v, const attn_bf16_t* o,
+                  const attn_bf16_t* dout, const float* lse, attn_bf16_t* dq, attn_bf16_t* dk, attn_bf16_t* dv,
+                  int B, int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nkv, d, causal, scale, workspace, workspace_bytes,
+                  stream, true);
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {

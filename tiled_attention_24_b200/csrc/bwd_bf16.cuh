@@ -19,6 +19,11 @@
 //   bwd_dq_kernel      one CTA per (batch*head, 128-query tile): walks the key
 //                      tiles, S = Q K^T and dP = dO V^T, dS in TMEM, and
 //                      dQ += dS K.
+// FP8-P variant (P8 = true; "Hardware-Aware FP4 FlashAttention-4" page: in
+// training, 4-bit probabilities made the backward diverge and 8-bit ones kept
+// it stable): the recomputed P is rounded to e4m3 (unit scale, P <= 1) before
+// it enters dV = P^T dO; dS uses P unrounded.  e4m3 values are exact in bf16,
+// so the bf16 MMA computes exactly the product with the 8-bit P.
 // Each kernel: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 2-5
 // compute (thread = TMEM lane).  The score pair of a tile is computed, turned
 // into P / dS, then the accumulating MMAs run; the next tile's scores are
@@ -141,7 +146,22 @@ __device__ __forceinline__ void bwd_store_row(uint32_t tacc, uint16_t* dst, floa
   }
 }
 
-// P = exp2(S * sl2 - lse2) and dS = P (dP - Dr) for 32 columns, packed bf16x2.
+// a pair of non-negative floats rounded to e4m3 (RNE, saturating), as bf16x2
+__device__ __forceinline__ uint32_t e4m3_round_bf16x2(float lo, float hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 c;\n\tcvt.rn.satfinite.e4m3x2.f32 c, %1, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
+      : "=r"(h2)
+      : "f"(hi), "f"(lo));
+  float a, b;
+  asm("{\n\t.reg .b16 x, y;\n\tmov.b32 {x, y}, %2;\n\tcvt.f32.f16 %0, x;\n\tcvt.f32.f16 %1, y;\n\t}"
+      : "=f"(a), "=f"(b)
+      : "r"(h2));
+  return pack_bf16(a, b);  // exact: every e4m3 value is a bf16 value
+}
+
+// P = exp2(S * sl2 - lse2) and dS = P (dP - Dr) for 32 columns, packed bf16x2
+// (P8: the P words hold e4m3-rounded P).
+template <bool P8 = false>
 __device__ __forceinline__ void bwd_p_ds(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float* lse2,
                                          const float* rd, float sl2, uint32_t vis_mask, uint32_t (&pp)[16],
                                          uint32_t (&pd)[16]) {
@@ -153,7 +173,10 @@ __device__ __forceinline__ void bwd_p_ds(const uint32_t (&s)[32], const uint32_t
     p1 = ((vis_mask >> (i + 1)) & 1u) ? p1 : 0.f;
     const float d0 = p0 * (__uint_as_float(dp[i]) - rd[i]);
     const float d1 = p1 * (__uint_as_float(dp[i + 1]) - rd[i + 1]);
-    pp[i / 2] = pack_bf16(p0, p1);
+    if constexpr (P8)
+      pp[i / 2] = e4m3_round_bf16x2(p0, p1);
+    else
+      pp[i / 2] = pack_bf16(p0, p1);
     pd[i / 2] = pack_bf16(d0, d1);
   }
 }
@@ -169,7 +192,7 @@ __device__ __forceinline__ uint32_t bwd_mask32(int lo, int hi) {  // bits [lo, h
 }
 
 // ============================================================== dK, dV
-template <int D>
+template <int D, bool P8 = false>
 __global__ void __launch_bounds__(192, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -320,7 +343,7 @@ __global__ void __launch_bounds__(192, 1)
         if (p.causal) lo = key - off - (q0 + c * 32);
         const uint32_t vis = bwd_mask32(lo, hi);
         uint32_t pp[16], pd[16];
-        bwd_p_ds(s, dp, cols + c * 32, cols + 128 + c * 32, p.sl2, vis, pp, pd);
+        bwd_p_ds<P8>(s, dp, cols + c * 32, cols + 128 + c * 32, p.sl2, vis, pp, pd);
         // P^T and dS^T over columns already read (16 words land in the first
         // half of the 32 columns this chunk index has passed)
         tmem_st16(tbase + lane_off + T_S + c * 16, pp);
