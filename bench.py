@@ -448,7 +448,7 @@ def run_ours(args):
     for part, key in (("decode", "decode_split"), ("longseq_noncausal", "fwd_bf16_longseq_noncausal"),
                       ("prefill_causal", "fwd_bf16_prefill_causal"), ("lowp_int8", "fwd_int8_lowp"),
                       ("lowp_fp4_direct_p", "fwd_fp4_direct_p_lowp"),
-                      ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp")):
+                      ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp"), ("lowp_fp8", "fwd_fp8_lowp")):
         if part in out_parts:
             out_parts[part]["traffic"] = traffic.get(key)
     for nm in ("lowp_int8", "lowp_fp4_direct_p", "lowp_fp4_quant_after_exp", "lowp_fp8"):
