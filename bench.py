@@ -249,21 +249,22 @@ def run_ours(args):
         bo_n, blse_n = torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
         ta.attn_fwd(q, k, v, bo_n, blse_n, False, wp.scale, stream)
         dout = make_qkv(wp, seed=1, device=dev, Nkv=1)[0]
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        # (names distinct from every later block's: the lambdas look them up when they run)
+        bdq, bdk, bdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         bws = torch.empty(ta.attn_bwd_workspace_bytes(wp.B, wp.H, wp.Nq), dtype=torch.uint8, device=dev)
         seg("prefill_bwd_noncausal",
-            lambda: ta.attn_bwd(q, k, v, bo_n, dout, blse_n, dq, dk, dv, False, wp.scale, bws, stream),
+            lambda: ta.attn_bwd(q, k, v, bo_n, dout, blse_n, bdq, bdk, bdv, False, wp.scale, bws, stream),
             2.5 * wp.flops(False), "TFLOP/s", peak_tc, "tensor", 3)
-        seg("prefill_bwd_causal", lambda: ta.attn_bwd(q, k, v, bo, dout, blse, dq, dk, dv, True, wp.scale, bws, stream),
+        seg("prefill_bwd_causal",
+            lambda: ta.attn_bwd(q, k, v, bo, dout, blse, bdq, bdk, bdv, True, wp.scale, bws, stream),
             2.5 * wp.flops(True), "TFLOP/s", peak_tc, "tensor", 3)
         # FP8-P backward (P rounded to e4m3 for dV), causal
         seg("prefill_bwd_fp8p_causal",
-            lambda: ta.attn_bwd_fp8p(q, k, v, bo, dout, blse, dq, dk, dv, True, wp.scale, bws, stream),
+            lambda: ta.attn_bwd_fp8p(q, k, v, bo, dout, blse, bdq, bdk, bdv, True, wp.scale, bws, stream),
             2.5 * wp.flops(True), "TFLOP/s", peak_tc, "tensor", 3)
         # the same tokens as a packed variable-length batch (causal, per sequence)
         vl = [4096, 2048, 1024, 3000, 5000, 1216]
-        vq, vk, vv, vcu, _ = make_varlen(vl, vl, wp.H, wp.H, wp.d, seed=0)
-        vq, vk, vv, vcu = vq.to(dev), vk.to(dev), vv.to(dev), vcu.to(dev)
+        vq, vk, vv, vcu = (t.to(dev) for t in make_varlen(vl, vl, wp.H, wp.H, wp.d, seed=0)[:4])
         vo = torch.empty_like(vq)
         vlse = torch.empty((wp.H, vq.shape[0]), dtype=torch.float32, device=dev)
         seg("prefill_varlen_causal",

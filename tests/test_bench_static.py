@@ -1,0 +1,61 @@
+"""Host-side guards that need no GPU.
+
+* bench.py builds its timed step from lambdas that look their tensors up when
+  they run; a name such a lambda reads must not be rebound later in the same
+  function (a later block reusing it would hand the kernel another tensor).
+* the binding rejects buffers whose shape or dtype does not match the call
+  before anything reaches the C ABI.
+"""
+import ast
+import os
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _assigned_names(fn):
+    counts = {}
+    for node in ast.walk(fn):
+        targets = []
+        if isinstance(node, ast.Assign):
+            targets = node.targets
+        elif isinstance(node, (ast.AugAssign, ast.AnnAssign)):
+            targets = [node.target]
+        elif isinstance(node, (ast.For, ast.comprehension)):
+            targets = [node.target]
+        for t in targets:
+            for n in ast.walk(t):
+                if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Store):
+                    counts[n.id] = counts.get(n.id, 0) + 1
+    return counts
+
+
+def _lambda_free_names(lam):
+    params = {a.arg for a in lam.args.args + lam.args.kwonlyargs}
+    return {n.id for n in ast.walk(lam.body) if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load)} - params
+
+
+def test_bench_step_lambdas_read_names_bound_once():
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    fn = next(n for n in ast.walk(tree) if isinstance(n, ast.FunctionDef) and n.name == "run_ours")
+    counts = _assigned_names(fn)
+    bad = set()
+    for lam in (n for n in ast.walk(fn) if isinstance(n, ast.Lambda)):
+        for name in _lambda_free_names(lam):
+            if counts.get(name, 0) > 1:
+                bad.add(name)
+    assert not bad, f"names read by step lambdas and assigned more than once: {sorted(bad)}"
+
+
+def test_binding_rejects_mis_shaped_buffers():
+    from tiled_attention_24_b200 import _binding as b
+    ok = torch.empty(2, 3, 4, dtype=torch.bfloat16)
+    b._expect((ok, (2, 3, 4), torch.bfloat16, "x"))
+    with pytest.raises(ValueError):
+        b._expect((ok, (2, 3, 5), torch.bfloat16, "x"))
+    with pytest.raises(ValueError):
+        b._expect((ok, (2, 3, 4), torch.float32, "x"))
+    with pytest.raises(ValueError):
+        b._at_least(torch.empty(10, dtype=torch.uint8), 11, "codes")

@@ -102,11 +102,30 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+_BF16, _F32, _I8, _U8, _I32 = torch.bfloat16, torch.float32, torch.int8, torch.uint8, torch.int32
+
+
+def _expect(*specs):
+    """(tensor, shape, dtype, name) tuples: every buffer must have exactly the
+    shape and dtype the call implies, so that no kernel writes or reads past a
+    caller's tensor (the C ABI sees only pointers and the sizes passed here)."""
+    for t, shape, dtype, name in specs:
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            raise ValueError(f"{name}: expected {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+
+
+def _at_least(t, nbytes: int, name: str):
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name}: needs {nbytes} bytes, got {t.numel() * t.element_size()}")
+
+
 def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
     """bf16 forward: q [B,H,Nq,d], k/v [B,H,Nkv,d] -> o (bf16), lse (fp32)."""
     _need_cuda(q, k, v, o, lse)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, Nq, d), _BF16, "q"), (k, (B, H, Nkv, d), _BF16, "k"), (v, (B, H, Nkv, d), _BF16, "v"),
+            (o, (B, H, Nq, d), _BF16, "o"), (lse, (B, H, Nq), _F32, "lse"))
     rc = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nkv, d, int(bool(causal)),
                          float(scale), _stream(stream))
     _check("attn_fwd", rc)
@@ -117,6 +136,8 @@ def attn_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float, stream=None):
     _need_cuda(q, k, v, o, lse)
     B, Hq, Nq, d = q.shape
     Hkv, Nkv = k.shape[1], k.shape[2]
+    _expect((q, (B, Hq, Nq, d), _BF16, "q"), (k, (B, Hkv, Nkv, d), _BF16, "k"), (v, (B, Hkv, Nkv, d), _BF16, "v"),
+            (o, (B, Hq, Nq, d), _BF16, "o"), (lse, (B, Hq, Nq), _F32, "lse"))
     rc = load().attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nkv, d,
                              int(bool(causal)), float(scale), _stream(stream))
     _check("attn_fwd_gqa", rc)
@@ -127,6 +148,8 @@ def attn_decode_gqa(q, k, v, o, lse, scale: float, num_splits: int, workspace, s
     _need_cuda(q, k, v, o, lse, workspace)
     B, Hq, _, d = q.shape
     Hkv, Nkv = k.shape[1], k.shape[2]
+    _expect((q, (B, Hq, 1, d), _BF16, "q"), (k, (B, Hkv, Nkv, d), _BF16, "k"), (v, (B, Hkv, Nkv, d), _BF16, "v"),
+            (o, (B, Hq, 1, d), _BF16, "o"), (lse, (B, Hq, 1), _F32, "lse"))
     rc = load().attn_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nkv, d, float(scale),
                                 int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream))
@@ -142,6 +165,9 @@ def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, work
     _need_cuda(q, k, v, o, dout, lse, dq, dk, dv, workspace)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, Nq, d), _BF16, "q"), (k, (B, H, Nkv, d), _BF16, "k"), (v, (B, H, Nkv, d), _BF16, "v"),
+            (o, (B, H, Nq, d), _BF16, "o"), (dout, (B, H, Nq, d), _BF16, "dout"), (lse, (B, H, Nq), _F32, "lse"),
+            (dq, (B, H, Nq, d), _BF16, "dq"), (dk, (B, H, Nkv, d), _BF16, "dk"), (dv, (B, H, Nkv, d), _BF16, "dv"))
     rc = load().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream))
@@ -153,6 +179,9 @@ def attn_bwd_fp8p(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float,
     _need_cuda(q, k, v, o, dout, lse, dq, dk, dv, workspace)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, Nq, d), _BF16, "q"), (k, (B, H, Nkv, d), _BF16, "k"), (v, (B, H, Nkv, d), _BF16, "v"),
+            (o, (B, H, Nq, d), _BF16, "o"), (dout, (B, H, Nq, d), _BF16, "dout"), (lse, (B, H, Nq), _F32, "lse"),
+            (dq, (B, H, Nq, d), _BF16, "dq"), (dk, (B, H, Nkv, d), _BF16, "dk"), (dv, (B, H, Nkv, d), _BF16, "dv"))
     rc = load().attn_bwd_fp8p(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                               _ptr(dv), B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
@@ -168,6 +197,8 @@ def attn_decode(q, k, v, o, lse, scale: float, num_splits: int, workspace, strea
     _need_cuda(q, k, v, o, lse, workspace)
     B, H, _, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, 1, d), _BF16, "q"), (k, (B, H, Nkv, d), _BF16, "k"), (v, (B, H, Nkv, d), _BF16, "v"),
+            (o, (B, H, 1, d), _BF16, "o"), (lse, (B, H, 1), _F32, "lse"))
     rc = load().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
                             int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream))
@@ -180,6 +211,8 @@ def attn_decode_noalloc(q, k, v, o, lse, scale: float, num_splits: int, stream=N
     _need_cuda(q, k, v, o, lse)
     B, H, _, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, 1, d), _BF16, "q"), (k, (B, H, Nkv, d), _BF16, "k"), (v, (B, H, Nkv, d), _BF16, "v"),
+            (o, (B, H, 1, d), _BF16, "o"), (lse, (B, H, 1), _F32, "lse"))
     rc = load().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nkv, d, float(scale),
                                     int(num_splits), _stream(stream))
     _check("attn_decode_noalloc", rc)
@@ -192,6 +225,9 @@ def attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, max_seqlen_q: int, causal: bool
     total_q, H, d = q.shape
     total_k, Hkv, _ = k.shape
     B = cu_q.shape[0] - 1
+    _expect((q, (total_q, H, d), _BF16, "q"), (k, (total_k, Hkv, d), _BF16, "k"), (v, (total_k, Hkv, d), _BF16, "v"),
+            (o, (total_q, H, d), _BF16, "o"), (lse, (H, total_q), _F32, "lse"), (cu_q, (B + 1,), _I32, "cu_q"),
+            (cu_k, (B + 1,), _I32, "cu_k"))
     rc = load().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q), _ptr(cu_k), B, H, Hkv,
                                 total_q, total_k, int(max_seqlen_q), d, int(bool(causal)), float(scale),
                                 _stream(stream))
@@ -204,6 +240,8 @@ def attn_decode_varlen(q, k, v, o, lse, seqlens_k, scale: float, num_splits: int
     _need_cuda(q, k, v, o, lse, seqlens_k, workspace)
     B, H, _, d = q.shape
     Hkv, Nkv = k.shape[1], k.shape[2]
+    _expect((q, (B, H, 1, d), _BF16, "q"), (k, (B, Hkv, Nkv, d), _BF16, "k"), (v, (B, Hkv, Nkv, d), _BF16, "v"),
+            (o, (B, H, 1, d), _BF16, "o"), (lse, (B, H, 1), _F32, "lse"), (seqlens_k, (B,), _I32, "seqlens_k"))
     rc = load().attn_decode_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, Hkv, Nkv,
                                    d, float(scale), int(num_splits), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
@@ -214,6 +252,8 @@ def attn_quantize_int8(x, xq, xs, per_head: bool, stream=None):
     """bf16 [B,H,N,d] -> int8 xq, fp32 xs ([B,H,N] per token or [B,H] per head)."""
     _need_cuda(x, xq, xs)
     B, H, N, d = x.shape
+    _expect((x, (B, H, N, d), _BF16, "x"), (xq, (B, H, N, d), _I8, "xq"),
+            (xs, (B, H) if per_head else (B, H, N), _F32, "xs"))
     _check("attn_quantize_int8", load().attn_quantize_int8(_ptr(x), _ptr(xq), _ptr(xs), B, H, N, d,
                                                              int(bool(per_head)), _stream(stream)))
 
@@ -222,6 +262,7 @@ def attn_quantize_int4(x, xq, xs, stream=None):
     """bf16 [B,H,N,d] -> INT4 codes in int8 containers, fp32 per-token scales."""
     _need_cuda(x, xq, xs)
     B, H, N, d = x.shape
+    _expect((x, (B, H, N, d), _BF16, "x"), (xq, (B, H, N, d), _I8, "xq"), (xs, (B, H, N), _F32, "xs"))
     _check("attn_quantize_int4", load().attn_quantize_int4(_ptr(x), _ptr(xq), _ptr(xs), B, H, N, d, _stream(stream)))
 
 
@@ -230,6 +271,9 @@ def attn_fwd_int8(q, qs, k, ks, v, vs, o, lse, causal: bool, scale: float, strea
     _need_cuda(q, qs, k, ks, v, vs, o, lse)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, Nq, d), _I8, "q"), (k, (B, H, Nkv, d), _I8, "k"), (v, (B, H, Nkv, d), _I8, "v"),
+            (qs, (B, H, Nq), _F32, "q_scale"), (ks, (B, H, Nkv), _F32, "k_scale"), (vs, (B, H), _F32, "v_scale"),
+            (o, (B, H, Nq, d), _F32, "o"), (lse, (B, H, Nq), _F32, "lse"))
     rc = load().attn_fwd_int8(_ptr(q), _ptr(qs), _ptr(k), _ptr(ks), _ptr(v), _ptr(vs), _ptr(o), _ptr(lse),
                               B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _stream(stream))
     _check("attn_fwd_int8", rc)
@@ -239,6 +283,8 @@ def attn_int8_scores(q, k, s, stream=None):
     """int32 S = q k^T of int8 [B,H,N,128] operands, through the INT8 MMA path."""
     _need_cuda(q, k, s)
     B, H, Nq, d = q.shape
+    _expect((q, (B, H, Nq, d), _I8, "q"), (k, (B, H, k.shape[2], d), _I8, "k"),
+            (s, (B, H, Nq, k.shape[2]), _I32, "s"))
     _check("attn_int8_scores", load().attn_int8_scores(_ptr(q), _ptr(k), _ptr(s), B, H, Nq, k.shape[2], d,
                                                          _stream(stream)))
 
@@ -255,6 +301,9 @@ def attn_quantize_nvfp4(x, codes, sf, mode: int, stream=None):
     """bf16 [B,H,N,128] -> packed e2m1 codes + tiled e4m3 scales (mode 0: Q/K, 1: V^T)."""
     _need_cuda(x, codes, sf)
     B, H, N, d = x.shape
+    _expect((x, (B, H, N, d), _BF16, "x"))
+    _at_least(codes, attn_nvfp4_codes_bytes(B, H, N, d, mode), "codes")
+    _at_least(sf, attn_nvfp4_sf_bytes(B, H, N, d, mode), "sf")
     _check("attn_quantize_nvfp4", load().attn_quantize_nvfp4(_ptr(x), _ptr(codes), _ptr(sf), B, H, N, d, int(mode),
                                                                _stream(stream)))
 
@@ -263,6 +312,11 @@ def attn_fwd_fp4(q, qsf, k, ksf, vt, vtsf, o, lse, B, H, Nq, Nkv, causal: bool, 
                  stream=None):
     """FP4 forward (codes/scales from attn_quantize_nvfp4) -> o fp32 [B,H,Nq,128], lse fp32."""
     _need_cuda(q, qsf, k, ksf, vt, vtsf, o, lse)
+    for t, n, m, nm in ((q, Nq, 0, "q"), (k, Nkv, 0, "k"), (vt, Nkv, 1, "vt")):
+        _at_least(t, attn_nvfp4_codes_bytes(B, H, n, 128, m), nm)
+    for t, n, m, nm in ((qsf, Nq, 0, "q_sf"), (ksf, Nkv, 0, "k_sf"), (vtsf, Nkv, 1, "vt_sf")):
+        _at_least(t, attn_nvfp4_sf_bytes(B, H, n, 128, m), nm)
+    _expect((o, (B, H, Nq, 128), _F32, "o"), (lse, (B, H, Nq), _F32, "lse"))
     rc = load().attn_fwd_fp4(_ptr(q), _ptr(qsf), _ptr(k), _ptr(ksf), _ptr(vt), _ptr(vtsf), _ptr(o), _ptr(lse),
                              B, H, Nq, Nkv, 128, int(bool(causal)), float(scale), int(p_mode), _stream(stream))
     _check("attn_fwd_fp4", rc)
@@ -271,6 +325,11 @@ def attn_fwd_fp4(q, qsf, k, ksf, vt, vtsf, o, lse, B, H, Nq, Nkv, causal: bool, 
 def attn_fp4_scores(q, qsf, k, ksf, s, B, H, Nq, Nkv, stream=None):
     """fp32 S = deq(q) deq(k)^T through the block-scaled FP4 MMA path."""
     _need_cuda(q, qsf, k, ksf, s)
+    for t, n, nm in ((q, Nq, "q"), (k, Nkv, "k")):
+        _at_least(t, attn_nvfp4_codes_bytes(B, H, n, 128, 0), nm)
+    for t, n, nm in ((qsf, Nq, "q_sf"), (ksf, Nkv, "k_sf")):
+        _at_least(t, attn_nvfp4_sf_bytes(B, H, n, 128, 0), nm)
+    _expect((s, (B, H, Nq, Nkv), _F32, "s"))
     _check("attn_fp4_scores", load().attn_fp4_scores(_ptr(q), _ptr(qsf), _ptr(k), _ptr(ksf), _ptr(s), B, H, Nq, Nkv,
                                                        128, _stream(stream)))
 
@@ -282,6 +341,10 @@ def attn_quantize_fp8(x, codes, scales, mode: int, signs=None, stream=None):
     if signs is not None:
         _need_cuda(signs)
     B, H, N, d = x.shape
+    _expect((x, (B, H, N, d), _BF16, "x"), (codes, (B, H, N, d), _U8, "codes"),
+            (scales, (B, H, N) if mode == 0 else (B, H, d), _F32, "scales"))
+    if signs is not None:
+        _expect((signs, (d,), _F32, "signs"))
     _check("attn_quantize_fp8", load().attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(scales), B, H, N, d, int(mode),
                                                            None if signs is None else _ptr(signs),
                                                            _stream(stream)))
@@ -292,6 +355,9 @@ def attn_fwd_fp8(q, qs, k, ks, v, vs, o, lse, causal: bool, scale: float, rotate
     _need_cuda(q, qs, k, ks, v, vs, o, lse)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
+    _expect((q, (B, H, Nq, d), _U8, "q"), (k, (B, H, Nkv, d), _U8, "k"), (v, (B, H, Nkv, d), _U8, "v"),
+            (qs, (B, H, Nq), _F32, "q_scale"), (ks, (B, H, Nkv), _F32, "k_scale"), (vs, (B, H, d), _F32, "v_scale"),
+            (o, (B, H, Nq, d), _F32, "o"), (lse, (B, H, Nq), _F32, "lse"))
     rc = load().attn_fwd_fp8(_ptr(q), _ptr(qs), _ptr(k), _ptr(ks), _ptr(v), _ptr(vs), _ptr(o), _ptr(lse),
                              B, H, Nq, Nkv, d, int(bool(causal)), float(scale), int(bool(rotated)),
                              _stream(stream))
