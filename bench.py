@@ -337,7 +337,7 @@ def run_ours(args):
             ta.attn_quantize_fp8(xq, c8[0], s8f[0], 0, signs, stream)
             ta.attn_quantize_fp8(xk, c8[1], s8f[1], 0, signs, stream)
             ta.attn_quantize_fp8(xv, c8[2], s8f[2], 1, None, stream)
-        seg("lowp_fp8_quantise", qf8, 3 * xq.numel() * 2 + 3 * xq.numel(), "GB/s", peak_hbm, "hbm", 3)
+        seg("lowp_fp8_quantise", qf8, 3 * xq.numel() * 2 + 3 * xq.numel(), "GB/s", peak_hbm, "hbm", 5)
         seg("lowp_fp8", lambda: ta.attn_fwd_fp8(c8[0], s8f[0], c8[1], s8f[1], c8[2], s8f[2], of, lf, False,
                                                 wq.scale, True, stream),
             wq.flops(False), "TFLOP/s", peak_f8, "tensor", 1)
