@@ -24,10 +24,15 @@
 // it stable): the recomputed P is rounded to e4m3 (unit scale, P <= 1) before
 // it enters dV = P^T dO; dS uses P unrounded.  e4m3 values are exact in bf16,
 // so the bf16 MMA computes exactly the product with the 8-bit P.
-// Each kernel: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 2-5
-// compute (thread = TMEM lane).  The score pair of a tile is computed, turned
-// into P / dS, then the accumulating MMAs run; the next tile's scores are
-// issued after them (their TMEM columns are reused).
+// Each kernel: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps
+// 2-17 compute: four warps per TMEM lane quarter (thread = lane = row of the
+// tile), each over 32 of the 128 columns, since P and dS are elementwise and
+// need no row reduction.  The two score groups of a tile have their own
+// barriers and the compute warps work in two phases, P from S first (kept in
+// fp32 registers), then dS from dP, so that the tensor core never waits for a
+// whole tile: dkdv issues S^T(t), dP^T(t) | dV(t), S^T(t+1) | dK(t), dP^T(t+1)
+// and dq issues S(t), dP(t) | S(t+1) | dQ(t), dP(t+1), each group as soon as
+// the compute phase it depends on has released its TMEM columns.
 #pragma once
 #include "ptx.cuh"
 #include "fwd_bf16.cuh"  // FwdCfg tile geometry, fwd_tile_kv_count, wait_bar_drain
@@ -78,10 +83,13 @@ struct BwdCfg {
   static constexpr int STAGE = 2 * TILE;
   static constexpr int FIX_OFF = 0;                   // the tile pair kept for the whole CTA
   static constexpr int ST_OFF = 2 * TILE;             // ring of tile pairs
-  static constexpr int COL_OFF = ST_OFF + NST * STAGE;  // dkdv: per-warp LSE / Dr columns [4][2][128]
-  static constexpr int BAR_OFF = COL_OFF + 4 * 2 * 128 * 4;
+  // compute warps: 4 per TMEM lane quarter, one 32-column chunk of the tile each
+  static constexpr int NCW = 16;
+  static constexpr int COL_OFF = ST_OFF + NST * STAGE;  // dkdv: per-warp LSE / Dr of its chunk [16][2][32]
+  static constexpr int BAR_OFF = COL_OFF + NCW * 2 * 32 * 4;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 64 + NCW * 32;  // producer, MMA issuer, compute warps
+  static constexpr int CT = NCW * 32;            // compute threads (barrier counts)
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);  // 128 x 128 scores
   static constexpr uint32_t ID_ACC = idesc_bf16_f32(128, D, true);   // accumulate, B MN-major
 };
@@ -90,8 +98,12 @@ struct BwdBars {
   uint64_t fix_full;
   uint64_t st_full[2];
   uint64_t st_empty[2];
-  uint64_t s_full;   // scores of the current tile pair in TMEM
-  uint64_t p_full;   // P / dS written back (count 128)
+  uint64_t s_full;   // S (S^T) of the current tile in TMEM
+  uint64_t dp_full;  // dP (dP^T) of the current tile in TMEM
+  uint64_t p_full;   // dkdv: P^T written back; dq: S read (all compute threads)
+  uint64_t ds_full;  // dS (dS^T) written back (all compute threads)
+  uint64_t s_read;   // dkdv: every compute thread holds its S^T chunk (P^T words may land)
+  uint64_t dp_read;  // dkdv: every compute thread holds its dP^T chunk
   uint64_t acc_full; // accumulators final
   uint64_t drain;
   uint32_t tmem_base;
@@ -99,20 +111,14 @@ struct BwdBars {
 };
 static_assert(sizeof(BwdBars) <= 256, "barrier block too large");
 
-// Score MMAs of one tile pair: D0 = A0 B0^T, D1 = A1 B1^T (K-major operands).
+// One score MMA group: D = A B^T (128 x 128, K-major operands).
 template <int D>
-__device__ __forceinline__ void bwd_issue_scores(uint32_t d0, uint32_t d1, uint64_t a0, uint64_t b0, uint64_t a1,
-                                                 uint64_t b1) {
+__device__ __forceinline__ void bwd_issue_score(uint32_t d, uint64_t a, uint64_t b) {
   using C = BwdCfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
-    mma_f16_ss(d0, a0 + off, b0 + off, C::ID_S, kk > 0);
-  }
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
-    mma_f16_ss(d1, a1 + off, b1 + off, C::ID_S, kk > 0);
+    mma_f16_ss(d, a + off, b + off, C::ID_S, kk > 0);
   }
 }
 // Accumulating MMA: Dacc (+)= A(tmem, 128 x 128 bf16) B(smem tile, MN-major).
@@ -124,24 +130,21 @@ __device__ __forceinline__ void bwd_issue_acc(uint32_t dacc, uint32_t a_tmem, ui
     mma_f16_ts(dacc, a_tmem + kk * 8, b + (uint64_t)(kk * (2048 >> 4)), C::ID_ACC, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// Rows of a [128 x D] fp32 accumulator in TMEM (this thread's lane) -> bf16
-// global row, times `mul`.
-template <int D>
-__device__ __forceinline__ void bwd_store_row(uint32_t tacc, uint16_t* dst, float mul, bool write) {
-#pragma unroll 1
-  for (int cc = 0; cc < D / 32; ++cc) {
-    uint32_t a[32];
-    tmem_ld32(tacc + cc * 32, a);
-    tmem_ld_wait(a);
-    if (write) {
+// 32 columns of a [128 x D] fp32 accumulator in TMEM (this thread's lane) ->
+// 32 bf16 of a global row, times `mul` (write = false: TMEM read only; the
+// load is warp-collective).
+__device__ __forceinline__ void bwd_store_chunk(uint32_t tacc, uint16_t* dst, float mul, bool write) {
+  uint32_t a[32];
+  tmem_ld32(tacc, a);
+  tmem_ld_wait(a);
+  if (write) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t w[4];
+    for (int g = 0; g < 4; ++g) {
+      uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w[e] = pack_bf16(__uint_as_float(a[g * 8 + 2 * e]) * mul, __uint_as_float(a[g * 8 + 2 * e + 1]) * mul);
-        *reinterpret_cast<uint4*>(dst + cc * 32 + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      for (int e = 0; e < 4; ++e)
+        w[e] = pack_bf16(__uint_as_float(a[g * 8 + 2 * e]) * mul, __uint_as_float(a[g * 8 + 2 * e + 1]) * mul);
+      *reinterpret_cast<uint4*>(dst + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
@@ -159,28 +162,6 @@ __device__ __forceinline__ uint32_t e4m3_round_bf16x2(float lo, float hi) {
   return pack_bf16(a, b);  // exact: every e4m3 value is a bf16 value
 }
 
-// P = exp2(S * sl2 - lse2) and dS = P (dP - Dr) for 32 columns, packed bf16x2
-// (P8: the P words hold e4m3-rounded P).
-template <bool P8 = false>
-__device__ __forceinline__ void bwd_p_ds(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float* lse2,
-                                         const float* rd, float sl2, uint32_t vis_mask, uint32_t (&pp)[16],
-                                         uint32_t (&pd)[16]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    float p0 = ex2(fmaf(__uint_as_float(s[i]), sl2, -lse2[i]));
-    float p1 = ex2(fmaf(__uint_as_float(s[i + 1]), sl2, -lse2[i + 1]));
-    p0 = ((vis_mask >> i) & 1u) ? p0 : 0.f;
-    p1 = ((vis_mask >> (i + 1)) & 1u) ? p1 : 0.f;
-    const float d0 = p0 * (__uint_as_float(dp[i]) - rd[i]);
-    const float d1 = p1 * (__uint_as_float(dp[i + 1]) - rd[i + 1]);
-    if constexpr (P8)
-      pp[i / 2] = e4m3_round_bf16x2(p0, p1);
-    else
-      pp[i / 2] = pack_bf16(p0, p1);
-    pd[i / 2] = pack_bf16(d0, d1);
-  }
-}
-
 // visible columns [c0, c0 + 32) of a row: key k sees query q iff q < Nq,
 // k < Nkv and (not causal or k <= q + Nkv - Nq)
 __device__ __forceinline__ uint32_t bwd_mask32(int lo, int hi) {  // bits [lo, hi) within 0..31
@@ -193,7 +174,7 @@ __device__ __forceinline__ uint32_t bwd_mask32(int lo, int hi) {  // bits [lo, h
 
 // ============================================================== dK, dV
 template <int D, bool P8 = false>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const BwdParams p) {
@@ -219,7 +200,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&bars->st_empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->s_full), 1);
-    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_full), C::CT);
+    mbar_init(smem_u32(&bars->ds_full), C::CT);
+    mbar_init(smem_u32(&bars->s_read), C::CT);
+    mbar_init(smem_u32(&bars->dp_read), C::CT);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -279,24 +264,41 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint64_t dK = smem_desc(sbase + C::FIX_OFF, 16, 1024);
       const uint64_t dV = smem_desc(sbase + C::FIX_OFF + C::TILE, 16, 1024);
-      for (int t = 0; t < nit && ok; ++t) {
-        const int s = t % C::NST;
-        ok = wait_bar(smem_u32(&bars->st_full[s]), (t / C::NST) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
+      auto stage = [&](int t) { return sbase + C::ST_OFF + (t % C::NST) * C::STAGE; };
+      auto stage_full = [&](int t) -> bool {
+        const bool r = wait_bar(smem_u32(&bars->st_full[t % C::NST]), (t / C::NST) & 1, abort_flag, p.timeout_ns);
         tc_fence_after();
-        const uint32_t st = sbase + C::ST_OFF + s * C::STAGE;
-        // S^T = K Q_i^T, dP^T = V dO_i^T
-        bwd_issue_scores<D>(tbase + T_S, tbase + T_DP, dK, smem_desc(st, 16, 1024), dV,
-                            smem_desc(st + C::TILE, 16, 1024));
+        return r;
+      };
+      // S^T(0) = K Q_0^T, dP^T(0) = V dO_0^T
+      if (ok && nit > 0 && (ok = stage_full(0))) {
+        bwd_issue_score<D>(tbase + T_S, dK, smem_desc(stage(0), 16, 1024));
         tc_commit(smem_u32(&bars->s_full));
+        bwd_issue_score<D>(tbase + T_DP, dV, smem_desc(stage(0) + C::TILE, 16, 1024));
+        tc_commit(smem_u32(&bars->dp_full));
+      }
+      for (int t = 0; t < nit && ok; ++t) {
+        const uint32_t st = stage(t);
         ok = wait_bar(smem_u32(&bars->p_full), t & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO_i, dK += dS^T Q_i (B operands MN-major: keys of the
-        // contraction are the tile's rows)
+        // dV += P^T dO_t (B operand MN-major: keys of the contraction are the tile's rows)
         bwd_issue_acc<D>(tbase + T_DV, tbase + T_S, smem_desc(st + C::TILE, C::HALF, 1024), t > 0);
+        if (t + 1 < nit) {  // S^T(t+1) over the P^T(t) columns, after the dV MMAs in the pipe
+          if (!(ok = stage_full(t + 1))) break;
+          bwd_issue_score<D>(tbase + T_S, dK, smem_desc(stage(t + 1), 16, 1024));
+          tc_commit(smem_u32(&bars->s_full));
+        }
+        ok = wait_bar(smem_u32(&bars->ds_full), t & 1, abort_flag, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        // dK += dS^T Q_t
         bwd_issue_acc<D>(tbase + T_DK, tbase + T_DP, smem_desc(st, C::HALF, 1024), t > 0);
-        tc_commit(smem_u32(&bars->st_empty[s]));
+        tc_commit(smem_u32(&bars->st_empty[t % C::NST]));
+        if (t + 1 < nit) {  // dP^T(t+1) over the dS^T(t) columns, after the dK MMAs
+          bwd_issue_score<D>(tbase + T_DP, dV, smem_desc(stage(t + 1) + C::TILE, 16, 1024));
+          tc_commit(smem_u32(&bars->dp_full));
+        }
       }
       if (ok) tc_commit(smem_u32(&bars->acc_full));
       if (!ok) {
@@ -306,52 +308,93 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    const int quarter = warp & 3;
+    // compute warp: TMEM lane quarter warp % 4 (its key rows), query columns [32c, 32c + 32)
+    const int cw = warp - 2;
+    const int quarter = warp & 3, c = cw >> 2;
     const int rr = quarter * 32 + lane;
     const int key = k0 + rr;  // this thread's key row
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float* cols = reinterpret_cast<float*>(smem + C::COL_OFF) + (warp - 2) * 256;  // [lse2 128][rd 128]
+    float* cols = reinterpret_cast<float*>(smem + C::COL_OFF) + cw * 64;  // [lse2 32][rd 32] of the chunk
     const float* lse_bh = p.lse + (size_t)bh * p.Nq;
     const float* rd_bh = p.rowdot + (size_t)bh * p.Nq;
     bool ok = true;
     for (int t = 0; t < nit && ok; ++t) {
-      const int q0 = (it0 + t) * 128;
-      // column statistics of this query tile, per warp: LSE in log2 units
-      // (+inf past the end, so that P = 0) and Dr
+      const int qc = (it0 + t) * 128 + 32 * c;  // first query column of this chunk
+      // column statistics of the chunk: LSE in log2 units (+inf past the end,
+      // so that P = 0) and Dr
       __syncwarp();
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int q = q0 + lane * 4 + e;
-        cols[lane * 4 + e] = (q < p.Nq) ? lse_bh[q] * 1.4426950408889634f : INFINITY;
-        cols[128 + lane * 4 + e] = (q < p.Nq) ? rd_bh[q] : 0.f;
+      {
+        const int q = qc + lane;
+        cols[lane] = (q < p.Nq) ? lse_bh[q] * 1.4426950408889634f : INFINITY;
+        cols[32 + lane] = (q < p.Nq) ? rd_bh[q] : 0.f;
       }
       __syncwarp();
       ok = wait_bar(smem_u32(&bars->s_full), t & 1, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tbase + lane_off + T_S + c * 32, s);
-        tmem_ld32(tbase + lane_off + T_DP + c * 32, dp);
-        tmem_ld_wait(s);
-        tmem_ld_wait(dp);
+      // phase 1: P^T = exp2(S^T sl2 - lse2) (masked), kept in fp32 for dS^T
+      float pf[32];
+      uint32_t pp[16];
+      {
+        uint32_t sv[32];
+        tmem_ld32(tbase + lane_off + T_S + c * 32, sv);
+        tmem_ld_wait(sv);
         // visible: q < Nq, key < Nkv, and (causal) q >= key - off
-        int lo = 0, hi = p.Nq - (q0 + c * 32);
+        int lo = 0, hi = p.Nq - qc;
         if (key >= p.Nkv) hi = 0;
-        if (p.causal) lo = key - off - (q0 + c * 32);
+        if (p.causal) lo = key - off - qc;
         const uint32_t vis = bwd_mask32(lo, hi);
-        uint32_t pp[16], pd[16];
-        bwd_p_ds<P8>(s, dp, cols + c * 32, cols + 128 + c * 32, p.sl2, vis, pp, pd);
-        // P^T and dS^T over columns already read (16 words land in the first
-        // half of the 32 columns this chunk index has passed)
-        tmem_st16(tbase + lane_off + T_S + c * 16, pp);
-        tmem_st16(tbase + lane_off + T_DP + c * 16, pd);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ((vis >> i) & 1u) ? ex2(fmaf(__uint_as_float(sv[i]), p.sl2, -cols[i])) : 0.f;
+          const float p1 = ((vis >> (i + 1)) & 1u) ? ex2(fmaf(__uint_as_float(sv[i + 1]), p.sl2, -cols[i + 1])) : 0.f;
+          pf[i] = p0;
+          pf[i + 1] = p1;
+          if constexpr (P8)
+            pp[i / 2] = e4m3_round_bf16x2(p0, p1);
+          else
+            pp[i / 2] = pack_bf16(p0, p1);
+        }
       }
+      // P^T words (bf16x2; P8: e4m3-rounded) of chunk c go to columns
+      // [16c, 16c + 16), scores another warp of this quarter reads: store
+      // them once every compute thread holds its chunk
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->s_read));
+      ok = wait_bar(smem_u32(&bars->s_read), t & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(tbase + lane_off + T_S + c * 16, pp);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full));
+      // phase 2: dS^T = P^T o (dP^T - Dr)
+      ok = wait_bar(smem_u32(&bars->dp_full), t & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pd[16];
+      {
+        uint32_t dp[32];
+        tmem_ld32(tbase + lane_off + T_DP + c * 32, dp);
+        tmem_ld_wait(dp);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+          pd[i / 2] = pack_bf16(pf[i] * (__uint_as_float(dp[i]) - cols[32 + i]),
+                                pf[i + 1] * (__uint_as_float(dp[i + 1]) - cols[33 + i]));
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->dp_read));
+      ok = wait_bar(smem_u32(&bars->dp_read), t & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(tbase + lane_off + T_DP + c * 16, pd);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->ds_full));
     }
     if (ok) {
       ok = wait_bar(smem_u32(&bars->acc_full), 0, abort_flag, p.timeout_ns);
@@ -360,13 +403,16 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) {
       tc_fence_after();
       const bool w = key < p.Nkv;
-      if (nit > 0) {
-        bwd_store_row<D>(tbase + lane_off + T_DV, p.dv + ((size_t)bh * p.Nkv + key) * D, 1.f, w);
-        bwd_store_row<D>(tbase + lane_off + T_DK, p.dk + ((size_t)bh * p.Nkv + key) * D, p.scale, w);
-      } else if (w) {  // no query sees these keys
-        for (int e = 0; e < D; e += 8) {
-          *reinterpret_cast<uint4*>(p.dv + ((size_t)bh * p.Nkv + key) * D + e) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(p.dk + ((size_t)bh * p.Nkv + key) * D + e) = make_uint4(0, 0, 0, 0);
+      // units of 32 accumulator columns: dV chunks, then dK chunks; four warps per quarter share them
+      for (int u = c; u < 2 * (D / 32); u += 4) {
+        const bool is_dv = u < D / 32;
+        const int cc = is_dv ? u : u - D / 32;
+        uint16_t* dst = (is_dv ? p.dv : p.dk) + ((size_t)bh * p.Nkv + key) * D + cc * 32;
+        if (nit > 0) {
+          bwd_store_chunk(tbase + lane_off + (is_dv ? T_DV : T_DK) + cc * 32, dst, is_dv ? 1.f : p.scale, w);
+        } else if (w) {  // no query sees these keys
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) *reinterpret_cast<uint4*>(dst + e) = make_uint4(0, 0, 0, 0);
         }
       }
     }
@@ -382,7 +428,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // ============================================================== dQ
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
@@ -405,7 +451,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&bars->st_empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->s_full), 1);
-    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_full), C::CT);
+    mbar_init(smem_u32(&bars->ds_full), C::CT);
+    mbar_init(smem_u32(&bars->s_read), C::CT);
+    mbar_init(smem_u32(&bars->dp_read), C::CT);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -419,8 +469,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
-  // TMEM: S [0,128), dP [128,256) (dS bf16 in [128,192)), dQ [256, 256+D)
-  const uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  // TMEM: S [0,128), dP [128,256), dQ [256, 256+D), dS (bf16x2) [384, 448):
+  // dS has columns of its own, so no compute warp writes over scores another reads
+  const uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DS = 384;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -464,22 +515,36 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint64_t dQ = smem_desc(sbase + C::FIX_OFF, 16, 1024);
       const uint64_t dDO = smem_desc(sbase + C::FIX_OFF + C::TILE, 16, 1024);
-      for (int t = 0; t < nj && ok; ++t) {
-        const int s = t % C::NST;
-        ok = wait_bar(smem_u32(&bars->st_full[s]), (t / C::NST) & 1, abort_flag, p.timeout_ns);
-        if (!ok) break;
+      auto stage = [&](int t) { return sbase + C::ST_OFF + (t % C::NST) * C::STAGE; };
+      auto stage_full = [&](int t) -> bool {
+        const bool r = wait_bar(smem_u32(&bars->st_full[t % C::NST]), (t / C::NST) & 1, abort_flag, p.timeout_ns);
         tc_fence_after();
-        const uint32_t st = sbase + C::ST_OFF + s * C::STAGE;
-        // S = Q K_j^T, dP = dO V_j^T
-        bwd_issue_scores<D>(tbase + T_S, tbase + T_DP, dQ, smem_desc(st, 16, 1024), dDO,
-                            smem_desc(st + C::TILE, 16, 1024));
+        return r;
+      };
+      // S(0) = Q K_0^T, dP(0) = dO V_0^T
+      if (ok && nj > 0 && (ok = stage_full(0))) {
+        bwd_issue_score<D>(tbase + T_S, dQ, smem_desc(stage(0), 16, 1024));
         tc_commit(smem_u32(&bars->s_full));
-        ok = wait_bar(smem_u32(&bars->p_full), t & 1, abort_flag, p.timeout_ns);
+        bwd_issue_score<D>(tbase + T_DP, dDO, smem_desc(stage(0) + C::TILE, 16, 1024));
+        tc_commit(smem_u32(&bars->dp_full));
+      }
+      for (int t = 0; t < nj && ok; ++t) {
+        if (t + 1 < nj) {  // S(t+1) once the compute warps hold S(t) in registers
+          ok = wait_bar(smem_u32(&bars->p_full), t & 1, abort_flag, p.timeout_ns);
+          if (!ok || !(ok = stage_full(t + 1))) break;
+          bwd_issue_score<D>(tbase + T_S, dQ, smem_desc(stage(t + 1), 16, 1024));
+          tc_commit(smem_u32(&bars->s_full));
+        }
+        ok = wait_bar(smem_u32(&bars->ds_full), t & 1, abort_flag, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        // dQ += dS K_j (K_j rows are the contraction: B MN-major)
-        bwd_issue_acc<D>(tbase + T_DQ, tbase + T_DP, smem_desc(st, C::HALF, 1024), t > 0);
-        tc_commit(smem_u32(&bars->st_empty[s]));
+        // dQ += dS K_t (K_t rows are the contraction: B MN-major)
+        bwd_issue_acc<D>(tbase + T_DQ, tbase + T_DS, smem_desc(stage(t), C::HALF, 1024), t > 0);
+        tc_commit(smem_u32(&bars->st_empty[t % C::NST]));
+        if (t + 1 < nj) {  // dP(t+1) once the compute warps hold dP(t) (ds_full)
+          bwd_issue_score<D>(tbase + T_DP, dDO, smem_desc(stage(t + 1) + C::TILE, 16, 1024));
+          tc_commit(smem_u32(&bars->dp_full));
+        }
       }
       if (ok) tc_commit(smem_u32(&bars->acc_full));
       if (!ok) {
@@ -489,45 +554,58 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    const int quarter = warp & 3;
+    // compute warp: TMEM lane quarter warp % 4 (its query rows), key columns [32c, 32c + 32)
+    const int cw = warp - 2;
+    const int quarter = warp & 3, c = cw >> 2;
     const int rr = quarter * 32 + lane;
     const int row = q0 + rr;  // this thread's query row
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const bool live = row < p.Nq;
     const float lse2 = live ? p.lse[(size_t)bh * p.Nq + row] * 1.4426950408889634f : INFINITY;
     const float rd = live ? p.rowdot[(size_t)bh * p.Nq + row] : 0.f;
-    float lse2v[32], rdv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      lse2v[i] = lse2;
-      rdv[i] = rd;
-    }
     bool ok = true;
     for (int t = 0; t < nj && ok; ++t) {
-      const int kb = t * 128;
+      const int kc = t * 128 + 32 * c;  // first key column of this chunk
       ok = wait_bar(smem_u32(&bars->s_full), t & 1, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tbase + lane_off + T_S + c * 32, s);
-        tmem_ld32(tbase + lane_off + T_DP + c * 32, dp);
-        tmem_ld_wait(s);
-        tmem_ld_wait(dp);
+      // phase 1: P = exp2(S sl2 - lse2) (masked) into fp32 registers; then
+      // the S columns are free for S(t+1)
+      float pf[32];
+      {
+        uint32_t sv[32];
+        tmem_ld32(tbase + lane_off + T_S + c * 32, sv);
+        tmem_ld_wait(sv);
         // visible keys: k < Nkv and (causal) k <= row + off
-        int hi = p.Nkv - (kb + c * 32);
-        if (p.causal) hi = min(hi, row + off - (kb + c * 32) + 1);
+        int hi = p.Nkv - kc;
+        if (p.causal) hi = min(hi, row + off - kc + 1);
         if (!live) hi = 0;
         const uint32_t vis = bwd_mask32(0, hi);
-        uint32_t pp[16], pd[16];
-        bwd_p_ds(s, dp, lse2v, rdv, p.sl2, vis, pp, pd);
-        tmem_st16(tbase + lane_off + T_DP + c * 16, pd);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          pf[i] = ((vis >> i) & 1u) ? ex2(fmaf(__uint_as_float(sv[i]), p.sl2, -lse2)) : 0.f;
       }
-      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full));
+      // phase 2: dS = P o (dP - Dr), bf16 into this chunk's dS columns
+      ok = wait_bar(smem_u32(&bars->dp_full), t & 1, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pd[16];
+      {
+        uint32_t dp[32];
+        tmem_ld32(tbase + lane_off + T_DP + c * 32, dp);
+        tmem_ld_wait(dp);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+          pd[i / 2] = pack_bf16(pf[i] * (__uint_as_float(dp[i]) - rd), pf[i + 1] * (__uint_as_float(dp[i + 1]) - rd));
+      }
+      tmem_st16(tbase + lane_off + T_DS + c * 16, pd);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->ds_full));
     }
     if (ok) {
       ok = wait_bar(smem_u32(&bars->acc_full), 0, abort_flag, p.timeout_ns);
@@ -536,10 +614,13 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) {
       tc_fence_after();
       uint16_t* dst = p.dq + ((size_t)bh * p.Nq + row) * D;
-      if (nj > 0) {
-        bwd_store_row<D>(tbase + lane_off + T_DQ, dst, p.scale, live);
-      } else if (live) {  // no key visible to this tile
-        for (int e = 0; e < D; e += 8) *reinterpret_cast<uint4*>(dst + e) = make_uint4(0, 0, 0, 0);
+      for (int cc = c; cc < D / 32; cc += 4) {
+        if (nj > 0) {
+          bwd_store_chunk(tbase + lane_off + T_DQ + cc * 32, dst + cc * 32, p.scale, live);
+        } else if (live) {  // no key visible to this tile
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) *reinterpret_cast<uint4*>(dst + cc * 32 + e) = make_uint4(0, 0, 0, 0);
+        }
       }
     }
   }
