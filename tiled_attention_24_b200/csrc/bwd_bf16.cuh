@@ -318,17 +318,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const float* lse_bh = p.lse + (size_t)bh * p.Nq;
     const float* rd_bh = p.rowdot + (size_t)bh * p.Nq;
     bool ok = true;
+    // column statistics of a chunk: LSE in log2 units (+inf past the end, so
+    // that P = 0) and Dr; lane i loads column i, one tile ahead of their use
+    auto load_stats = [&](int tt, float& ls, float& r) {
+      const int q = (it0 + tt) * 128 + 32 * c + lane;
+      ls = (q < p.Nq) ? lse_bh[q] * 1.4426950408889634f : INFINITY;
+      r = (q < p.Nq) ? rd_bh[q] : 0.f;
+    };
+    float nls = 0.f, nrd = 0.f;
+    if (nit > 0) load_stats(0, nls, nrd);
     for (int t = 0; t < nit && ok; ++t) {
       const int qc = (it0 + t) * 128 + 32 * c;  // first query column of this chunk
-      // column statistics of the chunk: LSE in log2 units (+inf past the end,
-      // so that P = 0) and Dr
       __syncwarp();
-      {
-        const int q = qc + lane;
-        cols[lane] = (q < p.Nq) ? lse_bh[q] * 1.4426950408889634f : INFINITY;
-        cols[32 + lane] = (q < p.Nq) ? rd_bh[q] : 0.f;
-      }
+      cols[lane] = nls;
+      cols[32 + lane] = nrd;
       __syncwarp();
+      if (t + 1 < nit) load_stats(t + 1, nls, nrd);
       ok = wait_bar(smem_u32(&bars->s_full), t & 1, abort_flag, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
