@@ -29,8 +29,9 @@ constexpr int DEC_THREADS = 128;
 constexpr int DEC_SB = 512;  // keys per sub-block
 constexpr int DEC_UNROLL = 8;
 // grouped kernel: loads in flight per lane, by heads per CTA (measured on
-// B200 with B64 Hq32 N_kv 8192: G = 4 is fastest with 4, G = 8 with 8)
-__host__ __device__ constexpr int dec_group_unroll(int G) { return G == 4 ? 4 : 8; }
+// B200 with B64 Hq32 N_kv 8192, G = 4: 0.499 ms with 8, 0.516 with 4,
+// 1.07 with 2; G = 8 also fastest with 8)
+__host__ __device__ constexpr int dec_group_unroll(int) { return 8; }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
