@@ -182,18 +182,21 @@ def run_reference(args):
         return 0
     vals = []
     desc, thr = "", 1
-    for _ in range(args.warmup_ref):
-        oracle_sample(5.0)
+    # each step is a bounded sample (whole (head, mode) passes until the cap),
+    # sized so that the W + K steps take about 150 s at most
+    cap = min(20.0, max(0.3, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(cap)
     t_all = time.perf_counter()
-    for _ in range(args.steps_ref):
-        v, desc, thr, _ = oracle_sample(20.0)
+    for _ in range(args.steps):
+        v, desc, thr, _ = oracle_sample(cap)
         vals.append(v)
     wall = time.perf_counter() - t_all
     val = statistics.mean(vals)
     line = {
         "impl": "reference", "metric": "attn fwd TFLOP/s (prefill B4 H16 N4096 d128, non-causal + causal)",
-        "value": val, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps_ref, "warmup": args.warmup_ref,
-        "ms_per_step": wall / max(1, args.steps_ref) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "value": val, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
         "config": {"workload": "prefill", "B": 4, "H": 16, "Nq": 4096, "Nkv": 4096, "d": 128,
                    "causal": ["false", "true"], "sample": "bounded oracle sample"},
@@ -504,8 +507,6 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="decode batch override (profiling aid; 0 = the workload's 64)")
     args = ap.parse_args()
-    args.steps_ref = max(1, min(args.steps, 3))
-    args.warmup_ref = 0
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
