@@ -274,8 +274,9 @@ def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = 
                 move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
                 if jb > 0:
                     rescales += int(np.count_nonzero(move & np.isfinite(m)))
-                f = np.where(move & np.isfinite(m),
-                             np.exp2(np.where(move & np.isfinite(m), m - m_new, 0.0)), 1.0)
+                with np.errstate(invalid="ignore"):  # -inf - -inf in lanes the where() discards
+                    f = np.where(move & np.isfinite(m),
+                                 np.exp2(np.where(move & np.isfinite(m), m - m_new, 0.0)), 1.0)
                 acc *= f[:, None]
                 l *= f
                 m = np.where(move, m_new, m)
