@@ -450,6 +450,8 @@ def run_ours(args):
                 "kernel": "fwd_bf16_kernel<128>, prefill B4 H16 N4096 d128 non-causal",
                 "peak_source": f"{peak_src} bf16 burst"}
     for part, key in (("decode", "decode_split"), ("longseq_noncausal", "fwd_bf16_longseq_noncausal"),
+                      ("longseq_causal", "fwd_bf16_longseq_causal"), ("prefill_varlen_causal", "fwd_bf16_varlen_causal"),
+                      ("prefill_noncausal", "fwd_bf16_prefill_noncausal"),
                       ("prefill_causal", "fwd_bf16_prefill_causal"), ("lowp_int8", "fwd_int8_lowp"),
                       ("lowp_fp4_direct_p", "fwd_fp4_direct_p_lowp"),
                       ("lowp_fp4_quant_after_exp", "fwd_fp4_quant_after_exp_lowp"), ("lowp_fp8", "fwd_fp8_lowp")):
