@@ -103,6 +103,14 @@ def test_bwd_workspace_and_validation(lib):
                             a["scale"], ws, a["ws_bytes"], None)
     assert call(d=96) == -2 and call(scale=0.0) == -1 and call(B=-1) == -1 and call(Nkv=-2) == -1
     assert call(ws_bytes=16) == -1 and call(B=0) == 0
+    # the FP8-P entry point validates exactly like attn_bwd
+    def call8(**kw):
+        a = dict(B=1, H=2, Nq=64, Nkv=64, d=128, causal=0, scale=0.1, ws_bytes=n)
+        a.update(kw)
+        return lib.attn_bwd_fp8p(P, P, P, P, P, P, P, P, P, a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
+                                 a["scale"], ws, a["ws_bytes"], None)
+    assert call8(d=96) == -2 and call8(scale=0.0) == -1 and call8(B=-1) == -1 and call8(ws_bytes=16) == -1
+    assert call8(B=0) == 0
 
 
 def test_fp8_host_validation(lib):
