@@ -24,6 +24,8 @@ import math
 
 import numpy as np
 
+from .outcomes import near_midpoint
+
 LOG2E = 1.0 / math.log(2.0)
 LN2 = math.log(2.0)
 
@@ -88,7 +90,7 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None,
 
 
 def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = None, p_round=None,
-                       flip_band=None):
+                       p_grid=None, p_rel=2e-5):
     """Gradients of O = softmax(scale * Q K^T, masked) V with respect to Q, K
     and V for an upstream gradient dO, in float64 -- the calculus of the
     definition, with P materialised (the quantity [FA-trading] "Backward:
@@ -103,11 +105,12 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
 
     ``p_round`` (a function on arrays) rounds P where it is the operand of
     dV = round(P)^T dO only (the FP8-P backward of [FP4-FA4]: 8-bit
-    probabilities in the backward); dS keeps P unrounded.  With ``flip_band``
-    = (midpoints, step, rel) it also returns, per dV element, a bound on what
-    P elements within ``rel`` (relative) of a rounding midpoint change if
-    they round to the other neighbour (``step(P)`` = that neighbour's
-    distance): sum_i flip_ij |dO_ic|."""
+    probabilities in the backward); dS keeps P unrounded.  With ``p_grid``
+    (the sorted non-negative values ``p_round`` rounds to) it also returns
+    the interval (dV_lo, dV_hi) of dV over both roundings of every P element
+    within ``p_rel`` (relative) of a rounding midpoint of that grid: dV is
+    linear in the rounded P, so each such element adds its change times dO
+    to one end of the interval (``oracle.outcomes``)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
@@ -116,7 +119,8 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    fb = np.zeros_like(v)
+    dv_lo = np.zeros_like(v)
+    dv_hi = np.zeros_like(v)
     vis = visible_mask(Nq, Nkv, causal)
     for b in range(B):
         for h in range(H):
@@ -132,14 +136,16 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
             dv[b, h] = Pv.T @ do[b, h]
             dq[b, h] = scale * (dS @ k[b, h])
             dk[b, h] = scale * (dS.T @ q[b, h])
-            if flip_band is not None:
-                mids, step, rel = flip_band
-                near = np.zeros(P.shape, dtype=bool)
-                for t in mids:
-                    near |= np.abs(P - t) <= rel * t
-                fb[b, h] = np.where(near & (P > 0), step(P), 0.0).T @ np.abs(do[b, h])
-    if flip_band is not None:
-        return dq, dk, dv, fb
+            if p_grid is not None:
+                flag, alt = near_midpoint(P, p_grid, Pv, p_rel * P)
+                delta = np.where(flag & (P > 0), alt - Pv, 0.0)             # [Nq, Nkv]
+                up, dn = np.maximum(delta, 0.0), np.minimum(delta, 0.0)
+                dpos, dneg = np.maximum(do[b, h], 0.0), np.minimum(do[b, h], 0.0)
+                # sum_i min(0, delta_ij dO_ic) and sum_i max(0, delta_ij dO_ic)
+                dv_lo[b, h] = dv[b, h] + up.T @ dneg + dn.T @ dpos
+                dv_hi[b, h] = dv[b, h] + up.T @ dpos + dn.T @ dneg
+    if p_grid is not None:
+        return dq, dk, dv, (dv_lo, dv_hi)
     return dq, dk, dv
 
 

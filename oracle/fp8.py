@@ -42,7 +42,8 @@ import math
 import numpy as np
 
 from .attention import LN2, LOG2E, _f64, visible_mask
-from .lowp import UE4M3_VALUES, _near_half  # noqa: F401  (value table of the format)
+from .lowp import UE4M3_VALUES, _RangeCollector  # value table of the format; interval collector
+from .outcomes import EVAL_REL, FlipRecorder, eval_band, near_midpoint
 
 F32 = np.float32
 E4M3_MAX = 448.0
@@ -109,14 +110,67 @@ def quantize_fp8_channels(v):
     return q, s
 
 
+def _fp8_rows(x, vvs, tau, Bc, outcomes, invert=None):
+    """Steps 4-5 for the rows of one (batch, head): x [R, Nkv] base-2 scores
+    (masked = -inf), vvs [Nkv, d] = codes(V) * s_V (the channel scales folded
+    in, which is exact in exact arithmetic).  ``invert`` [R, n_blocks] bool
+    reverses the lazy-rescale decision of those (row, block) pairs.  Returns
+    (num [R, d], l, m, FlipRecorder or None, ambiguous [R, n_blocks])."""
+    R, Nkv = x.shape
+    nblk = -(-Nkv // Bc)
+    num = np.zeros((R, vvs.shape[1]))
+    l = np.zeros(R)
+    m = np.full(R, -np.inf)
+    rec = FlipRecorder() if outcomes else None
+    amb = np.zeros((R, nblk), dtype=bool)
+    for jb, j0 in enumerate(range(0, Nkv, Bc)):
+        cols = slice(j0, min(Nkv, j0 + Bc))
+        xb = x[:, cols]
+        m_blk = xb.max(axis=1)
+        m_new = np.maximum(m, m_blk)
+        move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
+        if tau > 0:
+            both = np.isfinite(m) & np.isfinite(m_blk)
+            mb0, m0 = np.where(both, m_blk, 0.0), np.where(both, m, 0.0)
+            amb[:, jb] = both & (np.abs(mb0 - (m0 + tau)) <= EVAL_REL * (np.abs(mb0) + np.abs(m0) + 1.0))
+            if invert is not None:
+                # the other decision: move to the block max (if the block raises it at all)
+                flip = invert[:, jb] & both
+                move = np.where(flip, ~move & (m_new > m), move)
+        grow = move & np.isfinite(m)
+        f = np.ones_like(m)
+        with np.errstate(invalid="ignore"):  # -inf - -inf where not grow (not used)
+            np.exp2(m - m_new, out=f, where=grow)
+        num *= f[:, None]
+        l *= f
+        m = np.where(move, m_new, m)
+        ms = np.where(np.isfinite(m), m, 0.0)
+        fin = np.isfinite(xb) & np.isfinite(m)[:, None]
+        p = np.zeros_like(xb)
+        np.exp2(np.where(fin, xb - ms[:, None], 0.0), out=p, where=fin)
+        P = e4m3_encode_value(p)
+        if outcomes:
+            band = eval_band(p, np.where(fin, xb, 0.0), ms[:, None], 1e-12)
+            flag, alt = near_midpoint(p, UE4M3_VALUES, P, band)
+            r_, c_ = np.nonzero(flag & fin)
+            rec.add_elements(r_, c_ + j0, (alt - P)[r_, c_], ms[r_])
+        l += P.sum(axis=1)
+        num += P @ vvs[cols]
+    return num, l, m, rec, amb
+
+
 def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=128,
-                  with_flip_bound=False, rows=None, tau=0.0):
+                  outcomes=False, rows=None, tau=0.0, max_branches=64):
     """Emulated FP8 forward (steps 3-5 of the module docstring) from code values
     and scales; ``rot_d`` = d when Q and K were rotated (the product is then d
     times Q K^T), 1 otherwise.  Returns (O, LSE) float64 and, with
-    ``with_flip_bound``, (flip_bound, lse_flip_bound, flips): how far O and
-    LSE can move if a P element within fp32 evaluation error of an e4m3
-    rounding midpoint rounds the other way on the device."""
+    ``outcomes``, also an ``OutcomeRange`` over both roundings of every P
+    element within fp32 evaluation error of an e4m3 rounding midpoint
+    (``oracle.outcomes``).  Where a lazy-rescale decision (block max above
+    the reference by more than tau) lies within that error of the threshold,
+    a device may decide either way: the row is then followed down both
+    decisions (up to ``max_branches`` paths per row) and its interval is the
+    hull of theirs; ``ambiguous_rescales`` counts such decisions."""
     qv, kv, vv = _f64(qv), _f64(kv), _f64(vv)
     B, H, Nq_all, d = qv.shape
     Nkv = kv.shape[2]
@@ -126,62 +180,54 @@ def attention_fp8(qv, qs, kv, ks, vv, vs, causal=False, scale=None, rot_d=1, Bc=
     Nq = ridx.size
     O = np.zeros((B, H, Nq, d))
     LSE = np.full((B, H, Nq), -np.inf)
-    FB = np.zeros((B, H, Nq, d))
-    LB = np.zeros((B, H, Nq))
-    flips = 0
+    rng = _RangeCollector(O.shape) if outcomes else None
     vis = visible_mask(Nq_all, Nkv, causal, ridx)
-    # e4m3 rounding midpoints up to the largest P~ (2^tau): the value between two neighbours
-    mids = (UE4M3_VALUES[:-1] + UE4M3_VALUES[1:]) / 2.0
-    mids = mids[mids <= 2.0 ** tau * 1.07]
     for b in range(B):
         for h in range(H):
             S = (qv[b, h, ridx] @ kv[b, h].T).astype(F32).astype(np.float64)
             x = S * (_f64(qs)[b, h, ridx][:, None] * _f64(ks)[b, h][None, :]) * (scale * LOG2E / rot_d)
             x = np.where(vis, x, -np.inf)
-            acc = np.zeros((Nq, d))
-            l = np.zeros(Nq)
-            m = np.full(Nq, -np.inf)
-            wflip = np.zeros((Nq, Nkv))
-            for j0 in range(0, Nkv, Bc):
-                cols = slice(j0, min(Nkv, j0 + Bc))
-                xb = x[:, cols]
-                m_new = np.maximum(m, xb.max(axis=1))
-                move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
-                grow = move & np.isfinite(m)
-                f = np.ones_like(m)
-                with np.errstate(invalid="ignore"):  # -inf - -inf where not grow (not used)
-                    np.exp2(m - m_new, out=f, where=grow)
-                acc *= f[:, None]
-                l *= f
-                m = np.where(move, m_new, m)
-                ms = np.where(np.isfinite(m), m, 0.0)
-                fin = np.isfinite(xb) & np.isfinite(m)[:, None]
-                p = np.zeros_like(xb)
-                np.exp2(np.where(fin, xb - ms[:, None], 0.0), out=p, where=fin)
-                P = e4m3_encode_value(p)
-                if with_flip_bound:
-                    # fp32 evaluation of x and of exp2: a few ulps of |x|, |m|
-                    dx = 2e-6 * (np.abs(np.where(fin, xb, 0.0)) + np.abs(ms)[:, None] + 1.0)
-                    band = p * LN2 * dx + 1e-7
-                    near = np.zeros_like(p, dtype=bool)
-                    for t in mids:
-                        near |= np.abs(p - t) < band
-                    near &= fin
-                    # a flip moves P by one e4m3 step: at most 2^-3 * P (normal) or 2^-9
-                    step = np.maximum(p * 0.125, 2.0 ** -9)
-                    wflip[:, cols] = np.where(near, step, 0.0)
-                l += P.sum(axis=1)
-                acc += P @ vv[b, h, cols]
+            vvs = vv[b, h] * _f64(vs)[b, h][None, :]
+            num, l, m, rec, amb = _fp8_rows(x, vvs, tau, Bc, outcomes)
             ok = l > 0
             ls = np.where(ok, l, 1.0)
-            sv = _f64(vs)[b, h]
-            O[b, h] = np.where(ok[:, None], acc * sv[None, :] / ls[:, None], 0.0)
+            O[b, h] = np.where(ok[:, None], num / ls[:, None], 0.0)
             LSE[b, h] = np.where(ok, LN2 * (np.where(ok, m, 0.0) + np.log2(ls)), -np.inf)
-            if with_flip_bound:
-                flips += int(np.count_nonzero(wflip))
-                vdeq = vv[b, h] * sv[None, :]
-                FB[b, h] = (wflip @ np.abs(vdeq) + wflip.sum(axis=1)[:, None] * np.abs(O[b, h])) / ls[:, None]
-                LB[b, h] = wflip.sum(axis=1) / ls * 1.01
-    if with_flip_bound:
-        return O, LSE, FB, LB, flips
+            if outcomes:
+                rng.add(b, h, rec, num, l, m, vvs, 1.0)
+                for r in np.flatnonzero(amb.any(axis=1)):
+                    _fp8_branch_hull(rng, b, h, r, x[r:r + 1], vvs, tau, Bc, amb[r], max_branches)
+    if outcomes:
+        return O, LSE, rng.result(O, LSE)
     return O, LSE
+
+
+def _fp8_branch_hull(rng, b, h, r, xr, vvs, tau, Bc, amb_r, max_branches):
+    """Follow every combination of decisions at the ambiguous blocks of row r
+    (new ambiguities found on a branch are followed too) and widen the row's
+    interval in ``rng`` to the hull of all branches."""
+    nblk = amb_r.size
+    seen = set()
+    todo = [np.zeros(nblk, dtype=bool)]
+    pending = [np.flatnonzero(amb_r)]
+    branches = 0
+    while todo:
+        inv = todo.pop()
+        cand = pending.pop()
+        for jb in cand:
+            nxt = inv.copy()
+            nxt[jb] = ~nxt[jb]
+            key = nxt.tobytes()
+            if key in seen:
+                continue
+            seen.add(key)
+            branches += 1
+            if branches > max_branches:
+                raise ValueError(f"row {r}: more than {max_branches} lazy-rescale decision paths")
+            num, l, m, rec, amb = _fp8_rows(xr, vvs, tau, Bc, True, invert=nxt[None, :])
+            lo, hi, llo, lhi = rec.intervals(num, l, m, vvs, 1.0)
+            rng.widen(b, h, r, lo[0], hi[0], llo[0], lhi[0], m[0])
+            rng.flips += rec.count()
+            todo.append(nxt)
+            pending.append(np.flatnonzero(amb[0] & ~nxt))
+    rng.ambiguous += int(amb_r.sum())

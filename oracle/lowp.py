@@ -48,6 +48,7 @@ import math
 import numpy as np
 
 from .attention import LN2, LOG2E, _f64, visible_mask
+from .outcomes import FlipRecorder, OutcomeRange, eval_band, near_midpoint, subset_options
 
 F32 = np.float32
 
@@ -105,22 +106,16 @@ def int8_scores(qi, ki):
     return S.astype(np.int32)
 
 
-def _near_half(y, band):
-    """True where y lies within ``band`` of a rounding midpoint k + 1/2."""
-    return np.abs(y - (np.floor(y) + 0.5)) < band
-
-
 def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
-                   with_flip_bound=False, rows=None):
+                   outcomes=False, rows=None):
     """Emulated INT8 forward (steps 2-5 of the module docstring).
 
     qi, ki, vi: int8 [B,H,N,d]; qs, ks: fp32 [B,H,N]; vs: fp32 [B,H].
     ``rows`` restricts the computation to those query rows (rows are
-    independent).  Returns (O, LSE) float64 and, with ``with_flip_bound``,
-    (flip_bound [B,H,Nq,d],
-    lse_flip_bound [B,H,Nq], flips): how far O and LSE can move when an element
-    of 127 * 2^(x - m) that lies within the fp32 evaluation error of a rounding
-    midpoint rounds the other way on a device that computes x and 2^x in fp32.
+    independent).  Returns (O, LSE) float64 and, with ``outcomes``, also an
+    ``OutcomeRange``: the interval of O and LSE over both roundings of every
+    element of 127 * 2^(x - m) that lies within fp32 evaluation error of a
+    rounding midpoint (``oracle.outcomes``).
     """
     qi, ki, vi = np.asarray(qi), np.asarray(ki), np.asarray(vi)
     qs, ks, vs = _f64(qs), _f64(ks), _f64(vs)
@@ -132,9 +127,8 @@ def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
     Nq = ridx.size
     O = np.zeros((B, H, Nq, d))
     LSE = np.full((B, H, Nq), -np.inf)
-    FB = np.zeros((B, H, Nq, d))
-    LB = np.zeros((B, H, Nq))
-    flips = 0
+    rng = _RangeCollector(O.shape) if outcomes else None
+    grid = np.arange(128.0)
     vis = visible_mask(Nq_all, Nkv, causal, ridx)
     for b in range(B):
         for h in range(H):
@@ -144,8 +138,7 @@ def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
             acc = np.zeros((Nq, d))
             l = np.zeros(Nq)
             m = np.full(Nq, -np.inf)
-            flag = np.zeros((Nq, Nkv), dtype=bool)
-            vdeq = vi[b, h].astype(np.float64) * vs[b, h]
+            rec = FlipRecorder()
             for j0 in range(0, Nkv, Bc):
                 cols = slice(j0, min(Nkv, j0 + Bc))
                 xb = x[:, cols]
@@ -162,24 +155,66 @@ def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
                 np.exp2(np.where(fin, xb - ms[:, None], 0.0), out=p, where=fin)
                 y = 127.0 * p
                 P8 = np.rint(y)
-                # fp32 evaluation of x (few ulps of |x|, |m|) and of exp2
-                dx = 2e-6 * (np.abs(np.where(fin, xb, 0.0)) + np.abs(ms)[:, None] + 1.0)
-                flag[:, cols] = fin & _near_half(y, y * LN2 * dx + 1e-4)
+                if outcomes:
+                    band = eval_band(y, np.where(fin, xb, 0.0), ms[:, None], 1e-12)
+                    flag, alt = near_midpoint(y, grid, P8, band)
+                    r_, c_ = np.nonzero(flag & fin)
+                    rec.add_elements(r_, c_ + j0, (alt - P8)[r_, c_], ms[r_])
                 l += P8.sum(axis=1) / 127.0
                 acc += (P8 @ vi[b, h, cols].astype(np.float64)) * (vs[b, h] / 127.0)
             ok = l > 0
             ls = np.where(ok, l, 1.0)
             O[b, h] = np.where(ok[:, None], acc / ls[:, None], 0.0)
             LSE[b, h] = np.where(ok, LN2 * (np.where(ok, m, 0.0) + np.log2(ls)), -np.inf)
-            if with_flip_bound:
-                fl = flag.astype(np.float64)
-                nfl = fl.sum(axis=1)
-                flips += int(nfl.sum())
-                FB[b, h] = (fl @ np.abs(vdeq) + nfl[:, None] * np.abs(O[b, h])) / (127.0 * ls[:, None])
-                LB[b, h] = nfl / (127.0 * ls) * 1.01
-    if with_flip_bound:
-        return O, LSE, FB, LB, flips
+            if outcomes:
+                U = vi[b, h].astype(np.float64) * (vs[b, h] / 127.0)
+                rng.add(b, h, rec, acc, l, m, U, 1.0 / 127.0)
+    if outcomes:
+        return O, LSE, rng.result(O, LSE)
     return O, LSE
+
+
+class _RangeCollector:
+    """Gathers the per-(b, h) intervals of a blockwise quantised forward into
+    one ``OutcomeRange``."""
+
+    def __init__(self, shape):
+        self.O_lo = np.zeros(shape)
+        self.O_hi = np.zeros(shape)
+        self.l_lo = np.zeros(shape[:-1])
+        self.l_hi = np.zeros(shape[:-1])
+        self.m = np.zeros(shape[:-1])
+        self.flips = 0
+        self.flagged_rows = 0
+        self.ambiguous = 0
+
+    def add(self, b, h, rec, num, l, m, U, w):
+        lo, hi, llo, lhi = rec.intervals(num, l, m, U, w)
+        self.O_lo[b, h], self.O_hi[b, h] = lo, hi
+        self.l_lo[b, h], self.l_hi[b, h] = llo, lhi
+        self.m[b, h] = np.where(np.isfinite(m), m, 0.0)
+        self.flips += rec.count()
+        self.flagged_rows += len(rec.vars)
+
+    def widen(self, b, h, r, lo, hi, llo, lhi, m):
+        """Hull of row r's interval with another decision path's, whose
+        reference max is m (the LSE ends are compared on a common base)."""
+        self.O_lo[b, h, r] = np.minimum(self.O_lo[b, h, r], lo)
+        self.O_hi[b, h, r] = np.maximum(self.O_hi[b, h, r], hi)
+        m0 = self.m[b, h, r]
+        # l at reference m equals l * 2^(m - m0) at reference m0
+        self.l_lo[b, h, r] = min(self.l_lo[b, h, r], llo * 2.0 ** (m - m0))
+        self.l_hi[b, h, r] = max(self.l_hi[b, h, r], lhi * 2.0 ** (m - m0))
+
+    def result(self, O, LSE):
+        fin = np.isfinite(LSE)
+        lse_lo = np.where(fin, LN2 * (self.m + np.log2(np.where(fin, self.l_lo, 1.0))), -np.inf)
+        lse_hi = np.where(fin, LN2 * (self.m + np.log2(np.where(fin, self.l_hi, 1.0))), -np.inf)
+        # rows that see no key: O = 0 exactly on both sides
+        O_lo = np.where(fin[..., None], self.O_lo, O)
+        O_hi = np.where(fin[..., None], self.O_hi, O)
+        return OutcomeRange(O_lo, O_hi, lse_lo, lse_hi, self.flips, self.flagged_rows,
+                            int(np.prod(LSE.shape)), self.ambiguous)
 
 
 # ----------------------------------------------------------------------------
@@ -292,14 +327,16 @@ def quant_after_exp_values(p, block=16):
 
 
 def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None,
-                  Bc=128, with_flip_bound=False):
+                  Bc=128, outcomes=False):
     """Emulated FP4 forward (steps 2-4 of the module docstring).
 
     q_deq, k_deq, v_deq: dequantised NVFP4 operands [B,H,N,d] (float64; use
-    ``nvfp4_dequantize``).  Returns (O, LSE) and, with ``with_flip_bound``,
-    (flip_bound, lse_flip_bound, flips) as in ``attention_int8``: the change of
-    O and LSE if a P element that sits within the device's fp32 error of an
-    e2m1 (or e4m3 scale) rounding boundary falls on the other side."""
+    ``nvfp4_dequantize``).  Returns (O, LSE) and, with ``outcomes``, also an
+    ``OutcomeRange`` over both roundings of every P element that lies within
+    the device's fp32 evaluation error of an e2m1 rounding midpoint, and, for
+    quantise-after-exp, over both roundings of a block scale amax / 6 that
+    lies that close to an e4m3 midpoint (the block's codes then follow the
+    chosen scale).  See ``oracle.outcomes``."""
     q, k, v = _f64(q_deq), _f64(k_deq), _f64(v_deq)
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
@@ -308,11 +345,8 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
     p_unit = 6.0 if p_mode == DIRECT_P else 1.0
     O = np.zeros((B, H, Nq, d))
     LSE = np.full((B, H, Nq), -np.inf)
-    FB = np.zeros((B, H, Nq, d))
-    LB = np.zeros((B, H, Nq))
-    flips = 0
+    rng = _RangeCollector(O.shape) if outcomes else None
     vis = visible_mask(Nq, Nkv, causal)
-    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
     for b in range(B):
         for h in range(H):
             x = (q[b, h] @ k[b, h].T) * (scale * LOG2E)
@@ -320,7 +354,7 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
             acc = np.zeros((Nq, d))
             l = np.zeros(Nq)
             m = np.full(Nq, -np.inf)
-            wflip = np.zeros((Nq, Nkv))      # per element: worst change of P~/p_unit
+            rec = FlipRecorder()
             for j0 in range(0, Nkv, Bc):
                 j1 = min(Nkv, j0 + Bc)
                 cols = slice(j0, j1)
@@ -335,12 +369,14 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
                 ms = np.where(np.isfinite(m), m, 0.0)
                 fin = np.isfinite(xb) & np.isfinite(m)[:, None]
                 xp = np.where(fin, xb - ms[:, None], -np.inf)
-                dx = 2e-6 * (np.abs(np.where(fin, xb, 0.0)) + np.abs(ms)[:, None] + 1.0)
                 if p_mode == DIRECT_P:
                     Pt, _ = direct_p_values(xp)
-                    y = np.where(fin, 6.0 * np.exp2(np.minimum(np.where(fin, xp, 0.0), 0.0)), 0.0)
-                    near = fin & (np.abs(y[..., None] - mids).min(axis=-1) < y * LN2 * dx + 1e-6)
-                    wflip[:, cols] = np.where(near, 2.0, 0.0) / p_unit
+                    if outcomes:
+                        y = np.where(fin, 6.0 * np.exp2(np.minimum(np.where(fin, xp, 0.0), 0.0)), 0.0)
+                        band = eval_band(y, np.where(fin, xb, 0.0), ms[:, None], 1e-12)
+                        flag, alt = near_midpoint(y, E2M1_VALUES, Pt, band)
+                        r_, c_ = np.nonzero(flag & fin)
+                        rec.add_elements(r_, c_ + j0, (alt - Pt)[r_, c_], ms[r_])
                 else:
                     width = j1 - j0
                     pad = (-width) % 16
@@ -350,28 +386,74 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
                     pp = np.pad(p32, ((0, 0), (0, pad)))
                     Pt_full, _, sf = quant_after_exp_values(pp)
                     Pt = Pt_full[:, :width]
-                    # boundaries: the code boundaries of p / sf, and the scale's own
-                    s = np.repeat(ue4m3_decode(sf), 16, axis=-1)[:, :width]
-                    r = np.where(s > 0, p / np.where(s > 0, s, 1.0), 0.0)
-                    near = fin & (np.abs(r[..., None] - mids).min(axis=-1) < r * LN2 * dx + 1e-6)
-                    amax = pp.reshape(Nq, -1, 16).max(axis=-1) / 6.0
-                    sv = UE4M3_VALUES
-                    smid = (sv[1:] + sv[:-1]) / 2.0
-                    snear = np.abs(amax[..., None] - smid).min(axis=-1) < amax * LN2 * dx.max() + 1e-12
-                    snear = np.repeat(snear, 16, axis=-1)[:, :width]
-                    step = np.where(near, np.maximum(s, 0) * 2.0, 0.0)
-                    step = np.where(snear & fin, np.maximum(step, 0.25 * np.maximum(p, 0.0) + s), step)
-                    wflip[:, cols] = step / p_unit
+                    if outcomes:
+                        xe = np.pad(np.where(fin, xb, 0.0), ((0, 0), (0, pad)))
+                        _qae_flips(rec, pp.astype(np.float64), Pt_full, sf, xe, ms, j0, width)
                 l += Pt.sum(axis=1) / p_unit
                 acc += (Pt @ v[b, h, cols]) / p_unit
             ok = l > 0
             ls = np.where(ok, l, 1.0)
             O[b, h] = np.where(ok[:, None], acc / ls[:, None], 0.0)
             LSE[b, h] = np.where(ok, LN2 * (np.where(ok, m, 0.0) + np.log2(ls)), -np.inf)
-            if with_flip_bound:
-                flips += int(np.count_nonzero(wflip))
-                FB[b, h] = (wflip @ np.abs(v[b, h]) + wflip.sum(axis=1)[:, None] * np.abs(O[b, h])) / ls[:, None]
-                LB[b, h] = wflip.sum(axis=1) / ls * 1.01
-    if with_flip_bound:
-        return O, LSE, FB, LB, flips
+            if outcomes:
+                rng.add(b, h, rec, acc, l, m, v[b, h] / p_unit, 1.0 / p_unit)
+    if outcomes:
+        return O, LSE, rng.result(O, LSE)
     return O, LSE
+
+
+def _qae_codes(p, s):
+    """Rows of 16 fp32 probabilities p [R, 16] against scales s [R]: the ratio
+    p / s (fp32 divide, zero where s = 0), its e2m1 magnitude and the
+    dequantised value (magnitude * s)."""
+    s32 = np.asarray(s, dtype=F32)
+    safe = np.where(s32 > 0, s32, F32(1.0)).astype(F32)
+    r = np.where((s32 > 0)[:, None], (p.astype(F32) / safe[:, None]).astype(F32), F32(0.0)).astype(np.float64)
+    mag = np.abs(e2m1_decode(e2m1_encode(r)))
+    return mag * np.asarray(s, dtype=np.float64)[:, None], r, mag
+
+
+def _qae_flips(rec, pp, Pt_full, sf, xe, ms, j0, width):
+    """Flagged variables of one key block under quantise-after-exp.
+
+    pp [R, n16] the block's fp32 probabilities (zero padded to 16-key groups),
+    Pt_full their oracle values, sf the oracle's e4m3 scale codes [R, n16/16],
+    xe the scores (0 where masked or padded), ms the row reference max.  A
+    16-key group whose amax / 6 lies within evaluation error of an e4m3
+    midpoint becomes one variable whose options are the other scale's codes
+    and every admissible rounding of the codes under either scale; otherwise
+    each code whose p / sf lies near an e2m1 midpoint is one binary variable."""
+    R, n = pp.shape
+    s_all = ue4m3_decode(sf)                               # [R, n/16]
+    for g in range(n // 16):
+        c0, c1 = g * 16, min(width, g * 16 + 16)
+        if c1 <= c0:
+            continue
+        nkeep = c1 - c0
+        p = pp[:, c0:c0 + 16]
+        xg = xe[:, c0:c0 + 16]
+        base = Pt_full[:, c0:c0 + 16]
+        s = s_all[:, g]
+        a = (p.max(axis=1).astype(F32) / F32(6.0)).astype(np.float64)
+        sflag, s_alt = near_midpoint(a, UE4M3_VALUES, s, eval_band(a, np.abs(xg).max(axis=1), ms, 1e-12))
+        _, ratio, mag = _qae_codes(p, s)
+        cflag, calt = near_midpoint(ratio, E2M1_VALUES, mag, eval_band(ratio, xg, ms[:, None], 1e-12))
+        cflag &= p > 0
+        keys = np.arange(j0 + c0, j0 + c1)
+        for r in np.flatnonzero(sflag | cflag[:, :nkeep].any(axis=1)):
+            s_r = s[r]
+            if sflag[r]:
+                opts = []
+                if cflag[r].any():
+                    opts.append(subset_options(base[r], calt[r] * s_r, cflag[r]))
+                va, ra, ma = _qae_codes(p[r:r + 1], s_alt[r:r + 1])
+                aflag, aalt = near_midpoint(ra[0], E2M1_VALUES, ma[0], eval_band(ra[0], xg[r], ms[r], 1e-12))
+                aflag &= p[r] > 0
+                opts.append((va[0] - base[r])[None, :])
+                if aflag.any():
+                    opts.append(subset_options(va[0], aalt * s_alt[r], aflag) + (va[0] - base[r])[None, :])
+                rec.add_group(r, keys, np.vstack(opts)[:, :nkeep], ms[r])
+            else:
+                js = np.flatnonzero(cflag[r, :nkeep])
+                rec.add_elements(np.full(js.size, r), keys[js], (calt[r] * s_r - base[r])[js],
+                                 np.full(js.size, ms[r]))

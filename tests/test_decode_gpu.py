@@ -1,9 +1,11 @@
-"""GPU parity of attn_decode (split-KV + combine) against the fp64 oracle."""
+"""GPU parity of attn_decode (split-KV + combine) against the fp64 oracle.
+O, LSE and the split workspace sit between guard bands (tests._guard)."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import attention as A
+from tests import _guard as G
 from tests._parity import assert_bf16_close
 from workloads import WORKLOADS, make_qkv
 
@@ -16,7 +18,7 @@ pytestmark = pytest.mark.gpu
 def test_decode_small(cuda_lib, d, Nkv, splits):
     q, k, v = make_qkv("decode", seed=2, B=2, H=3, Nq=1, Nkv=Nkv, d=d)
     scale = d ** -0.5
-    o, lse = cuda_lib.decode(q.cuda(), k.cuda(), v.cuda(), scale, splits)
+    o, lse = G.decode(cuda_lib, q.cuda(), k.cuda(), v.cuda(), scale, splits)
     assert cuda_lib.attn_check_status() == 0
     O, L = A.decode(q, k, v, scale)
     assert_bf16_close(o, lse, O, L, f"decode Nkv={Nkv} splits={splits}")
@@ -34,7 +36,7 @@ def test_split_count_does_not_change_the_result_beyond_rounding(cuda_lib):
 def test_full_decode_workload_sampled_heads(cuda_lib):
     w = WORKLOADS["decode"]
     q, k, v = make_qkv(w, seed=0, device="cuda")
-    o, lse = cuda_lib.decode(q, k, v, w.scale, w.num_splits)
+    o, lse = G.decode(cuda_lib, q, k, v, w.scale, w.num_splits)
     assert cuda_lib.attn_check_status() == 0
     g = np.random.default_rng(0)
     for b, h in [(0, 0), (w.B - 1, w.H - 1)] + [tuple(x) for x in g.integers(0, [w.B, w.H], size=(10, 2))]:

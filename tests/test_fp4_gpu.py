@@ -5,8 +5,16 @@
 * block-scaled FP4 GEMM: S = deq(Q) deq(K)^T against the exact fp64 product
   of the dequantised operands (fp32 accumulation);
 * forward, Direct-P and quantise-after-exp: within 5e-3 max-abs of the
-  oracle's step-by-step FP4 emulation, plus the oracle's bound for P elements
-  that sit within fp32 evaluation error of a rounding boundary (reported).
+  oracle's step-by-step FP4 emulation.  A P element within fp32 evaluation
+  error of an e2m1 rounding midpoint (or, for quantise-after-exp, a block
+  scale amax / 6 that close to an e4m3 midpoint) may round either way on the
+  device; the oracle gives the interval of outputs over every such choice
+  (``oracle.outcomes``) and the device must lie within 5e-3 of it.  Flagged
+  rows and elements are reported and bounded.
+
+Every output, including the padded, transposed V codes and the tiled scale
+layouts, sits between guard bands that must survive the call
+(``tests._guard``).
 """
 import numpy as np
 import pytest
@@ -14,11 +22,11 @@ import torch
 
 from oracle import attention as A
 from oracle import lowp as Q
+from tests import _guard as G
+from tests._parity import assert_within_outcomes, visible_scores
 from workloads import WORKLOADS, make_qkv
 
 pytestmark = pytest.mark.gpu
-O_ABS = 5e-3
-LSE_ABS = 1e-3
 
 
 def _np(t):
@@ -49,7 +57,7 @@ def test_nvfp4_quantiser_bit_exact(cuda_lib, name, N):
     q, _, v = make_qkv(name, seed=3, B=1, H=2, Nq=N, Nkv=N, d=128)
     q[0, 0, 0] = 0
     BH, T = 2, (N + 127) // 128
-    codes, sf = cuda_lib.quantize_nvfp4(q.cuda(), 0)
+    codes, sf = G.quantize_nvfp4(cuda_lib, q.cuda(), 0)
     assert cuda_lib.attn_check_status() == 0
     rc, rs = Q.quantize_nvfp4(q, axis=-1)
     got_c = unpack_codes(codes, (BH, N, 128)).reshape(1, 2, N, 128)
@@ -58,7 +66,7 @@ def test_nvfp4_quantiser_bit_exact(cuda_lib, name, N):
     assert np.array_equal(got_s, rs)
     assert (untile_sf(sf, BH, T)[:, N:] == 0).all()
     # V: blocks along tokens, transposed codes; the oracle sees the zero padding
-    vc, vs = cuda_lib.quantize_nvfp4(v.cuda(), 1)
+    vc, vs = G.quantize_nvfp4(cuda_lib, v.cuda(), 1)
     Np = T * 128
     vpad = torch.zeros(1, 2, Np, 128, dtype=torch.bfloat16)
     vpad[:, :, :N] = v
@@ -88,11 +96,13 @@ def _deq_inputs(q, k, v):
 @pytest.mark.parametrize("Nq,Nkv", [(128, 128), (200, 300), (1, 1), (513, 129)])
 def test_fp4_block_scaled_scores(cuda_lib, Nq, Nkv):
     q, k, _ = make_qkv("lowp", seed=Nq + Nkv, B=1, H=2, Nq=Nq, Nkv=Nkv, d=128)
-    qc, qs = cuda_lib.quantize_nvfp4(q.cuda(), 0)
-    kc, ks = cuda_lib.quantize_nvfp4(k.cuda(), 0)
-    s = torch.empty((1, 2, Nq, Nkv), dtype=torch.float32, device="cuda")
+    qc, qs = G.quantize_nvfp4(cuda_lib, q.cuda(), 0)
+    kc, ks = G.quantize_nvfp4(cuda_lib, k.cuda(), 0)
+    sg = G.Guarded((1, 2, Nq, Nkv), torch.float32)
+    s = sg.t
     cuda_lib.attn_fp4_scores(qc, qs, kc, ks, s, 1, 2, Nq, Nkv)
     assert cuda_lib.attn_check_status() == 0
+    sg.check("attn_fp4_scores")
     qd, kd, _ = _deq_inputs(q, k, k[:, :, :1])
     ref = np.einsum("bhid,bhjd->bhij", qd, kd)
     got = _np(s).astype(np.float64)
@@ -101,26 +111,22 @@ def test_fp4_block_scaled_scores(cuda_lib, Nq, Nkv):
 
 def _check_fp4(ta, q, k, v, causal, scale, mode, rows=None, what=""):
     B, H, Nq, d = q.shape
-    o, lse = ta.forward_fp4(q.cuda(), k.cuda(), v.cuda(), causal, scale, mode)
+    o, lse = G.forward_fp4(ta, q.cuda(), k.cuda(), v.cuda(), causal, scale, mode, what)
     assert ta.attn_check_status() == 0
     qd, kd, vd = _deq_inputs(q, k, v)
     if rows is not None:
         qd = qd[:, :, rows]
         if causal:
             raise ValueError("row sampling is for non-causal runs")
-    O, L, FB, LB, flips = Q.attention_fp4(qd, kd, vd, mode, causal, scale, with_flip_bound=True)
+    O, L, R = Q.attention_fp4(qd, kd, vd, mode, causal, scale, outcomes=True)
     og, lg = _np(o).astype(np.float64), _np(lse).astype(np.float64)
     if rows is not None:
         og, lg = og[:, :, rows], lg[:, :, rows]
-    assert np.isfinite(og).all()
-    err = np.abs(og - O)
-    assert (err <= O_ABS + FB).all(), f"{what}: O err {err.max():.3e} (beyond bound {(err - FB).max():.3e}), flips {flips}"
-    fin = np.isfinite(L)
-    assert np.isneginf(lg[~fin]).all()
-    assert (np.abs(lg[fin] - L[fin]) <= LSE_ABS + LB[fin]).all(), what
+    n_scores = B * H * visible_scores(Nq, k.shape[2], causal, rows)
+    err, _ = assert_within_outcomes(og, lg, O, L, R, what, n_scores)
     Oe, _ = A.attention(q, k, v, causal, scale, rows=rows)
     cos = float((og * Oe).sum() / (np.linalg.norm(og) * np.linalg.norm(Oe) + 1e-300))
-    return float(err.max()), flips, cos
+    return err, R.flips, cos
 
 
 @pytest.mark.parametrize("mode", [0, 1], ids=["direct_p", "quant_after_exp"])
@@ -151,7 +157,7 @@ def test_fp4_full_lowp_workload_sampled_rows(cuda_lib, mode):
     same operands)."""
     w = WORKLOADS["lowp"]
     q, k, v = make_qkv(w, seed=0)
-    o, lse = cuda_lib.forward_fp4(q.cuda(), k.cuda(), v.cuda(), False, w.scale, mode)
+    o, lse = G.forward_fp4(cuda_lib, q.cuda(), k.cuda(), v.cuda(), False, w.scale, mode, "fp4 lowp full")
     assert cuda_lib.attn_check_status() == 0
     og, lg = _np(o).astype(np.float64), _np(lse).astype(np.float64)
     assert np.isfinite(og).all() and np.isfinite(lg).all()
@@ -159,7 +165,6 @@ def test_fp4_full_lowp_workload_sampled_rows(cuda_lib, mode):
     for b, h in [(0, 0), (1, 23), (0, 11)]:
         sl = (slice(b, b + 1), slice(h, h + 1))
         qd, kd, vd = _deq_inputs(q[sl], k[sl], v[sl])
-        O, L, FB, LB, flips = Q.attention_fp4(qd[:, :, rows], kd, vd, mode, False, w.scale, with_flip_bound=True)
-        err = np.abs(og[b:b + 1, h:h + 1, rows] - O)
-        assert (err <= O_ABS + FB).all(), f"b={b} h={h}: {err.max():.3e}, flips {flips}"
-        assert (np.abs(lg[b:b + 1, h:h + 1, rows] - L) <= LSE_ABS + LB).all()
+        O, L, R = Q.attention_fp4(qd[:, :, rows], kd, vd, mode, False, w.scale, outcomes=True)
+        assert_within_outcomes(og[b:b + 1, h:h + 1, rows], lg[b:b + 1, h:h + 1, rows], O, L, R,
+                               f"fp4 mode {mode} lowp full b={b} h={h}", rows.size * w.Nkv)

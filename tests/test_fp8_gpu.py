@@ -4,9 +4,15 @@ oracle, through the C ABI.
 * quantisers (rotation by the fast Walsh-Hadamard transform, per-row and
   per-channel e4m3): bit-exact codes and fp32 scales;
 * forward: within 5e-3 max-abs of the oracle's step-by-step FP8 emulation
-  (lazy rescale threshold 8, as the kernel) plus,
-  for rows where a P element sat within fp32 evaluation error of an e4m3
-  rounding midpoint, the oracle's bound on what that rounding can change.
+  (lazy rescale threshold 8, as the kernel).  A P element within fp32
+  evaluation error of an e4m3 rounding midpoint, or a rescale decision that
+  close to the threshold, may go either way on the device; the oracle gives
+  the interval of outputs over every such choice (``oracle.outcomes``) and
+  the device must lie within 5e-3 of it.  Flagged rows and elements are
+  reported and bounded.
+
+Every output sits between guard bands that must survive the call
+(``tests._guard``).
 """
 import numpy as np
 import pytest
@@ -14,11 +20,11 @@ import torch
 
 from oracle import attention as A
 from oracle import fp8 as F
+from tests import _guard as G
+from tests._parity import assert_within_outcomes, visible_scores
 from workloads import WORKLOADS, make_qkv, rotation_signs
 
 pytestmark = pytest.mark.gpu
-O_ABS = 5e-3
-LSE_ABS = 1e-3
 
 
 def _np(t):
@@ -40,7 +46,7 @@ def test_fp8_row_quantiser_bit_exact(cuda_lib, name, rotate, d):
     q, _, v = make_qkv(name, seed=5, B=2, H=3, Nq=257, Nkv=130, d=d)
     q[0, 1, 7] = 0                                    # an all-zero row
     signs = rotation_signs(d, 3) if rotate else None
-    codes, sc = cuda_lib.quantize_fp8(q.cuda(), 0, None if signs is None else signs.cuda())
+    codes, sc = G.quantize_fp8(cuda_lib, q.cuda(), 0, None if signs is None else signs.cuda())
     assert cuda_lib.attn_check_status() == 0
     rv, rs = F.quantize_fp8_rows(q, None if signs is None else signs.numpy())
     assert np.array_equal(_np(sc), rs)
@@ -51,7 +57,7 @@ def test_fp8_row_quantiser_bit_exact(cuda_lib, name, rotate, d):
 def test_fp8_channel_quantiser_bit_exact(cuda_lib, d):
     _, _, v = make_qkv("lowp", seed=6, B=2, H=3, Nq=1, Nkv=333, d=d)
     v[1, 2, :, 5] = 0                                 # an all-zero channel
-    codes, sc = cuda_lib.quantize_fp8(v.cuda(), 1)
+    codes, sc = G.quantize_fp8(cuda_lib, v.cuda(), 1)
     assert cuda_lib.attn_check_status() == 0
     rv, rs = F.quantize_fp8_channels(v)
     assert np.array_equal(_np(sc), rs)
@@ -64,33 +70,26 @@ def _check_fp8(ta, q, k, v, causal, scale, rotate, rows=None, what="", seed=0):
     d = q.shape[-1]
     signs = rotation_signs(d, seed) if rotate else None
     sg = None if signs is None else signs.cuda()
-    qc, qs = ta.quantize_fp8(q.cuda(), 0, sg)
-    kc, ks = ta.quantize_fp8(k.cuda(), 0, sg)
-    vc, vs = ta.quantize_fp8(v.cuda(), 1)
+    qc, qs = G.quantize_fp8(ta, q.cuda(), 0, sg)
+    kc, ks = G.quantize_fp8(ta, k.cuda(), 0, sg)
+    vc, vs = G.quantize_fp8(ta, v.cuda(), 1)
     B, H, Nq, _ = q.shape
-    o = torch.empty((B, H, Nq, d), dtype=torch.float32, device="cuda")
-    lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
-    ta.attn_fwd_fp8(qc, qs, kc, ks, vc, vs, o, lse, causal, scale, rotate)
+    o, lse = G.fwd_fp8(ta, qc, qs, kc, ks, vc, vs, causal, scale, rotate, what)
     assert ta.attn_check_status() == 0
     sn = None if signs is None else signs.numpy()
     rqv, rqs = F.quantize_fp8_rows(q, sn)
     rkv, rks = F.quantize_fp8_rows(k, sn)
     rvv, rvs = F.quantize_fp8_channels(v)
-    O, L, FB, LB, flips = F.attention_fp8(rqv, rqs, rkv, rks, rvv, rvs, causal, scale,
-                                          rot_d=d if rotate else 1, with_flip_bound=True, rows=rows,
-                                          tau=8.0)
+    O, L, R = F.attention_fp8(rqv, rqs, rkv, rks, rvv, rvs, causal, scale,
+                              rot_d=d if rotate else 1, outcomes=True, rows=rows, tau=8.0)
     og, lg = _np(o).astype(np.float64), _np(lse).astype(np.float64)
     if rows is not None:
         og, lg = og[:, :, rows], lg[:, :, rows]
-    assert np.isfinite(og).all()
-    err = np.abs(og - O)
-    assert (err <= O_ABS + FB).all(), f"{what}: O err {err.max():.3e}, flips {flips}"
-    fin = np.isfinite(L)
-    assert (np.isneginf(lg[~fin])).all()
-    assert (np.abs(lg[fin] - L[fin]) <= LSE_ABS + LB[fin]).all(), what
+    n_scores = B * H * visible_scores(Nq, k.shape[2], causal, rows)
+    err, _ = assert_within_outcomes(og, lg, O, L, R, what, n_scores)
     Oe, _ = A.attention(q, k, v, causal, scale, rows=rows)
     cos = float((og * Oe).sum() / (np.linalg.norm(og) * np.linalg.norm(Oe) + 1e-300))
-    return float(err.max()), flips, cos
+    return err, R.flips, cos
 
 
 @pytest.mark.parametrize("rotate", [False, True])

@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 
 from oracle import attention as A
+from tests import _guard as G
 from tests._parity import assert_bf16_close
 from workloads import WORKLOADS, make_qkv
 
@@ -24,7 +25,7 @@ def gqa_inputs(name, seed, B, Hq, Hkv, Nq, Nkv, d, device="cpu"):
 def test_fwd_gqa(cuda_lib, shape, causal):
     B, Hq, Hkv, Nq, Nkv, d = shape
     q, k, v = gqa_inputs("prefill", 31, B, Hq, Hkv, Nq, Nkv, d)
-    o, lse = cuda_lib.forward(q.cuda(), k.cuda(), v.cuda(), causal, d ** -0.5)
+    o, lse = G.forward(cuda_lib, q.cuda(), k.cuda(), v.cuda(), causal, d ** -0.5)
     assert cuda_lib.attn_check_status() == 0
     O, L = A.attention_gqa(q, k, v, causal, d ** -0.5)
     assert_bf16_close(o, lse, O, L, f"gqa {shape} causal={causal}")
@@ -49,7 +50,7 @@ def test_fwd_gqa_equals_expanded_heads(cuda_lib):
 def test_decode_gqa(cuda_lib, shape):
     B, Hq, Hkv, Nkv, d, splits = shape
     q, k, v = gqa_inputs("decode", 8, B, Hq, Hkv, 1, Nkv, d)
-    o, lse = cuda_lib.decode(q.cuda(), k.cuda(), v.cuda(), d ** -0.5, splits)
+    o, lse = G.decode(cuda_lib, q.cuda(), k.cuda(), v.cuda(), d ** -0.5, splits)
     assert cuda_lib.attn_check_status() == 0
     O, L = A.attention_gqa(q, k, v, False, d ** -0.5)
     assert_bf16_close(o, lse, O, L, f"decode gqa {shape}")
@@ -61,7 +62,7 @@ def test_decode_gqa_full_size_sampled_heads(cuda_lib):
     checks sampled (batch, head) pairs."""
     w = WORKLOADS["decode"]
     q, k, v = gqa_inputs(w, 0, w.B, w.H, w.H // 4, 1, w.Nkv, w.d, device="cuda")
-    o, lse = cuda_lib.decode(q, k, v, w.scale, w.num_splits)
+    o, lse = G.decode(cuda_lib, q, k, v, w.scale, w.num_splits)
     assert cuda_lib.attn_check_status() == 0
     g = np.random.default_rng(3)
     for b, h in [(0, 0), (w.B - 1, w.H - 1)] + [tuple(x) for x in g.integers(0, [w.B, w.H], size=(8, 2))]:

@@ -1,11 +1,15 @@
 """GPU parity of the variable-length (packed) forward and of decode with a
 cache length per batch entry against the fp64 oracle, through the C ABI.  Same
-tolerances as the bf16 path (max-abs 2e-2, mean-abs 2e-3 on O, 1e-3 on LSE)."""
+tolerances as the bf16 path (max-abs 2e-2, mean-abs 2e-3 on O, 1e-3 on LSE).
+Outputs and workspaces sit between guard bands (tests._guard): the varlen
+epilogue stores rows directly, so a row past its sequence would land in the
+next sequence's rows or past the packed tensor."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import attention as A
+from tests import _guard as G
 from tests._parity import assert_bf16_close
 from workloads import make_qkv, make_varlen
 
@@ -21,7 +25,7 @@ MIXES = {
 
 def _run(ta, lq, lk, H, Hkv, d, causal, seed=0):
     q, k, v, cu_q, cu_k = make_varlen(lq, lk, H, Hkv, d, seed)
-    o, lse = ta.forward_varlen(q.cuda(), k.cuda(), v.cuda(), cu_q.cuda(), cu_k.cuda(), max(lq), causal, d ** -0.5)
+    o, lse = G.forward_varlen(ta, q.cuda(), k.cuda(), v.cuda(), cu_q.cuda(), cu_k.cuda(), max(lq), causal, d ** -0.5)
     assert ta.attn_check_status() == 0
     O, L = A.attention_varlen(q, k, v, cu_q.numpy(), cu_k.numpy(), causal, d ** -0.5)
     return o, lse, O, L, (q, k, v, cu_q, cu_k)
@@ -70,7 +74,7 @@ def test_decode_varlen(cuda_lib, d, Hkv):
     q, k, v = make_qkv("decode", seed=8, B=B, H=H, Nkv=N, d=d)
     k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
     lens = torch.tensor([3000, 0, 1, 1234, 129], dtype=torch.int32)
-    o, lse = cuda_lib.decode_varlen(q.cuda(), k.cuda(), v.cuda(), lens.cuda(), d ** -0.5, num_splits=16)
+    o, lse = G.decode_varlen(cuda_lib, q.cuda(), k.cuda(), v.cuda(), lens.cuda(), d ** -0.5, 16)
     assert cuda_lib.attn_check_status() == 0
     O, L = A.decode_varlen(q, k, v, lens.numpy(), d ** -0.5)
     assert_bf16_close(o, lse, O, L, f"decode varlen d={d} Hkv={Hkv}")

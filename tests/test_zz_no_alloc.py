@@ -4,11 +4,13 @@ plug-ins without an allocator, paths that must never enter the driver's
 allocator).  It keeps its split partials in a fixed array inside the library
 instead of a caller-provided workspace.
 
-Checked through the C ABI against attn_decode (the entry point with a
-workspace) on two calls in a row with different inputs and shapes -- the
-second call must not see anything the first one left in the shared array --
-within the tolerances the other parity tests use.  Also checks that a
-request too large for the fixed array is refused before anything runs.
+Checked through the C ABI on calls in a row with different inputs and shapes
+(the later calls must not see anything an earlier one left in the shared
+array): each result is bit-identical to attn_decode (the entry point with a
+workspace, which runs the same kernels with the same splits) and within the
+bf16 tolerances of the fp64 oracle's decode.  One call uses more splits than
+there are keys, so some chunks are empty.  Also checks that a request too
+large for the fixed array is refused before anything runs.
 
 This file is collected last on purpose (name), so a run that stops at the
 first failure has already run every other test.
@@ -18,7 +20,8 @@ import ctypes
 import pytest
 import torch
 
-from tests._parity import LSE_ABS, O_MAX_ABS
+from oracle import attention as A
+from tests._parity import assert_bf16_close
 from workloads import make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -35,18 +38,23 @@ def _noalloc(lib, q, k, v, scale, splits):
     return rc, o, lse
 
 
-def test_noalloc_decode_matches_workspace_decode_twice(cuda_lib):
+def test_noalloc_decode_matches_workspace_decode_and_oracle(cuda_lib):
     lib = cuda_lib.load()
-    cases = [(8, 16, 3000, 128, 16, 31), (3, 5, 777, 64, 7, 32)]
+    # (B, H, Nkv, d, splits, seed): the largest first, then smaller ones that
+    # reuse the front of the array; the third has 16 splits over 5 keys
+    cases = [(8, 16, 3000, 128, 16, 31), (3, 5, 777, 64, 7, 32), (2, 3, 5, 128, 16, 33)]
     for B, H, Nkv, d, splits, seed in cases:
-        q, k, v = (t.cuda() for t in make_qkv("decode", seed=seed, B=B, H=H, Nq=1, Nkv=Nkv, d=d))
+        qc, kc, vc = make_qkv("decode", seed=seed, B=B, H=H, Nq=1, Nkv=Nkv, d=d)
+        q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
         scale = d ** -0.5
         o_ref, lse_ref = cuda_lib.decode(q, k, v, scale, splits)
         rc, o, lse = _noalloc(lib, q, k, v, scale, splits)
         assert rc == 0, cuda_lib.attn_status_string(rc)
         assert cuda_lib.attn_check_status() == 0
-        assert (o.float() - o_ref.float()).abs().max().item() <= O_MAX_ABS
-        assert (lse - lse_ref).abs().max().item() <= LSE_ABS
+        what = f"noalloc B={B} H={H} Nkv={Nkv} d={d} splits={splits}"
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), what
+        O, L = A.decode(qc, kc, vc, scale)
+        assert_bf16_close(o, lse, O, L, what)
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch(cuda_lib):
