@@ -18,11 +18,12 @@ A step is one pass of the hot path over the seeded synthetic workloads:
              quantisers + INT8 forward, NVFP4 quantisers + FP4 forward with
              Direct-P and with quantise-after-exp, FP8 quantisers (Hadamard
              rotation of Q, K) + FP8 forward.
-Inputs are resident in HBM before timing starts and are larger than the
-126 MB L2 (prefill Q+K+V = 201 MB, decode K+V = 8.6 GB), so no L2 flush is
-needed between steps.  Every launch is bracketed by CUDA events on the
-launching stream; `value` is prefill FLOPs / summed prefill kernel time and
-`parts` gives every segment's rate against its roofline.
+Inputs are resident in HBM before timing starts; before every launch 256 MB
+are written to flush the 126 MB L2 (outside the launch's own CUDA events, on
+the launching stream).  `value` is prefill FLOPs / summed prefill kernel time
+and `parts` gives every segment's rate against its roofline.  The INT8, FP8
+and FP4 peaks are the measured bf16 peak times the measured ratio of this
+GPU's tcgen05 MMA rates (libtiledattn_probe).
 
 `e2e` measures the same metric through the public API with host buffers:
 each step copies Q, K, V from pinned host memory, runs both forwards and
@@ -63,6 +64,23 @@ def load_peaks():
         return p, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def measure_peaks(dev):
+    """Tensor-core ceilings per MMA kind and MUFU exponential rates, measured
+    on this GPU by libtiledattn_probe (one CTA per SM, SM cycles from the
+    kernels' own clock and TFLOP/s from CUDA events).  Rates are taken at
+    N = 128, the MMA shape the attention kernels issue, and at N = 256."""
+    from tiled_attention_24_b200 import _probe
+    mma = {}
+    for kind in ("bf16", "int8", "fp8", "fp4"):
+        mma[kind] = _probe.mma_rate(kind, 128, device=dev)
+        if kind != "fp4":
+            mma[kind + "_n256"] = _probe.mma_rate(kind, 256, device=dev)
+    mufu = {f"ex2_{t}threads": _probe.ex2_rate(t, 8, device=dev)["ex2_per_clk_sm"] for t in (1024, 256, 128)}
+    mufu["ex2_256threads_ilp1"] = _probe.ex2_rate(256, 1, device=dev)["ex2_per_clk_sm"]
+    mufu["softmax_scores_per_clk_sm_256threads"] = _probe.softmax_rate(256, device=dev)["scores_per_clk_sm"]
+    return {"mma": mma, "mufu": mufu}
 
 
 def dist_env():
@@ -176,6 +194,209 @@ def oracle_sample(seconds_cap: float = 30.0):
     return flops / dt / 1e12, desc, cpu_threads(), dt
 
 
+def _cos(a, b):
+    a, b = a.ravel(), b.ravel()
+    return float((a * b).sum() / (math.sqrt(float((a * a).sum()) * float((b * b).sum())) + 1e-300))
+
+
+def oracle_leg(ta, dev, stream, D, rows_per_head=16):
+    """The fp64 oracle (test infrastructure) as the CPU baseline and as the
+    accuracy reference of every configuration and path, on a bounded sample:
+    a few (batch, head) slices and ``rows_per_head`` query rows of each (the
+    oracle's cost is linear in the rows, so its rate on the sample is its rate
+    on the full workload).  Each part's device outputs for those rows come
+    from a fresh launch.  Returns (per-config oracle rates, per-part accuracy).
+
+    Accuracy: max-abs / mean-abs against the oracle (bf16 paths: the plain
+    definition; quantised paths: the step-by-step emulation, with the distance
+    outside the interval of admissible roundings), and the cosine similarity
+    of the sampled outputs with the unquantised fp64 attention."""
+    import numpy as np
+
+    from oracle import attention as A  # test infrastructure: CPU baseline / accuracy leg only
+    from oracle import fp8 as F
+    from oracle import lowp as Q
+    rng = np.random.default_rng(0)
+    cpu, acc = {}, {}
+
+    def rows_of(n):
+        r = set(rng.choice(n, size=min(n, rows_per_head - 3), replace=False).tolist()) | {0, n // 2, n - 1}
+        return np.array(sorted(r))
+
+    def host(t, b, h, rows):
+        return t[b:b + 1, h:h + 1][:, :, rows].double().cpu().numpy()
+
+    def time_oracle(fn):
+        t0 = time.perf_counter()
+        out = fn()
+        return out, time.perf_counter() - t0
+
+    def bf16_part(name, wl, q, k, v, o, lse, causal, run, heads, unit_rate=True):
+        run()
+        torch.cuda.synchronize()
+        errs, worst, flops, secs, cos = [], 0.0, 0.0, 0.0, []
+        for b, h in heads:
+            rows = rows_of(wl.Nq)
+            qs, ks, vs = (t[b:b + 1, h:h + 1].cpu() for t in (q, k, v))
+            (O, L), dt = time_oracle(lambda: A.attention(qs, ks, vs, causal, wl.scale, rows=rows))
+            secs += dt
+            vis = A.visible_mask(wl.Nq, wl.Nkv, causal, rows).sum()
+            flops += 4.0 * vis * wl.d
+            og = host(o, b, h, rows)
+            e = np.abs(og - O)
+            errs.append(e)
+            fin = np.isfinite(L)
+            lg = host(lse, b, h, rows)
+            worst = max(worst, float(np.abs(lg[fin] - L[fin]).max(initial=0.0)))
+            cos.append(_cos(og, O))
+        e = np.concatenate([x.ravel() for x in errs])
+        acc[name] = {"vs": "fp64 definition", "max_abs": float(e.max()), "mean_abs": float(e.mean()),
+                     "lse_max_abs": worst, "cos_fp64": min(cos), "rows": int(sum(x.shape[2] for x in errs))}
+        return flops / secs / 1e12, secs
+
+    t_all = time.perf_counter()
+    if "prefill" in D:
+        q, k, v, o, lse = D["prefill"]
+        wp = WORKLOADS["prefill"]
+        for causal in (False, True):
+            nm = "prefill_causal" if causal else "prefill_noncausal"
+            r, dt = bf16_part(nm, wp, q, k, v, o, lse, causal,
+                              lambda c=causal: ta.attn_fwd(q, k, v, o, lse, c, wp.scale, stream), [(0, 0), (3, 15)])
+            cpu[nm] = {"value": r, "unit": "TFLOP/s", "seconds": dt}
+    if "tiny" in D:
+        q, k, v, o, lse = D["tiny"]
+        wt = WORKLOADS["tiny"]
+        for causal in (False, True):
+            nm = "tiny_causal" if causal else "tiny_noncausal"
+            r, dt = bf16_part(nm, wt, q, k, v, o, lse, causal,
+                              lambda c=causal: ta.attn_fwd(q, k, v, o, lse, c, wt.scale, stream), [(0, 0), (0, 1)])
+            cpu[nm] = {"value": r, "unit": "TFLOP/s", "seconds": dt}
+    if "longseq" in D:
+        q, k, v, o, lse = D["longseq"]
+        wl = WORKLOADS["longseq"]
+        for causal in (False, True):
+            nm = "longseq_causal" if causal else "longseq_noncausal"
+            r, dt = bf16_part(nm, wl, q, k, v, o, lse, causal,
+                              lambda c=causal: ta.attn_fwd(q, k, v, o, lse, c, wl.scale, stream), [(0, 0), (0, 11)])
+            cpu[nm] = {"value": r, "unit": "TFLOP/s", "seconds": dt}
+    if "decode" in D:
+        dq, dk, dv, do, dlse, dws, gk, gv = D["decode"]
+        wd = WORKLOADS["decode"]
+        for nm, kk, vv, grp in (("decode", dk, dv, 1), ("decode_gqa", gk, gv, wd.H // gk.shape[1])):
+            (ta.attn_decode if grp == 1 else ta.attn_decode_gqa)(dq, kk, vv, do, dlse, wd.scale, wd.num_splits,
+                                                                 dws, stream)
+            torch.cuda.synchronize()
+            errs, secs, nbytes, worst = [], 0.0, 0.0, 0.0
+            for b, h in [(0, 0), (dq.shape[0] - 1, wd.H - 1), (7, 5), (33, 18)]:
+                kh = h // grp
+                args_ = [t[b:b + 1, hh:hh + 1].cpu() for t, hh in ((dq, h), (kk, kh), (vv, kh))]
+                (O, L), dt = time_oracle(lambda: A.decode(*args_, wd.scale))
+                secs += dt
+                nbytes += 2 * args_[1].numel() * 2
+                e = np.abs(do[b:b + 1, h:h + 1].double().cpu().numpy() - O)
+                errs.append(e)
+                worst = max(worst, float(np.abs(dlse[b:b + 1, h:h + 1].double().cpu().numpy() - L).max()))
+            e = np.concatenate([x.ravel() for x in errs])
+            acc[nm] = {"vs": "fp64 definition", "max_abs": float(e.max()), "mean_abs": float(e.mean()),
+                       "lse_max_abs": worst, "rows": len(errs)}
+            cpu[nm] = {"value": nbytes / secs / 1e9, "unit": "GB/s", "seconds": secs}
+    if "varlen" in D:
+        vq, vk, vv, vo, vlse, vcu, lens = D["varlen"]
+        wp = WORKLOADS["prefill"]
+        ta.attn_fwd_varlen(vq, vk, vv, vo, vlse, vcu, vcu, max(lens), True, wp.scale, stream)
+        torch.cuda.synchronize()
+        # the first packed sequence (4096 tokens), heads 0 and 9: plain causal attention on its slice
+        n0 = lens[0]
+        errs, secs, flops = [], 0.0, 0.0
+        for h in (0, 9):
+            rows = rows_of(n0)
+            sl = [t[:n0, h].unsqueeze(0).unsqueeze(0).cpu() for t in (vq, vk, vv)]
+            (O, L), dt = time_oracle(lambda: A.attention(*sl, True, wp.scale, rows=rows))
+            secs += dt
+            flops += 4.0 * A.visible_mask(n0, n0, True, rows).sum() * wp.d
+            errs.append(np.abs(vo[:n0, h][rows].double().cpu().numpy() - O[0, 0]))
+        e = np.concatenate([x.ravel() for x in errs])
+        acc["prefill_varlen_causal"] = {"vs": "fp64 definition", "max_abs": float(e.max()),
+                                        "mean_abs": float(e.mean()), "rows": int(sum(x.shape[0] for x in errs))}
+        cpu["prefill_varlen_causal"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "seconds": secs}
+    if "bwd" in D:
+        q, k, v, bo, blse, dout, bdq, bdk, bdv, bws = D["bwd"]
+        wp = WORKLOADS["prefill"]
+        ta.attn_bwd(q, k, v, bo, dout, blse, bdq, bdk, bdv, True, wp.scale, bws, stream)
+        torch.cuda.synchronize()
+        sl = [t[0:1, 0:1].cpu() for t in (q, k, v, dout)]
+        ref, dt = time_oracle(lambda: A.attention_backward(*sl, True, wp.scale))
+        out = {"vs": "fp64 gradients of the definition (one head)"}
+        for nm_, g, r in zip(("dq", "dk", "dv"), (bdq, bdk, bdv), ref):
+            e = np.abs(g[0:1, 0:1].double().cpu().numpy() - r)
+            out[nm_ + "_max_abs_over_ref_max"] = float(e.max() / np.abs(r).max())
+        acc["prefill_bwd_causal"] = out
+        cpu["prefill_bwd_causal"] = {"value": 2.5 * 4.0 * wp.Nq * wp.Nkv * wp.d / 2 / dt / 1e12, "unit": "TFLOP/s",
+                                     "seconds": dt}
+    if "lowp" in D:
+        L_ = D["lowp"]
+        xq, xk, xv, xo, xl = L_["bf16"]
+        wq = WORKLOADS["lowp"]
+        r, dt = bf16_part("lowp_bf16", wq, xq, xk, xv, xo, xl, False,
+                          lambda: ta.attn_fwd(xq, xk, xv, xo, xl, False, wq.scale, stream), [(0, 0), (1, 23)])
+        cpu["lowp_bf16"] = {"value": r, "unit": "TFLOP/s", "seconds": dt}
+        heads = [(0, 0), (1, 23)]
+        samples = {hd: rows_of(wq.Nq) for hd in heads}
+        exact = {}
+        for (b, h), rows in samples.items():
+            sl = [t[b:b + 1, h:h + 1].cpu() for t in (xq, xk, xv)]
+            exact[(b, h)] = (sl, A.attention(*sl, False, wq.scale, rows=rows)[0])
+
+        def quant_part(name, run, o_dev, l_dev, emulate, unit):
+            run()
+            torch.cuda.synchronize()
+            errs, outs, cosv, secs, flops, flagged = [], [], [], 0.0, 0.0, 0
+            for (b, h), rows in samples.items():
+                sl, Oe = exact[(b, h)]
+                (O, L, R), dt = time_oracle(lambda: emulate(sl, rows))
+                secs += dt
+                flops += 4.0 * rows.size * wq.Nkv * wq.d
+                og = host(o_dev, b, h, rows)
+                lg = host(l_dev, b, h, rows)
+                errs.append(np.abs(og - O))
+                outs.append(R.distance(og, lg)[0])
+                flagged += R.flagged_rows
+                cosv.append(_cos(og, Oe))
+            e = np.concatenate([x.ravel() for x in errs])
+            acc[name] = {"vs": "fp64 step-by-step emulation", "max_abs": float(e.max()), "mean_abs": float(e.mean()),
+                         "outside_interval": max(outs), "flagged_rows": flagged,
+                         "rows": int(sum(x.shape[2] for x in errs)), "cos_fp64": min(cosv)}
+            cpu[name] = {"value": flops / secs / 1e12, "unit": unit, "seconds": secs}
+
+        i8, s8, of, lf = L_["int8"]
+
+        def emu_int8(sl, rows):
+            a = Q.quantize_int8_rows(sl[0]), Q.quantize_int8_rows(sl[1]), Q.quantize_int8_heads(sl[2])
+            return Q.attention_int8(*a[0], *a[1], *a[2], False, wq.scale, outcomes=True, rows=rows)
+        quant_part("lowp_int8", lambda: ta.attn_fwd_int8(i8[0], s8[0], i8[1], s8[1], i8[2], s8[2], of, lf, False,
+                                                          wq.scale, stream), of, lf, emu_int8, "TOPS")
+        c4, f4 = L_["fp4"]
+        for mode, nm in ((0, "lowp_fp4_direct_p"), (1, "lowp_fp4_quant_after_exp")):
+            def emu_fp4(sl, rows, mode=mode):
+                qd = Q.nvfp4_dequantize(*Q.quantize_nvfp4(sl[0], axis=-1), axis=-1)[:, :, rows]
+                kd = Q.nvfp4_dequantize(*Q.quantize_nvfp4(sl[1], axis=-1), axis=-1)
+                vd = Q.nvfp4_dequantize(*Q.quantize_nvfp4(sl[2], axis=-2), axis=-2)
+                return Q.attention_fp4(qd, kd, vd, mode, False, wq.scale, outcomes=True)
+            quant_part(nm, lambda mode=mode: ta.attn_fwd_fp4(c4[0], f4[0], c4[1], f4[1], c4[2], f4[2], of, lf,
+                                                             *xq.shape[:3], xk.shape[2], False, wq.scale, mode,
+                                                             stream), of, lf, emu_fp4, "TFLOP/s")
+        c8, s8f, signs = L_["fp8"]
+        sn = signs.cpu().numpy()
+
+        def emu_fp8(sl, rows):
+            a = F.quantize_fp8_rows(sl[0], sn), F.quantize_fp8_rows(sl[1], sn), F.quantize_fp8_channels(sl[2])
+            return F.attention_fp8(*a[0], *a[1], *a[2], False, wq.scale, rot_d=wq.d, outcomes=True, rows=rows,
+                                   tau=8.0)
+        quant_part("lowp_fp8", lambda: ta.attn_fwd_fp8(c8[0], s8f[0], c8[1], s8f[1], c8[2], s8f[2], of, lf, False,
+                                                        wq.scale, True, stream), of, lf, emu_fp8, "TFLOP/s")
+    return cpu, acc, time.perf_counter() - t_all
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -222,15 +443,24 @@ def run_ours(args):
     parts = set(args.only.split(","))
     peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    # dense INT8 / FP4 peaks are not in the measured set: nominal (4.5 POPS,
-    # 9 PFLOPS) scaled by measured/nominal bf16 (1683 / 2250), labelled as such
-    ratio = peak_tc / 2250.0
-    peak_i8 = float(peaks.get("int8_tops", 4500.0 * ratio))
-    peak_f4 = float(peaks.get("fp4_tflops", 9000.0 * ratio))
-    peak_f8 = float(peaks.get("fp8_tflops", 4500.0 * ratio))
-    lowp_peak_src = "measured" if "int8_tops" in peaks else "nominal x (measured/nominal bf16)"
+    # INT8 / FP8 / FP4 dense peaks: the measured bf16 GEMM peak times the
+    # measured ratio of this GPU's tcgen05 MMA rates (kind::i8, f8f6f4,
+    # mxf4nvf4 against kind::f16, same 128x128 shape, operands in shared memory)
+    probes = measure_peaks(dev) if not args.no_probe else None
+    if probes:
+        base = probes["mma"]["bf16"]["flop_per_clk_sm"]
+        peak_i8 = peak_tc * probes["mma"]["int8"]["flop_per_clk_sm"] / base
+        peak_f8 = peak_tc * probes["mma"]["fp8"]["flop_per_clk_sm"] / base
+        peak_f4 = peak_tc * probes["mma"]["fp4"]["flop_per_clk_sm"] / base
+        lowp_peak_src = (f"measured: {peak_src} bf16 GEMM peak x this GPU's tcgen05 MMA-rate ratio "
+                         f"(kind vs kind::f16, 128x128, libtiledattn_probe)")
+    else:
+        ratio = peak_tc / 2250.0
+        peak_i8, peak_f8, peak_f4 = 4500.0 * ratio, 4500.0 * ratio, 9000.0 * ratio
+        lowp_peak_src = "nominal x (measured/nominal bf16)"
 
     segs = []   # (name, fn, work, unit, peak, bound, launches)
+    D = {}      # device tensors of every part, for the oracle leg after timing
 
     def seg(name, fn, work, unit, peak, bound, launches):
         segs.append((name, fn, work, unit, peak, bound, launches))
@@ -241,6 +471,11 @@ def run_ours(args):
         q, k, v = (t.to(dev) for t in make_qkv(wp, seed=0))
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        D["prefill"] = (q, k, v, o, lse)
+        wt = WORKLOADS["tiny"]
+        D["tiny"] = tuple(t.to(dev) for t in make_qkv(wt, seed=0)) + (
+            torch.empty((wt.B, wt.H, wt.Nq, wt.d), dtype=torch.bfloat16, device=dev),
+            torch.empty((wt.B, wt.H, wt.Nq), dtype=torch.float32, device=dev))
         seg("prefill_noncausal", lambda: ta.attn_fwd(q, k, v, o, lse, False, wp.scale, stream),
             wp.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
         seg("prefill_causal", lambda: ta.attn_fwd(q, k, v, o, lse, True, wp.scale, stream),
@@ -255,6 +490,7 @@ def run_ours(args):
         # (names distinct from every later block's: the lambdas look them up when they run)
         bdq, bdk, bdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         bws = torch.empty(ta.attn_bwd_workspace_bytes(wp.B, wp.H, wp.Nq), dtype=torch.uint8, device=dev)
+        D["bwd"] = (q, k, v, bo, blse, dout, bdq, bdk, bdv, bws)
         seg("prefill_bwd_noncausal",
             lambda: ta.attn_bwd(q, k, v, bo_n, dout, blse_n, bdq, bdk, bdv, False, wp.scale, bws, stream),
             2.5 * wp.flops(False), "TFLOP/s", peak_tc, "tensor", 3)
@@ -270,6 +506,7 @@ def run_ours(args):
         vq, vk, vv, vcu = (t.to(dev) for t in make_varlen(vl, vl, wp.H, wp.H, wp.d, seed=0)[:4])
         vo = torch.empty_like(vq)
         vlse = torch.empty((wp.H, vq.shape[0]), dtype=torch.float32, device=dev)
+        D["varlen"] = (vq, vk, vv, vo, vlse, vcu, vl)
         seg("prefill_varlen_causal",
             lambda: ta.attn_fwd_varlen(vq, vk, vv, vo, vlse, vcu, vcu, max(vl), True, wp.scale, stream),
             sum(2.0 * wp.H * n * n * wp.d for n in vl), "TFLOP/s", peak_tc, "tensor", 1)
@@ -285,6 +522,7 @@ def run_ours(args):
         # grouped-query decode: 4 query heads per cache head (the same queries,
         # the first H/4 cache heads); GB/s counts the cache bytes it must read
         gk, gv = dk[:, :wd.H // 4].contiguous(), dv[:, :wd.H // 4].contiguous()
+        D["decode"] = (dq, dk, dv, do, dlse, dws, gk, gv)
         seg("decode_gqa", lambda: ta.attn_decode_gqa(dq, gk, gv, do, dlse, wd.scale, wd.num_splits, dws, stream),
             2 * gk.numel() * gk.element_size(), "GB/s", peak_hbm, "hbm", 2)
     wl = WORKLOADS["longseq"]
@@ -292,6 +530,7 @@ def run_ours(args):
         lq, lk, lv = (t.to(dev) for t in make_qkv(wl, seed=0))
         lo = torch.empty_like(lq)
         llse = torch.empty(lq.shape[:3], dtype=torch.float32, device=dev)
+        D["longseq"] = (lq, lk, lv, lo, llse)
         seg("longseq_noncausal", lambda: ta.attn_fwd(lq, lk, lv, lo, llse, False, wl.scale, stream),
             wl.flops(False), "TFLOP/s", peak_tc, "tensor", 1)
         seg("longseq_causal", lambda: ta.attn_fwd(lq, lk, lv, lo, llse, True, wl.scale, stream),
@@ -309,6 +548,7 @@ def run_ours(args):
         s8.append(torch.empty((B5, H5), dtype=torch.float32, device=dev))
         of = torch.empty((B5, H5, N5, D5), dtype=torch.float32, device=dev)
         lf = torch.empty((B5, H5, N5), dtype=torch.float32, device=dev)
+        D["lowp"] = {"bf16": (xq, xk, xv, xo, xl), "int8": (i8, s8, of, lf)}
 
         def q8():
             ta.attn_quantize_int8(xq, i8[0], s8[0], False, stream)
@@ -326,6 +566,7 @@ def run_ours(args):
         def q4():
             for t, c, f, m in zip((xq, xk, xv), c4, f4, (0, 0, 1)):
                 ta.attn_quantize_nvfp4(t, c, f, m, stream)
+        D["lowp"]["fp4"] = (c4, f4)
         seg("lowp_fp4_quantise", q4, 3 * xq.numel() * 2 + sum(c.numel() for c in c4), "GB/s", peak_hbm, "hbm", 3)
         for mode, nm in ((0, "lowp_fp4_direct_p"), (1, "lowp_fp4_quant_after_exp")):
             seg(nm, (lambda mode=mode: ta.attn_fwd_fp4(c4[0], f4[0], c4[1], f4[1], c4[2], f4[2], of, lf, B5, H5,
@@ -340,25 +581,30 @@ def run_ours(args):
             ta.attn_quantize_fp8(xq, c8[0], s8f[0], 0, signs, stream)
             ta.attn_quantize_fp8(xk, c8[1], s8f[1], 0, signs, stream)
             ta.attn_quantize_fp8(xv, c8[2], s8f[2], 1, None, stream)
+        D["lowp"]["fp8"] = (c8, s8f, signs)
         seg("lowp_fp8_quantise", qf8, 3 * xq.numel() * 2 + 3 * xq.numel(), "GB/s", peak_hbm, "hbm", 5)
         seg("lowp_fp8", lambda: ta.attn_fwd_fp8(c8[0], s8f[0], c8[1], s8f[1], c8[2], s8f[2], of, lf, False,
                                                 wq.scale, True, stream),
             wq.flops(False), "TFLOP/s", peak_f8, "tensor", 1)
 
     nseg = len(segs)
+    # every launch starts with a cold L2: 256 MB written (> the 126 MB L2)
+    # between launches, outside the launch's event bracket
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step(ev):
-        ev[0].record(stream)
         for i, sg in enumerate(segs):
+            flush.fill_(i & 0xFF)
+            ev[2 * i].record(stream)
             sg[1]()
-            ev[i + 1].record(stream)
+            ev[2 * i + 1].record(stream)
 
     def barrier():
         if ws > 1:
             import torch.distributed as dist
             dist.barrier()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nseg + 1)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nseg)] for _ in range(args.steps)]
     for _ in range(args.warmup):
         step(evs[0])
     torch.cuda.synchronize()
@@ -383,7 +629,8 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device watchdog status {status}")
 
-    sums = [t_start.elapsed_time(t_end)] + [sum(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nseg)]
+    sums = [t_start.elapsed_time(t_end)] + [sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs)
+                                            for i in range(nseg)]
     sums = max_over_ranks(sums, dev)
     total_ms, seg_ms = sums[0], sums[1:]
     out_parts = {}
@@ -436,10 +683,22 @@ def run_ours(args):
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps}
 
-    cpu = None
+    cpu, accuracy = None, None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cv, desc, thr, _ = oracle_sample(args.cpu_seconds)
-        cpu = {"value": cv, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc}
+        # the quantised operands the oracle leg compares against must be the
+        # ones of this input: run the quantisers once more
+        for sg in segs:
+            if sg[0].endswith("_quantise"):
+                sg[1]()
+        per, accuracy, secs = oracle_leg(ta, dev, stream, D, args.cpu_rows)
+        hd = [per[n] for n in ("prefill_noncausal", "prefill_causal") if n in per]
+        cv = (sum(x["value"] * x["seconds"] for x in hd) / sum(x["seconds"] for x in hd)) if hd else None
+        cpu = {"value": cv, "unit": "TFLOP/s", "cores": cpu_threads(), "host_cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": (f"fp64 numpy oracle on {args.cpu_rows} query rows of 2 (batch, head) slices per "
+                          f"config and path (rate = work of those rows / oracle time; linear in rows); value = "
+                          f"prefill non-causal + causal; {secs:.1f} s of CPU work in all"),
+               "per_config": per}
 
     traffic = load_traffic()
     pn = out_parts.get("prefill_noncausal")
@@ -467,11 +726,17 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, resident in HBM)",
         "config": {"workload": "prefill", "B": wp.B, "H": wp.H, "Nq": wp.Nq, "Nkv": wp.Nkv, "d": wp.d,
                    "causal": ["false", "true"], "parallelism": f"replicas x{ws}",
-                   "l2": "every input larger than L2 (126 MB) except the int8/fp4 operands; no flush",
+                   "l2": "flushed before every launch (256 MB written, outside the launch's events)",
                    "step": sorted(out_parts)},
         "roofline": roof,
         "parts": out_parts,
         "cpu_baseline": cpu,
+        "accuracy": accuracy,
+        "tensor_peaks": None if probes is None else {
+            "method": "libtiledattn_probe: back-to-back tcgen05.mma (M=128, operands in shared memory), one CTA "
+                      "per SM; flop_per_clk_sm from the kernel's clock64, tflops from CUDA events",
+            "mma": probes["mma"], "peak_used": {"int8": peak_i8, "fp8": peak_f8, "fp4": peak_f4, "bf16": peak_tc},
+            "mufu": probes["mufu"]},
         "e2e": e2e,
         "gpu_launches": args.steps * sum(sg[6] for sg in segs),
         "clocks": clk,
@@ -502,7 +767,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="reference arm: oracle seconds per step cap")
+    ap.add_argument("--cpu-rows", type=int, default=48, help="query rows per (batch, head) in the oracle leg")
+    ap.add_argument("--no-probe", action="store_true", help="skip the tensor-peak microbenchmarks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="prefill,decode,longseq,lowp",
                     help="comma list of step parts to run (prefill, decode, longseq, lowp); profiling aid")

@@ -145,7 +145,8 @@ def attention_int8(qi, qs, ki, ks, vi, vs, causal=False, scale=None, Bc=128,
                 m_new = np.maximum(m, xb.max(axis=1))
                 grow = np.isfinite(m) & (m_new > m)
                 f = np.ones_like(m)
-                np.exp2(m - m_new, out=f, where=grow)
+                with np.errstate(invalid="ignore"):  # -inf - -inf in lanes the where() discards
+                    np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
                 m = m_new
@@ -362,7 +363,8 @@ def attention_fp4(q_deq, k_deq, v_deq, p_mode=DIRECT_P, causal=False, scale=None
                 m_new = np.maximum(m, xb.max(axis=1))
                 grow = np.isfinite(m) & (m_new > m)
                 f = np.ones_like(m)
-                np.exp2(m - m_new, out=f, where=grow)
+                with np.errstate(invalid="ignore"):  # -inf - -inf in lanes the where() discards
+                    np.exp2(m - m_new, out=f, where=grow)
                 acc *= f[:, None]
                 l *= f
                 m = m_new

@@ -1,10 +1,19 @@
 """Comparison helpers shared by the GPU parity tests (tolerances in one place).
 
 bf16 path (outputs bf16 O, fp32 LSE): max-abs 2e-2 and mean-abs 2e-3 on O,
-1e-3 on LSE, all against the fp64 oracle.  Only for inputs with outlier
-channels, where |O| reaches tens and half an ulp of the bf16 output alone
-exceeds 2e-2, does the max-abs bound grow by that half ulp (``outliers=True``);
-the error before that widening is reported beside it.
+1e-3 on LSE, all against the fp64 oracle.
+
+Inputs with outlier channels (|V| up to ~80) need a bound derived from the
+arithmetic instead: the kernel rounds every probability to bf16 before P V
+(relative error <= 2^-8 per weight, the unit roundoff of an 8-bit significand) and its output to bf16, so
+
+    |O_dev - O|_c <= 2^-8 * sum_j P_j |V_jc| + half a bf16 ulp of |O_c|
+                     (+ fp32 accumulation, far smaller),
+
+where sum_j P_j |V_jc| is attention applied to |V| (the oracle computes it).
+With ``p_abs_v`` given, max-abs allows 2e-2 plus that bound and mean-abs 2e-3
+plus its mean; the error relative to the bound is reported.  For N(0,1)
+inputs the bound is below 1e-2 and the plain 2e-2 applies.
 """
 import numpy as np
 import torch
@@ -24,19 +33,27 @@ def to64(t):
     return t.detach().to("cpu").double().numpy()
 
 
-def assert_bf16_close(o_gpu, lse_gpu, o_ref, lse_ref, what="", outliers=False):
+def bf16_p_bound(o_ref, o_dev, p_abs_v):
+    """The arithmetic bound of the module docstring, per element."""
+    return 2.0 ** -8 * p_abs_v + half_ulp_bf16(np.maximum(np.abs(o_ref), np.abs(o_dev)))
+
+
+def assert_bf16_close(o_gpu, lse_gpu, o_ref, lse_ref, what="", p_abs_v=None):
     o = to64(o_gpu)
     lse = to64(lse_gpu)
     assert o.shape == o_ref.shape, (o.shape, o_ref.shape)
     assert np.isfinite(o).all(), f"{what}: non-finite O"
     err = np.abs(o - o_ref)
-    tol = O_MAX_ABS + (half_ulp_bf16(o_ref) if outliers else 0.0)
-    if outliers:
-        print(f"{what}: O max-abs {err.max(initial=0):.3e}, beyond half a bf16 ulp of |O| "
-              f"{np.maximum(err - half_ulp_bf16(o_ref), 0).max(initial=0):.3e}")
+    extra = 0.0 if p_abs_v is None else bf16_p_bound(o_ref, o, p_abs_v)
+    tol = O_MAX_ABS + extra
+    if p_abs_v is not None:
+        print(f"{what}: O max-abs {err.max(initial=0):.3e}, mean-abs {err.mean():.3e}; largest error / "
+              f"(2^-8 sum P|V| + half ulp) {(err / np.maximum(extra, 1e-30)).max(initial=0):.3f}; "
+              f"elements beyond 2e-2 {(err > O_MAX_ABS).sum()}")
     bad = err > tol
-    assert not bad.any(), f"{what}: O max-abs {err.max():.3e} (worst tol {tol[bad].min():.3e}, {bad.sum()} bad)"
-    assert err.mean() <= O_MEAN_ABS, f"{what}: O mean-abs {err.mean():.3e}"
+    assert not bad.any(), f"{what}: O max-abs {err.max():.3e} (worst tol {np.min(tol[bad]):.3e}, {bad.sum()} bad)"
+    mean_tol = O_MEAN_ABS + (0.0 if p_abs_v is None else float(np.mean(extra)))
+    assert err.mean() <= mean_tol, f"{what}: O mean-abs {err.mean():.3e} (tol {mean_tol:.3e})"
     fin = np.isfinite(lse_ref)
     assert (np.isneginf(lse[~fin])).all(), f"{what}: LSE should be -inf for rows that see no key"
     if fin.any():

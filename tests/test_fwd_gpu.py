@@ -4,9 +4,9 @@ Small cases run the oracle on every output; the full workloads (prefill
 B4 H16 N4096 d128; long sequence B1 H12 N23400 d64; the outlier workload B2
 H24 N8192 d128 with 4 channels x20 per head) are checked on sampled query
 rows of every head, in the same launch configuration the benchmark times.
-Tolerances: max-abs 2e-2, mean-abs 2e-3 on O, 1e-3 on LSE (on the outlier
-workload the max-abs bound grows by half a bf16 ulp of |O|, which reaches
-tens there).
+Tolerances: max-abs 2e-2, mean-abs 2e-3 on O, 1e-3 on LSE; on the outlier
+workload (|V| up to ~80) the bounds grow by what bf16 P and a bf16 output
+imply there, 2^-8 * sum_j P_j |V_j| + half an ulp of |O| (tests._parity).
 
 The lazy rescale ("FlashAttention 4" page, "Smarter online softmax
 rescaling": the reference max moves, and O is corrected in tensor memory,
@@ -130,7 +130,8 @@ def test_outlier_workload_sampled_rows(cuda_lib):
     o, lse = run(cuda_lib, q, k, v, False, w.scale)
     rows = _sample_rows(w.Nq, 40, 7)
     O, L = A.attention(q, k, v, False, w.scale, rows=rows)
-    assert_bf16_close(o[:, :, rows], lse[:, :, rows], O, L, "outlier workload", outliers=True)
+    PV, _ = A.attention(q, k, v.abs(), False, w.scale, rows=rows)     # sum_j P_j |V_j|
+    assert_bf16_close(o[:, :, rows], lse[:, :, rows], O, L, "outlier workload", p_abs_v=PV)
     assert torch.isfinite(lse).all()
 
 

@@ -1,4 +1,6 @@
-"""Build libtiledattn.so in-tree with nvcc for sm_100a.
+"""Build libtiledattn.so (the attention library) and libtiledattn_probe.so
+(the throughput microbenchmarks behind the roofline denominators) in-tree
+with nvcc for sm_100a.
 
     python -m tiled_attention_24_b200.build [--verbose]
 
@@ -19,6 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtiledattn.so")
 SOURCES = ["api.cu"]
+PROBE_LIB = os.path.join(PKG, "libtiledattn_probe.so")
+PROBE_SOURCES = ["probe.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -31,21 +35,30 @@ def nvcc_path() -> str:
 
 def _deps():
     files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
-    files.append(os.path.join(INCLUDE, "tiledattn.h"))
+    files += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     files.append(os.path.abspath(__file__))
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(verbose: bool = False, force: bool = False, out: str | None = None, defines=()) -> str:
+def build_probe(verbose: bool = False, force: bool = False) -> str:
+    """Compile libtiledattn_probe.so (include/tiledattn_probe.h)."""
+    if not force and up_to_date(PROBE_LIB):
+        return PROBE_LIB
+    return build(verbose=verbose, force=True, out=PROBE_LIB, sources=PROBE_SOURCES)
+
+
+def build(verbose: bool = False, force: bool = False, out: str | None = None, defines=(),
+          sources=None) -> str:
     """Compile libtiledattn.so (or `out`, with extra -D `defines`, for tuning
-    sweeps of compile-time kernel parameters)."""
+    sweeps of compile-time kernel parameters; `sources` for another library
+    of this package)."""
     lib = out or LIB
     if not force and out is None and not defines and up_to_date():
         return LIB
@@ -55,7 +68,7 @@ def build(verbose: bool = False, force: bool = False, out: str | None = None, de
     cmd += ["-D" + d for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
+    cmd += [os.path.join(CSRC, s) for s in (sources or SOURCES)]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if verbose or res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
@@ -73,3 +86,5 @@ if __name__ == "__main__":
     ap.add_argument("-D", dest="defines", action="append", default=[])
     a = ap.parse_args()
     print(build(verbose=a.verbose, force=True, out=a.out, defines=a.defines))
+    if a.out is None and not a.defines:
+        print(build_probe(verbose=a.verbose, force=True))
