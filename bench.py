@@ -68,15 +68,16 @@ def load_peaks():
 
 def measure_peaks(dev):
     """Tensor-core ceilings per MMA kind and MUFU exponential rates, measured
-    on this GPU by libtiledattn_probe (one CTA per SM, SM cycles from the
-    kernels' own clock and TFLOP/s from CUDA events).  Rates are taken at
-    N = 128, the MMA shape the attention kernels issue, and at N = 256."""
+    on this GPU by libtiledattn_probe (one CTA per SM, a straight-line issue
+    loop, SM cycles from the kernels' own clock and TFLOP/s from CUDA
+    events).  Rates are taken at N = 128, the MMA shape the attention kernels
+    issue, and at N = 256."""
     from tiled_attention_24_b200 import _probe
     mma = {}
     for kind in ("bf16", "int8", "fp8", "fp4"):
-        mma[kind] = _probe.mma_rate(kind, 128, device=dev)
+        mma[kind] = _probe.mma_tight_rate(kind, 128, device=dev)
         if kind != "fp4":
-            mma[kind + "_n256"] = _probe.mma_rate(kind, 256, device=dev)
+            mma[kind + "_n256"] = _probe.mma_tight_rate(kind, 256, device=dev)
     mufu = {f"ex2_{t}threads": _probe.ex2_rate(t, 8, device=dev)["ex2_per_clk_sm"] for t in (1024, 256, 128)}
     mufu["ex2_256threads_ilp1"] = _probe.ex2_rate(256, 1, device=dev)["ex2_per_clk_sm"]
     mufu["softmax_scores_per_clk_sm_256threads"] = _probe.softmax_rate(256, device=dev)["scores_per_clk_sm"]
@@ -733,8 +734,9 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "accuracy": accuracy,
         "tensor_peaks": None if probes is None else {
-            "method": "libtiledattn_probe: back-to-back tcgen05.mma (M=128, operands in shared memory), one CTA "
-                      "per SM; flop_per_clk_sm from the kernel's clock64, tflops from CUDA events",
+            "method": "libtiledattn_probe tap_mma_tight_rate: back-to-back tcgen05.mma (M=128, operands in "
+                      "shared memory, straight-line issue), one CTA per SM; flop_per_clk_sm from the kernel's "
+                      "clock64, tflops from CUDA events at the clock the loop ran at",
             "mma": probes["mma"], "peak_used": {"int8": peak_i8, "fp8": peak_f8, "fp4": peak_f4, "bf16": peak_tc},
             "mufu": probes["mufu"]},
         "e2e": e2e,

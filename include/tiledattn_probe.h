@@ -58,7 +58,9 @@ extern "C" {
 int tap_mma_rate(int kind, int n, int iters, int grid, int flags, unsigned long long* cycles, void* stream);
 
 /* The same measurement with the issue loop fixed at compile time: kind
- * (bf16, int8 or e4m3 only), N (128 or 256) and the A source as template
+ * (bf16, int8, e4m3; block-scaled e2m1 with n = 128 and no flag but
+ * TAP_COMMIT, 64-byte swizzled tiles and unit scale factors as the FP4
+ * attention kernel uses), N (128 or 256) and the A source as template
  * parameters, descriptors computed before the loop, `iters` groups of eight
  * MMAs (K = 256 bytes per row: the K sweep of a 128-deep tile pair) with
  * immediate offsets, all into one accumulator.  TAP_COMMIT adds a

@@ -45,6 +45,13 @@
 #pragma once
 #include "ptx.cuh"
 
+// Speculative barrier tests inside MMA groups (hide a wait's latency behind
+// the group's last MMA).  Off: every mbarrier operation of the issuing thread
+// first waits for its queued MMAs to drain, so the test itself leaves a
+// bubble in the tensor pipe (measured: ~70 cycles per group).
+#ifndef TA_SPEC_TEST
+#define TA_SPEC_TEST 0
+#endif
 #ifndef TA_POLY_PERIOD
 #define TA_POLY_PERIOD 4
 #endif
@@ -259,8 +266,7 @@ __global__ void __launch_bounds__(384, 1)
     // blocking) just before the last MMA of the current group is issued, so
     // that the test's latency hides behind that MMA.
     if (lane == 0) {
-      bool ok = wait_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
-      tc_fence_after();
+      bool ok = spin_bar(smem_u32(&bars->q_full), 0, abort_flag, p.timeout_ns);
       const uint64_t dQ0 = smem_desc(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dQ1 = smem_desc(sbase + C::Q_OFF + C::TILE, 16, 1024);
       const uint64_t dV0 = smem_desc(sbase + C::SLOT_OFF, C::HALF, 1024);
@@ -270,11 +276,11 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dq = t ? dQ1 : dQ0;
         const uint64_t dk = dK0 + (uint64_t)(st * (C::STAGE >> 4));
         const uint32_t dS = tbase + t * 128;
-        bool ready = true;
+        bool ready = TA_SPEC_TEST != 0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4);
-          if (kk == D / 16 - 1 && nb) ready = mbar_test_wait(nb, np);
+          if (TA_SPEC_TEST && kk == D / 16 - 1 && nb) ready = mbar_test_wait(nb, np);
           mma_f16_ss(dS, dq + off, dk + off, C::ID_S, kk > 0);
         }
         tc_commit(smem_u32(&bars->s_full[t]));
@@ -284,26 +290,34 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dv = dV0 + (uint64_t)(st * (C::STAGE >> 4));
         const uint32_t dO = tbase + C::T_O + t * D, aP = tbase + (C::SEP_P ? C::T_P + 64 * t : 128 * t);
         const uint32_t acc0 = (j > 0) ? 1u : 0u;
-        bool ready = true;
+        bool ready = TA_SPEC_TEST != 0;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
-          if (kk == 7 && nb) ready = mbar_test_wait(nb, np);
+          if (TA_SPEC_TEST && kk == 7 && nb) ready = mbar_test_wait(nb, np);
           mma_f16_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), C::ID_PV, kk > 0 ? 1u : acc0);
         }
         return ready;
       };
-      // wait for (bar, parity) unless a speculative test already saw it
+      // Barrier waits poll without suspending (spin_bar): a suspended
+      // try_wait can resume a few hundred cycles after the phase completes,
+      // and the softmax of the other tile is on the critical path behind it.
+      // A barrier the softmax arrives at (after writing or reading tensor
+      // memory) needs the tcgen05 fence; a TMA barrier does not (TMA writes
+      // and MMA operand reads are both in the async proxy, ordered by the
+      // barrier's transaction count).
       auto need = [&](bool seen, uint32_t bar, uint32_t par) -> bool {
-        if (!seen && !wait_bar(bar, par, abort_flag, p.timeout_ns)) return false;
+        if (!seen && !spin_bar(bar, par, abort_flag, p.timeout_ns)) return false;
         tc_fence_after();
         return true;
+      };
+      auto need_tma = [&](bool seen, uint32_t bar, uint32_t par) -> bool {
+        return seen || spin_bar(bar, par, abort_flag, p.timeout_ns);
       };
       const uint32_t pf0 = smem_u32(&bars->p_full[0]), pf1 = smem_u32(&bars->p_full[1]);
       int st = 0;        // stage of the current step (slot), its phase
       uint32_t sp = 0;
       if (ok && nmax > 0) {
-        ok = wait_bar(smem_u32(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns);
-        tc_fence_after();
+        ok = spin_bar(smem_u32(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns);
         if (ok) {
           if (n[0] > 0) issue_S(0, 0, 0, 0);
           if (n[1] > 0) issue_S(1, 0, 0, 0);
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(384, 1)
         bool seenSt = false;
         for (int j = 0; j < nmax && ok; ++j) {
           if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
-          if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
+          if (!(ok = need_tma(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
           int st1 = st + 1;
           uint32_t sp1 = sp;
           if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(384, 1)
         bool seenSt = false;
         for (int j = 0; j < nmax && ok; ++j) {
           if (++st == C::NSTAGE) { st = 0; sp ^= 1u; }
-          if (!(ok = need(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
+          if (!(ok = need_tma(seenSt, smem_u32(&bars->kv_full[st]), sp))) break;
           int st1 = st + 1;
           uint32_t sp1 = sp;
           if (st1 == C::NSTAGE) { st1 = 0; sp1 ^= 1u; }

@@ -238,6 +238,10 @@ __global__ void __launch_bounds__(128, 1) mma_tight_kernel(int iters, unsigned l
   uint32_t* w = reinterpret_cast<uint32_t*>(smem);
   for (int i = threadIdx.x; i < (A_BYTES + B_BYTES) / 4; i += blockDim.x)
     w[i] = fill_word(KIND, (uint32_t)i + 7919u * blockIdx.x);
+  // e2m1 scale factors (ue4m3 1.0), 1 KB after the barrier block
+  constexpr int SF_OFF = A_BYTES + B_BYTES + 1024;
+  if (KIND == TAP_KIND_F4)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) reinterpret_cast<uint32_t*>(smem + SF_OFF)[i] = 0x38383838u;
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bar[0]), 1);
     mbar_init(smem_u32(&bar[1]), 1);
@@ -293,8 +297,23 @@ __global__ void __launch_bounds__(128, 1) mma_tight_kernel(int iters, unsigned l
   }
   const int issuer = (SYNC & 8) ? (threadIdx.x >> 5) : 0;
   if ((threadIdx.x & 31) == 0 && ((SYNC & 8) ? issuer < 2 : threadIdx.x == 0)) {
-    constexpr uint32_t fmt = (KIND == TAP_KIND_BF16) ? kFmtBf16 : (KIND == TAP_KIND_I8) ? kFmtI8 : kFmtF8;
+    constexpr uint32_t fmt = (KIND == TAP_KIND_BF16) ? kFmtBf16
+                             : (KIND == TAP_KIND_I8)  ? kFmtI8
+                             : (KIND == TAP_KIND_F8)  ? kFmtF8
+                                                      : kFmtF4;
     constexpr uint32_t id = idesc_mn(fmt, N);
+    // e2m1 (block-scaled): 64-byte rows, 64-byte swizzle, four 128 x 64-byte
+    // tiles per operand (K = 512 per row), two MMAs (K = 64, 32 bytes) per
+    // tile; scale factors in columns [320, 336) (A) and [336, 352) (B)
+    const uint32_t t_sfa = tbase + 320, t_sfb = tbase + 336;
+    if (KIND == TAP_KIND_F4) {
+      const uint64_t dsf = desc_layout(sbase + SF_OFF, 128, 0);
+      for (int c = 0; c < 4; ++c) {
+        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(t_sfa + 4 * c), "l"(dsf) : "memory");
+        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(t_sfb + 4 * c), "l"(dsf) : "memory");
+      }
+    }
+    const uint64_t da4 = desc_layout(sbase, 512, 4), db4 = desc_layout(sbase + A_BYTES, 512, 4);
     // MN-major B (N contiguous, as the attention kernels read V): the tile is
     // two 64-element-wide halves (bf16; 128 wide for 8-bit) of K rows x 128
     // bytes, LBO = the distance between halves, SBO = 8 rows
@@ -321,7 +340,11 @@ __global__ void __launch_bounds__(128, 1) mma_tight_kernel(int iters, unsigned l
         const uint64_t bo = (uint64_t)(((kk >> 2) * N * 128 + (kk & 3) * 32) >> 4);
         const uint64_t bo_mn = (uint64_t)((kk * ROWS_PER_MMA * 128) >> 4);
         const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-        if (BMODE == 0) {
+        if (KIND == TAP_KIND_F4) {
+          const uint64_t ao4 = (uint64_t)(((kk >> 1) * 128 * 64 + (kk & 1) * 32) >> 4);
+          const uint64_t bo4 = (uint64_t)(((kk >> 1) * N * 64 + (kk & 1) * 32) >> 4);
+          mma_kind(KIND, tbase, da4 + ao4, db4 + bo4, id, acc, t_sfa + 4 * (kk & 1), t_sfb + 4 * (kk & 1));
+        } else if (BMODE == 0) {
           if (A_TMEM)
             mma_kind_ts(KIND, tbase, tbase + kTA + 8 * kk, db + bo, id, acc);
           else
@@ -496,6 +519,10 @@ TAP_API int tap_mma_tight_rate(int kind, int n, int iters, int grid, int flags, 
     case TAP_KIND_BF16: return tight_dispatch<TAP_KIND_BF16>(n, flags, iters, grid, cycles, st);
     case TAP_KIND_I8: return tight_dispatch<TAP_KIND_I8>(n, flags, iters, grid, cycles, st);
     case TAP_KIND_F8: return tight_dispatch<TAP_KIND_F8>(n, flags, iters, grid, cycles, st);
+    case TAP_KIND_F4:
+      if (n != 128 || flags & ~TAP_COMMIT) return -1;
+      return (flags & TAP_COMMIT) ? launch_tight<TAP_KIND_F4, 128, false, true>(iters, grid, cycles, st)
+                                  : launch_tight<TAP_KIND_F4, 128, false, false>(iters, grid, cycles, st);
     default: return -1;
   }
 }

@@ -85,6 +85,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Bounded wait that polls with mbarrier.test_wait and never suspends the
+// thread: for the MMA-issuing thread, which must issue the moment a phase
+// completes (a suspended try_wait can resume a few hundred cycles late).
+__device__ __forceinline__ bool spin_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicExch(&g_attn_status, -5 /* ATTN_ERR_TIMEOUT */);
+      return false;
+    }
+  }
+}
+
 // Pairwise exchange of one float between two threads of different warps
 // through a 64-bit shared slot {tag, value}: the writer stores (tag << 32 |
 // bits) in one 64-bit access; the reader polls its partner's slot until the
