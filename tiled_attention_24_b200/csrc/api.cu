@@ -491,10 +491,14 @@ static int decode_impl(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf
                                            (((size_t)BH * num_splits * d * sizeof(float) + 255) & ~size_t(255)));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float sl2 = scale * 1.4426950408889634f;
-  // query heads per CTA: the largest of 8, 4, 2 dividing the group (each
-  // cache row then crosses memory once per G query heads); 1 = plain kernel
+  // query heads per CTA: the largest of 4, 2 dividing the group (each cache
+  // row then crosses memory once per G query heads; a group of 8 runs as two
+  // CTAs of 4, the second reading the cache head from L2); 1 = plain kernel.
+  // Eight heads in one CTA take 255 registers and two CTAs per SM, too few
+  // loads in flight: 1560 GB/s against 2260 as two CTAs of 4 (B64 Hq32
+  // Hkv4 N_kv 8192 d128).
   const int grp = H / Hkv;
-  const int G = (grp % 8 == 0) ? 8 : (grp % 4 == 0) ? 4 : (grp % 2 == 0) ? 2 : 1;
+  const int G = (grp % 4 == 0) ? 4 : (grp % 2 == 0) ? 2 : 1;
   const unsigned grid = (unsigned)(BH / G * num_splits);
   if (G == 1) {
     if (d == 128)
@@ -508,9 +512,9 @@ static int decode_impl(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf
   ta::decode_split_group_kernel<DD, GG><<<grid, ta::DEC_THREADS, 0, st>>>(q, k, v, o_part, l_part, Nkv, \
                                                                          num_splits, chunk, sl2, grp, seqlens, H)
     if (d == 128) {
-      if (G == 8) TA_DECODE_GROUP(128, 8); else if (G == 4) TA_DECODE_GROUP(128, 4); else TA_DECODE_GROUP(128, 2);
+      if (G == 4) TA_DECODE_GROUP(128, 4); else TA_DECODE_GROUP(128, 2);
     } else {
-      if (G == 8) TA_DECODE_GROUP(64, 8); else if (G == 4) TA_DECODE_GROUP(64, 4); else TA_DECODE_GROUP(64, 2);
+      if (G == 4) TA_DECODE_GROUP(64, 4); else TA_DECODE_GROUP(64, 2);
     }
 #undef TA_DECODE_GROUP
   }

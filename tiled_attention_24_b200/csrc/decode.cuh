@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(DEC_THREADS)
     lse_part[part] = (nk > 0) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 }
 
-// Grouped-query split kernel: one CTA per (G consecutive query heads that
-// share a cache head, chunk).  Each key and value row is read from memory
+// Grouped-query split kernel: one CTA per (G = 2 or 4 consecutive query heads
+// that share a cache head, chunk).  Each key and value row is read from memory
 // once and used by all G query heads, so the bytes moved per query head drop
 // by G ([FA4-overview] "Compatibility and current status": several heads
 // share one key/value projection).  Same lane layout and sub-block online
