@@ -594,7 +594,8 @@ int attn_quantize_int8(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H
   const long long BH = (long long)B * H;
   if (!per_head) {
     const long long rows = BH * N;
-    const long long blocks = (rows + 7) / 8;
+    const long long per_block = (d == 128) ? ta::qrow_rows_per_block<128>() : ta::qrow_rows_per_block<64>();
+    const long long blocks = (rows + per_block - 1) / per_block;
     if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     if (d == 128)
       ta::quant_int8_rows_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
@@ -621,7 +622,8 @@ int attn_quantize_int4(const attn_bf16_t* x, int8_t* xq, float* xs, int B, int H
   if (!aligned16(x) || !aligned16(xq) || !aligned4(xs)) return ATTN_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const long long rows = (long long)B * H * N;
-  const long long blocks = (rows + 7) / 8;
+  const long long per_block = (d == 128) ? ta::qrow_rows_per_block<128>() : ta::qrow_rows_per_block<64>();
+  const long long blocks = (rows + per_block - 1) / per_block;
   if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (d == 128)
     ta::quant_int8_rows_kernel<128, 7><<<(unsigned)blocks, 256, 0, st>>>(x, xq, xs, rows);
@@ -671,7 +673,8 @@ int attn_quantize_fp8(const attn_bf16_t* x, uint8_t* codes, float* scales, int B
   const long long BH = (long long)B * H;
   if (mode == 0) {
     const long long rows = BH * N;
-    const long long blocks = (rows + 7) / 8;
+    const long long per_block = (d == 128) ? ta::qrow_rows_per_block<128>() : ta::qrow_rows_per_block<64>();
+    const long long blocks = (rows + per_block - 1) / per_block;
     if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     if (d == 128)
       ta::quant_fp8_rows_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(x, signs, codes, scales, rows);

@@ -21,43 +21,56 @@ __device__ __forceinline__ int8_t q8(float x, float s) {
   return (int8_t)v;
 }
 
-// One warp per row of D bf16 values (D = 64 or 128).  QMAX = 127 (INT8) or 7
-// (INT4 codes in int8 containers: the same token-level scheme at 4 bits).
+// Row quantiser: LPR = D / 8 lanes per row (16 bytes = 8 bf16 each; 16 lanes
+// at d = 128, 8 at d = 64), 32 / LPR rows per warp pass, QROW_PASSES passes
+// per warp whose loads are all issued before any row is quantised (bytes in
+// flight per lane: 16 x QROW_PASSES).  QMAX = 127 (INT8) or 7 (INT4 codes in
+// int8 containers: the same token-level scheme at 4 bits).
+constexpr int QROW_PASSES = 4;
+template <int D>
+__host__ __device__ constexpr long long qrow_rows_per_block() { return 8LL * (32 / (D / 8)) * QROW_PASSES; }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
+  v[0] = __uint_as_float(w.x << 16); v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(w.y << 16); v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  v[4] = __uint_as_float(w.z << 16); v[5] = __uint_as_float(w.z & 0xFFFF0000u);
+  v[6] = __uint_as_float(w.w << 16); v[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
 template <int D, int QMAX = 127>
 __global__ void __launch_bounds__(256) quant_int8_rows_kernel(const uint16_t* __restrict__ x, int8_t* __restrict__ xq,
                                                              float* __restrict__ xs, long long rows) {
-  constexpr int E = D / 32;  // elements per lane
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint16_t* src = x + row * D + lane * E;
-  float v[E];
-  if constexpr (E == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(src);
-    v[0] = __uint_as_float(w.x << 16);
-    v[1] = __uint_as_float(w.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(w.y << 16);
-    v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-  } else {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
-    v[0] = __uint_as_float(w << 16);
-    v[1] = __uint_as_float(w & 0xFFFF0000u);
+  constexpr int LPR = D / 8, RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31, sub = lane / LPR, cl = lane % LPR;
+  const long long row0 = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * (RPW * QROW_PASSES);
+  uint4 w[QROW_PASSES];
+#pragma unroll
+  for (int pss = 0; pss < QROW_PASSES; ++pss) {
+    const long long row = row0 + pss * RPW + sub;
+    w[pss] = (row < rows) ? *reinterpret_cast<const uint4*>(x + row * D + cl * 8) : make_uint4(0, 0, 0, 0);
   }
-  float amax = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[e]));
+  for (int pss = 0; pss < QROW_PASSES; ++pss) {
+    const long long row = row0 + pss * RPW + sub;
+    float v[8];
+    unpack_bf16x8(w[pss], v);
+    float amax = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, (float)QMAX);
-  uint32_t packed = 0;
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
 #pragma unroll
-  for (int e = 0; e < E; ++e) packed |= (uint32_t)(uint8_t)q8<QMAX>(v[e], s) << (8 * e);
-  if constexpr (E == 4) {
-    *reinterpret_cast<uint32_t*>(xq + row * D + lane * E) = packed;
-  } else {
-    *reinterpret_cast<uint16_t*>(xq + row * D + lane * E) = (uint16_t)packed;
+    for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, (float)QMAX);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      lo |= (uint32_t)(uint8_t)q8<QMAX>(v[e], s) << (8 * e);
+      hi |= (uint32_t)(uint8_t)q8<QMAX>(v[e + 4], s) << (8 * e);
+    }
+    if (row < rows) {
+      *reinterpret_cast<uint2*>(xq + row * D + cl * 8) = make_uint2(lo, hi);
+      if (cl == 0) xs[row] = s;
+    }
   }
-  if (lane == 0) xs[row] = s;
 }
 
 // Per-(batch, head) amax, accumulated with an integer atomicMax on the bit
@@ -240,63 +253,77 @@ __device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {  // lo -> 
   return r;
 }
 
-// One warp per row; D / 32 values per lane (element e = lane * E + i).
+// Same lane layout as the INT8 row quantiser: D / 8 lanes per row, 8 values
+// per lane (element e = lane_in_row * 8 + i), QROW_PASSES rows per lane with
+// all loads issued first.  The transform stages h = 1, 2, 4 run inside a lane,
+// h >= 8 across lanes (partner lane differs in bit h / 8), with the same fp32
+// operations in the same order as the stage definition.
 template <int D>
 __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const uint16_t* __restrict__ x,
                                                              const float* __restrict__ signs,
                                                              uint8_t* __restrict__ codes, float* __restrict__ xs,
                                                              long long rows) {
-  constexpr int E = D / 32;
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint16_t* src = x + row * D + lane * E;
-  float v[E];
+  constexpr int E = 8, LPR = D / 8, RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31, sub = lane / LPR, cl = lane % LPR;
+  const long long row0 = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * (RPW * QROW_PASSES);
+  float sg[E];
 #pragma unroll
-  for (int i = 0; i < E; ++i) v[i] = bf16_to_f32(src[i]);
-  if (signs != nullptr) {
+  for (int i = 0; i < E; ++i) sg[i] = (signs != nullptr) ? signs[cl * E + i] : 1.f;
+  uint4 w[QROW_PASSES];
 #pragma unroll
-    for (int i = 0; i < E; ++i) v[i] *= signs[lane * E + i];
-    // stages inside a lane
+  for (int pss = 0; pss < QROW_PASSES; ++pss) {
+    const long long row = row0 + pss * RPW + sub;
+    w[pss] = (row < rows) ? *reinterpret_cast<const uint4*>(x + row * D + cl * E) : make_uint4(0, 0, 0, 0);
+  }
 #pragma unroll
-    for (int h = 1; h < E; h <<= 1) {
+  for (int pss = 0; pss < QROW_PASSES; ++pss) {
+    const long long row = row0 + pss * RPW + sub;
+    float v[E];
+    unpack_bf16x8(w[pss], v);
+    if (signs != nullptr) {
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if ((i & h) == 0) {
-          const float a = v[i], b = v[i + h];
-          v[i] = a + b;
-          v[i + h] = a - b;
+      for (int i = 0; i < E; ++i) v[i] *= sg[i];
+      // stages inside a lane
+#pragma unroll
+      for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          if ((i & h) == 0) {
+            const float a = v[i], b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+          }
+        }
+      }
+      // stages across the lanes of the row: partner lane differs in bit h / E
+#pragma unroll
+      for (int h = E; h < D; h <<= 1) {
+        const int lm = h / E;
+        const bool upper = (cl & lm) != 0;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, v[i], lm);
+          v[i] = upper ? (o - v[i]) : (v[i] + o);
         }
       }
     }
-    // stages across lanes: partner lane differs in bit h / E
+    float amax = 0.f;
 #pragma unroll
-    for (int h = E; h < D; h <<= 1) {
-      const int lm = h / E;
-      const bool upper = (lane & lm) != 0;
+    for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], lm);
-        v[i] = upper ? (o - v[i]) : (v[i] + o);
-      }
+    for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      lo |= e4m3x2_bits(__fdiv_rn(v[i], s), __fdiv_rn(v[i + 1], s)) << (8 * i);
+      hi |= e4m3x2_bits(__fdiv_rn(v[i + 4], s), __fdiv_rn(v[i + 5], s)) << (8 * i);
+    }
+    if (row < rows) {
+      *reinterpret_cast<uint2*>(codes + row * D + cl * E) = make_uint2(lo, hi);
+      if (cl == 0) xs[row] = s;
     }
   }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
-  uint32_t packed = 0;
-#pragma unroll
-  for (int i = 0; i < E; i += 2)
-    packed |= e4m3x2_bits(__fdiv_rn(v[i], s), __fdiv_rn(v[i + 1], s)) << (8 * i);
-  if constexpr (E == 4) {
-    *reinterpret_cast<uint32_t*>(codes + row * D + lane * E) = packed;
-  } else {
-    *reinterpret_cast<uint16_t*>(codes + row * D + lane * E) = (uint16_t)packed;
-  }
-  if (lane == 0) xs[row] = s;
 }
 
 // V: one scale per (batch, head, channel) over the head's tokens.  Three
