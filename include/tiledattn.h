@@ -59,8 +59,11 @@ enum {
   ATTN_ERR_MISALIGNED = -3,  /* pointer not 16-byte aligned                 */
   ATTN_ERR_CUDA = -4,        /* CUDA runtime/driver error at launch         */
   ATTN_ERR_TIMEOUT = -5,     /* a kernel wait ran past its time limit       */
-  ATTN_ERR_TOO_LARGE = -6    /* request needs more than the library's fixed
+  ATTN_ERR_TOO_LARGE = -6,   /* request needs more than the library's fixed
                                 scratch (attn_decode_noalloc)               */
+  ATTN_ERR_BOUNDS = -7       /* debug build only: a kernel's TMA coordinate
+                                or tensor-memory address failed its check;
+                                the access was skipped (attn_debug_counters) */
 };
 
 /* Human-readable name of a status code (static string). */
@@ -387,8 +390,9 @@ ATTN_API int attn_fwd_fp8(const uint8_t* q, const float* q_scale, const uint8_t*
 
 /*
  * attn_check_status -- synchronise `stream`, read the device status word
- * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT), clear it and
- * return it; also returns ATTN_ERR_CUDA if the synchronisation itself fails.
+ * written by the kernels' watchdog (ATTN_OK or ATTN_ERR_TIMEOUT; in the debug
+ * build also ATTN_ERR_BOUNDS), clear it and return it; also returns
+ * ATTN_ERR_CUDA if the synchronisation itself fails.
  */
 ATTN_API int attn_check_status(void* stream);
 
@@ -405,6 +409,28 @@ ATTN_API void attn_set_wait_limit_ns(unsigned long long ns);
  * reports it.  Exercises the timeout path without a fault or a hang.
  */
 ATTN_API int attn_watchdog_selftest(unsigned long long limit_ns, void* stream);
+
+/*
+ * attn_debug_counters -- counters of the debug build (libtiledattn_debug.so,
+ * compiled with TA_DEBUG = 1): the product build returns
+ * ATTN_ERR_UNSUPPORTED and writes nothing.  Synchronises the device, copies
+ * four unsigned 64-bit counters to `out` (host memory, 4 entries) and, if
+ * `reset` is non-zero, clears them:
+ *   out[0]  lazy rescales of the bf16 forward: query rows whose reference max
+ *           moved (block max above it by more than 8 in log2 units) after
+ *           the row's first key block ("FlashAttention 4" page, smarter
+ *           online softmax rescaling), summed over launches;
+ *   out[1]  key tiles that causal bf16-forward CTAs skipped (tiles wholly in
+ *           the future of a query tile; "Can a full-day context beat one
+ *           minute?" page, causal masking);
+ *   out[2]  bounds violations: TMA coordinates or tensor-memory addresses
+ *           that failed the debug build's checks (each also records
+ *           ATTN_ERR_BOUNDS for attn_check_status and skips the access);
+ *   out[3]  reserved (0).
+ * Returns ATTN_ERR_INVALID_ARG for a null `out`, ATTN_ERR_CUDA if the copy
+ * fails.
+ */
+ATTN_API int attn_debug_counters(unsigned long long* out, int reset);
 
 #ifdef __cplusplus
 }

@@ -240,7 +240,8 @@ def attention_blockwise(q, k, v, causal: bool = False, scale: float | None = Non
 
 
 def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = None,
-                           Bc: int = 128, tau: float = 8.0, count_rescales: bool = False):
+                           Bc: int = 128, tau: float = 8.0, count_rescales: bool = False,
+                           rescale_rows: bool = False):
     """The deferred-normalisation form with lazy rescaling, base 2.
 
     [FA-trading] "FA2" item 1: the output accumulator stays unnormalised and is
@@ -255,7 +256,11 @@ def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = 
     same stale reference.
 
     Returns (O, LSE) and, if ``count_rescales``, the number of (row, block)
-    pairs in which the reference moved after the first block.
+    pairs in which the reference moved after the first block.  With
+    ``rescale_rows`` it returns (O, LSE, moves, margin) instead: per query row
+    ([B, H, Nq]) the number of such moves, and the smallest distance
+    |m_blk - (m + tau)| of any of its decisions after the first block (inf for
+    a row with none) -- how close the row came to the threshold.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, Nq, d = q.shape
@@ -266,6 +271,8 @@ def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = 
     LSE = np.full((B, H, Nq), -np.inf)
     vis = visible_mask(Nq, Nkv, causal)
     rescales = 0
+    moves = np.zeros((B, H, Nq), dtype=np.int64)
+    margin = np.full((B, H, Nq), np.inf)
     for b in range(B):
         for h in range(H):
             acc = np.zeros((Nq, v.shape[3]))
@@ -280,6 +287,11 @@ def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = 
                 move = np.isfinite(m_new) & (~np.isfinite(m) | (m_new > m + tau))
                 if jb > 0:
                     rescales += int(np.count_nonzero(move & np.isfinite(m)))
+                    moves[b, h] += move & np.isfinite(m)
+                    decided = np.isfinite(m) & np.isfinite(m_blk)
+                    with np.errstate(invalid="ignore"):
+                        gap = np.abs(m_blk - (m + tau))
+                    margin[b, h] = np.where(decided, np.minimum(margin[b, h], gap), margin[b, h])
                 with np.errstate(invalid="ignore"):  # -inf - -inf in lanes the where() discards
                     f = np.where(move & np.isfinite(m),
                                  np.exp2(np.where(move & np.isfinite(m), m - m_new, 0.0)), 1.0)
@@ -296,6 +308,8 @@ def attention_lazy_rescale(q, k, v, causal: bool = False, scale: float | None = 
             ls = np.where(ok, l, 1.0)
             O[b, h] = np.where(ok[:, None], acc / ls[:, None], 0.0)
             LSE[b, h] = np.where(ok, LN2 * (np.where(ok, m, 0.0) + np.log2(ls)), -np.inf)
+    if rescale_rows:
+        return O, LSE, moves, margin
     if count_rescales:
         return O, LSE, rescales
     return O, LSE

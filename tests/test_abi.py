@@ -157,3 +157,19 @@ def test_product_path_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.replace("oracle/", ""), f
+
+
+def test_debug_counters_only_in_debug_build(lib):
+    """The product library answers ATTN_ERR_UNSUPPORTED (before any CUDA
+    call); the debug build exports the same entry points and rejects a null
+    output on the host."""
+    buf = (ctypes.c_ulonglong * 4)()
+    assert lib.attn_debug_counters(ctypes.cast(buf, ctypes.c_void_p), 0) == -2
+    assert lib.attn_status_string(-7) == b"ATTN_ERR_BOUNDS"
+    from tiled_attention_24_b200 import build
+    path = build.build_debug()
+    dbg = ctypes.CDLL(path)
+    for n in sorted(_declared()):
+        assert hasattr(dbg, n), n
+    dbg.attn_debug_counters.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    assert dbg.attn_debug_counters(None, 0) == -1

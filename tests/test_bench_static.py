@@ -7,6 +7,7 @@
   before anything reaches the C ABI.
 """
 import ast
+import json
 import os
 
 import pytest
@@ -59,3 +60,26 @@ def test_binding_rejects_mis_shaped_buffers():
         b._expect((ok, (2, 3, 4), torch.float32, "x"))
     with pytest.raises(ValueError):
         b._at_least(torch.empty(10, dtype=torch.uint8), 11, "codes")
+
+
+def test_traffic_record_is_dropped_when_the_sources_change(tmp_path, monkeypatch):
+    """profiles/traffic.json holds ncu DRAM bytes stamped with a digest of the
+    kernel sources; a record from other sources reads as empty."""
+    from tiled_attention_24_b200 import traffic
+    log = tmp_path / "t.csv"
+    log.write_text(
+        "==PROF== Connected to process 1\n"
+        '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+        '"0","k","dram__bytes_read.sum","byte","1,000"\n'
+        '"0","k","dram__bytes_write.sum","byte","24"\n'
+        '"1","k","dram__bytes_read.sum","byte","7"\n'
+        '"1","k","dram__bytes_write.sum","byte","1"\n')
+    assert traffic.launch_bytes(str(log), 0) == 1024 and traffic.launch_bytes(str(log), 1) == 8
+    out = tmp_path / "traffic.json"
+    monkeypatch.setattr(traffic, "PATH", str(out))
+    traffic.main([f"a={log}:0", f"b={log}:1:8"])
+    assert traffic.load(str(out)) == {"a": 1024, "b": 64}
+    data = json.loads(out.read_text())
+    data["sources"] = "0" * 16
+    out.write_text(json.dumps(data))
+    assert traffic.load(str(out)) == {}

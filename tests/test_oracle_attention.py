@@ -167,6 +167,30 @@ def test_lazy_rescale_moves_the_reference_less_often():
     assert r8 < r0 and r8 == 0
 
 
+def test_lazy_rescale_per_row_moves_and_margins_by_hand():
+    """d = 1, q = 1, scale = ln 2 (so the base-2 logit of key j is k_j), blocks
+    of 2 keys.  Row maxima per block 0, 10, 15, 30: the reference starts at 0,
+    moves at block 1 (10 > 0 + 8, gap 2), stays at block 2 (15 < 10 + 8, gap
+    3), moves at block 3 (30 > 18, gap 12): two moves, margin 2."""
+    q = np.ones((1, 1, 1, 1))
+    k = np.array([0.0, -1.0, 10.0, 4.0, 15.0, 2.0, 30.0, 29.0]).reshape(1, 1, 8, 1)
+    v = np.arange(8.0).reshape(1, 1, 8, 1)
+    O, L, moves, margin = A.attention_lazy_rescale(q, k, v, False, math.log(2.0), 2, 8.0, rescale_rows=True)
+    assert moves[0, 0, 0] == 2 and abs(margin[0, 0, 0] - 2.0) < 1e-12
+    *_, total = A.attention_lazy_rescale(q, k, v, False, math.log(2.0), 2, 8.0, True)
+    assert total == 2
+    O2, L2 = A.attention(q, k, v, False, math.log(2.0))
+    np.testing.assert_allclose(O, O2, rtol=1e-12)
+
+
+def test_lazy_rescale_per_row_moves_sum_to_the_total():
+    q, k, v = rand(2, 2, 40, 8, scale=3.0), rand(2, 2, 70, 8, scale=3.0), rand(2, 2, 70, 8)
+    for causal in (False, True):
+        *_, total = A.attention_lazy_rescale(q, k, v, causal, 1.0, 8, 4.0, True)
+        *_, moves, margin = A.attention_lazy_rescale(q, k, v, causal, 1.0, 8, 4.0, rescale_rows=True)
+        assert moves.sum() == total and total > 0 and np.all(margin >= 0)
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3, 16, 40])
 def test_split_kv_combine_equals_unsplit(splits):
     q, k, v = rand(3, 2, 1, 16), rand(3, 2, 37, 16), rand(3, 2, 37, 16)

@@ -10,7 +10,7 @@ import math
 
 import torch
 
-from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_decode,  # noqa: F401
+from ._binding import (AttnError, LIB_PATH, attn_check_status, attn_debug_counters, attn_decode,  # noqa: F401
                        attn_decode_gqa, attn_decode_noalloc, attn_decode_workspace_bytes, attn_fp4_scores,
                        attn_fwd, attn_fwd_fp8, attn_fwd_gqa, attn_fwd_varlen, attn_decode_varlen, attn_quantize_fp8, attn_quantize_int4, attn_bwd, attn_bwd_fp8p, attn_bwd_workspace_bytes,
                        attn_fwd_fp4, attn_fwd_int8, attn_int8_scores, attn_nvfp4_codes_bytes,
@@ -26,7 +26,7 @@ __all__ = ["load", "attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "at
            "attn_bwd", "attn_bwd_fp8p", "attn_bwd_workspace_bytes", "backward",
            "attn_quantize_fp8", "attn_fwd_fp8", "quantize_fp8", "forward_fp8", "hadamard_signs",
            "attn_fwd_varlen", "attn_decode_varlen", "forward_varlen", "decode_varlen",
-           "DIRECT_P", "QUANT_AFTER_EXP"]
+           "attn_debug_counters", "DIRECT_P", "QUANT_AFTER_EXP"]
 
 DIRECT_P, QUANT_AFTER_EXP = 0, 1
 

@@ -19,7 +19,7 @@ LIB_PATH = os.environ.get("TILEDATTN_LIB") or os.path.join(_PKG, "libtiledattn.s
 ATTN_OK = 0
 STATUS_NAMES = {0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED",
                 -3: "ATTN_ERR_MISALIGNED", -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_TIMEOUT",
-                -6: "ATTN_ERR_TOO_LARGE"}
+                -6: "ATTN_ERR_TOO_LARGE", -7: "ATTN_ERR_BOUNDS"}
 
 # (name, restype, argtypes)
 _VP, _I, _F, _SZ, _ULL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_ulonglong
@@ -51,6 +51,7 @@ SIGNATURES = [
     ("attn_check_status", _I, [_VP]),
     ("attn_set_wait_limit_ns", None, [_ULL]),
     ("attn_watchdog_selftest", _I, [_ULL, _VP]),
+    ("attn_debug_counters", _I, [_VP, _I]),
 ]
 
 _lib = None
@@ -374,6 +375,15 @@ def attn_set_wait_limit_ns(ns: int) -> None:
 
 def attn_watchdog_selftest(limit_ns: int, stream=None) -> None:
     _check("attn_watchdog_selftest", load().attn_watchdog_selftest(int(limit_ns), _stream(stream)))
+
+
+def attn_debug_counters(reset: bool = False):
+    """The debug build's four counters (rescales, skipped causal tiles, bounds
+    violations, reserved); raises AttnError(ATTN_ERR_UNSUPPORTED) in the
+    product build."""
+    buf = (ctypes.c_ulonglong * 4)()
+    _check("attn_debug_counters", load().attn_debug_counters(ctypes.cast(buf, _VP), int(bool(reset))))
+    return [int(x) for x in buf]
 
 
 def attn_version() -> str:

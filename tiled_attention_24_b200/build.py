@@ -1,4 +1,5 @@
-"""Build libtiledattn.so (the attention library) and libtiledattn_probe.so
+"""Build libtiledattn.so (the attention library), libtiledattn_debug.so (the
+same with bounds checks and counters, TA_DEBUG = 1) and libtiledattn_probe.so
 (the throughput microbenchmarks behind the roofline denominators) in-tree
 with nvcc for sm_100a.
 
@@ -22,6 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtiledattn.so")
 SOURCES = ["api.cu"]
 PROBE_LIB = os.path.join(PKG, "libtiledattn_probe.so")
+DEBUG_LIB = os.path.join(PKG, "libtiledattn_debug.so")
 PROBE_SOURCES = ["probe.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -52,6 +54,15 @@ def build_probe(verbose: bool = False, force: bool = False) -> str:
     if not force and up_to_date(PROBE_LIB):
         return PROBE_LIB
     return build(verbose=verbose, force=True, out=PROBE_LIB, sources=PROBE_SOURCES)
+
+
+def build_debug(verbose: bool = False, force: bool = False) -> str:
+    """Compile libtiledattn_debug.so: the same library with TA_DEBUG = 1 (bounds
+    checks of every TMA coordinate and tensor-memory address, counters read by
+    attn_debug_counters)."""
+    if not force and up_to_date(DEBUG_LIB):
+        return DEBUG_LIB
+    return build(verbose=verbose, force=True, out=DEBUG_LIB, defines=["TA_DEBUG=1"])
 
 
 def build(verbose: bool = False, force: bool = False, out: str | None = None, defines=(),
@@ -88,3 +99,4 @@ if __name__ == "__main__":
     print(build(verbose=a.verbose, force=True, out=a.out, defines=a.defines))
     if a.out is None and not a.defines:
         print(build_probe(verbose=a.verbose, force=True))
+        print(build_debug(verbose=a.verbose, force=True))

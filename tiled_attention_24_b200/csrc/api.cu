@@ -345,6 +345,7 @@ const char* attn_status_string(int s) {
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
     case ATTN_ERR_TOO_LARGE: return "ATTN_ERR_TOO_LARGE";
+    case ATTN_ERR_BOUNDS: return "ATTN_ERR_BOUNDS";
     default: return "ATTN_ERR_UNKNOWN";
   }
 }
@@ -817,3 +818,16 @@ int attn_watchdog_selftest(unsigned long long limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+int attn_debug_counters(unsigned long long* out, int reset) {
+  if (!out) return ATTN_ERR_INVALID_ARG;
+  if (!TA_DEBUG) return ATTN_ERR_UNSUPPORTED;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(out, ta::g_attn_counters, sizeof(unsigned long long) * ta::TA_NCOUNTERS) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (reset) {
+    const unsigned long long zero[ta::TA_NCOUNTERS] = {};
+    if (cudaMemcpyToSymbol(ta::g_attn_counters, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}

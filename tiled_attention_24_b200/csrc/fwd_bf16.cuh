@@ -179,6 +179,8 @@ __global__ void __launch_bounds__(384, 1)
   }
   const int nmax = max(n[0], n[1]);
   volatile int* abort_flag = &bars->abort;
+  if (TA_DEBUG && threadIdx.x == 0 && p.causal)  // key tiles this CTA's query tiles never visit
+    debug_count(TA_CNT_SKIPPED_TILES, (present[0] ? Tc - n[0] : 0) + (present[1] ? Tc - n[1] : 0));
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
@@ -451,6 +453,10 @@ __global__ void __launch_bounds__(384, 1)
       const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
       // lazy rescale: move the reference max only when it rises by more than TAU
       const bool need = m_blk > m_ref + C::TAU;
+      if (TA_DEBUG) {  // rows whose reference moved after their first key block
+        const unsigned moved = __ballot_sync(__activemask(), need && m_ref != -INFINITY);
+        if (lane == 0) debug_count(TA_CNT_RESCALES, __popc(moved));
+      }
       float factor = 1.f;
       if (need) {
         factor = ex2(m_ref - m_blk);  // 0 when m_ref == -inf

@@ -111,6 +111,7 @@ struct FwdF4Bars {
 static_assert(sizeof(FwdF4Bars) <= 512, "barrier block too large");
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  if (!debug_check((dst & 15u) == 0 && (bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0)) return;
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
@@ -127,6 +128,7 @@ __device__ __forceinline__ uint64_t smem_desc_l(uint32_t saddr, uint32_t lbo, ui
 }
 // 32 rows x 16 bytes of shared memory -> TMEM, replicated to all 4 lane quarters
 __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  if (!debug_check((taddr >> 16) == 0 && (taddr & 0xFFFFu) + 4u <= 512u)) return;
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

@@ -68,6 +68,46 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // cleared by attn_check_status().
 __device__ int g_attn_status;
 
+// Debug build (TA_DEBUG = 1, libtiledattn_debug.so): counters read by
+// attn_debug_counters() -- lazy rescales of the bf16 forward (query rows whose
+// reference max moved after their first key block), KV tiles a causal CTA
+// skipped, and bounds violations -- and a check of every TMA coordinate and
+// tensor-memory address before the access.  A violation is counted, recorded
+// as ATTN_ERR_BOUNDS in the status word and the access is skipped (never a
+// trap); a wait it starves ends through the bounded waits.
+#ifndef TA_DEBUG
+#define TA_DEBUG 0
+#endif
+enum { TA_CNT_RESCALES = 0, TA_CNT_SKIPPED_TILES = 1, TA_CNT_BOUNDS = 2, TA_NCOUNTERS = 4 };
+__device__ unsigned long long g_attn_counters[TA_NCOUNTERS];
+
+__device__ __forceinline__ void debug_count(int which, unsigned long long n) {
+  if (TA_DEBUG && n) atomicAdd(&g_attn_counters[which], n);
+}
+// true when the access may proceed; in the debug build a failed check is
+// counted and reported (ATTN_ERR_BOUNDS) and the caller skips the access
+__device__ __forceinline__ bool debug_check(bool ok) {
+  if (!TA_DEBUG || ok) return true;
+  atomicAdd(&g_attn_counters[TA_CNT_BOUNDS], 1ull);
+  atomicExch(&g_attn_status, -7 /* ATTN_ERR_BOUNDS */);
+  return false;
+}
+// tensor memory: a 32x32b access of `cols` columns from this warp must stay in
+// its lane quarter and inside the 512 columns of an SM
+__device__ __forceinline__ bool tmem_ok(uint32_t taddr, uint32_t cols) {
+  if (!TA_DEBUG) return true;
+  const uint32_t lane = taddr >> 16, col = taddr & 0xFFFFu;
+  return debug_check(lane == 32u * ((threadIdx.x >> 5) & 3u) && col + cols <= 512u);
+}
+// TMA: the innermost coordinate a multiple of 16 elements (16 bytes for every
+// element size used here) and not negative; a store starts at no negative
+// coordinate; shared-memory side 128-byte aligned
+__device__ __forceinline__ bool tma_ok(uint32_t saddr, int c0, int c1, int c2, bool store) {
+  if (!TA_DEBUG) return true;
+  return debug_check((c0 & 15) == 0 && c0 >= 0 && (saddr & 127u) == 0 &&
+                     (!store || (c1 >= 0 && c2 >= 0)));
+}
+
 // Bounded wait on phase `parity` of an mbarrier.  `abort_flag` (shared) lets
 // one role that gave up release the others quickly.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -139,6 +179,7 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
                                             int c1, int c2) {
+  if (!tma_ok(dst, c0, c1, c2, false)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
@@ -147,6 +188,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int c0, int c1,
                                              int c2) {
+  if (!tma_ok(src, c0, c1, c2, true)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(m)),
@@ -234,6 +276,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 // 32 lanes x 32 columns of 32-bit TMEM cells: thread i of the warp gets lane
 // (base lane + i), columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (!tmem_ok(taddr, 32)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -259,6 +306,7 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  if (!tmem_ok(taddr, 32)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -272,7 +320,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 // One 32-bit TMEM column of 32 lanes (thread i: lane base + i).
 __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
-  uint32_t r;
+  uint32_t r = 0u;
+  if (!tmem_ok(taddr, 1)) return r;
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
   return r;
 }
@@ -280,10 +329,12 @@ __device__ __forceinline__ void tmem_ld_wait1(uint32_t& r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
 }
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  if (!tmem_ok(taddr, 1)) return;
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
 // 32 lanes x 16 columns (thread i: lane base + i, columns [col, col+16)).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  if (!tmem_ok(taddr, 16)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
