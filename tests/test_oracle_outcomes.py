@@ -352,3 +352,20 @@ def test_backward_fp8p_dv_interval_equals_brute_force():
     np.testing.assert_allclose(lo[0, 0], vals.min(axis=0), atol=1e-14)
     np.testing.assert_allclose(hi[0, 0], vals.max(axis=0), atol=1e-14)
     np.testing.assert_allclose(dv[0, 0], base.T @ do[0, 0], atol=1e-14)
+
+
+def test_a_planted_error_outside_the_interval_fails_the_check():
+    """The GPU tests' check (tests._parity.assert_within_outcomes) accepts
+    either realised rounding and rejects an output moved 2x the tolerance
+    beyond the interval."""
+    from tests._parity import Q_O_ABS, assert_within_outcomes
+    import torch
+    qi, qs, ki, ks, vi, vs = _int8_case(1.0)
+    O, L, R = Q.attention_int8(qi, qs, ki, ks, vi, vs, scale=LN2, outcomes=True)
+    n = 10_000  # the case is built to sit on a midpoint: keep the flag-rate check out of it
+    for nudge in (1 - 1e-6, 1 + 1e-6):
+        Oa, La = Q.attention_int8(*_int8_case(nudge), scale=LN2)
+        assert_within_outcomes(torch.from_numpy(Oa), torch.from_numpy(La), O, L, R, "realised", n)
+    bad = R.O_hi + 2 * Q_O_ABS
+    with pytest.raises(AssertionError):
+        assert_within_outcomes(torch.from_numpy(bad), torch.from_numpy(L), O, L, R, "planted", n)

@@ -19,6 +19,7 @@
 #include "fwd_fp4.cuh"
 #include "bwd_bf16.cuh"
 #include "fwd_fp8.cuh"
+#include "decode_tc.cuh"
 
 namespace {
 
@@ -41,16 +42,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH][N][d] bf16 viewed as a 3-D tensor (d, N, BH); boxes of 64 x 128 x 1
-// with 128-byte swizzle.  Rows past N read as zero and are not written.
-int make_tmap_bf16(CUtensorMap* m, const void* ptr, int d, int N, int BH) {
+// [BH][N][d] bf16 viewed as a 3-D tensor (d, N, BH); boxes of 64 x box_rows
+// x 1 with 128-byte swizzle.  Rows past N read as zero and are not written.
+int make_tmap_bf16(CUtensorMap* m, const void* ptr, int d, int N, int BH, int box_rows = 128) {
   auto enc = encode_fn();
   if (!enc) return ATTN_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// [rows][d] bf16 viewed as a 2-D tensor (d, rows); boxes of 64 x box_rows with
+// 128-byte swizzle.  Rows past `rows` read as zero.
+int make_tmap_rows(CUtensorMap* m, const void* ptr, int d, long long rows, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
@@ -334,6 +350,48 @@ __global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
 
 }  // namespace
 
+template <int G>
+static int launch_decode_tc_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, float* o_part,
+                              float* l_part, long long BH, int Nkv, int S, int chunk, float sl2, int grp,
+                              const int* seqlens, int H, cudaStream_t st) {
+  using C = ta::DecTcCfg;
+  if (cudaFuncSetAttribute(ta::decode_gqa_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const long long items = BH / G * S;
+  if (items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  // persistent: two CTAs per SM, each walking items with a stride of the grid
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const unsigned grid = (unsigned)std::min<long long>(items, 2LL * sms);
+  ta::decode_gqa_tc_kernel<G><<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, o_part, l_part, (int)items, Nkv, S,
+                                                                  chunk, sl2, grp, seqlens, H, g_wait_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Grouped-query decode on the tensor cores (d = 128): G query heads per CTA.
+static int launch_decode_tc(const void* q, const void* k, const void* v, float* o_part, float* l_part, int B, int H,
+                            int Hkv, int Nkv, int G, int S, int chunk, float sl2, int grp, const int* seqlens,
+                            cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_rows(&tq, q, 128, (long long)B * H, 8)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, 128, Nkv, B * Hkv, ta::DecTcCfg::KT)) != ATTN_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, 128, Nkv, B * Hkv, ta::DecTcCfg::KT)) != ATTN_OK) return rc;
+  const long long BH = (long long)B * H;
+  switch (G) {
+    case 8: return launch_decode_tc_g<8>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 7: return launch_decode_tc_g<7>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 6: return launch_decode_tc_g<6>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 5: return launch_decode_tc_g<5>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 4: return launch_decode_tc_g<4>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 3: return launch_decode_tc_g<3>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    case 2: return launch_decode_tc_g<2>(tq, tk, tv, o_part, l_part, BH, Nkv, S, chunk, sl2, grp, seqlens, H, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
 extern "C" {
 
 const char* attn_status_string(int s) {
@@ -499,6 +557,16 @@ static int decode_impl(const attn_bf16_t* q, const attn_bf16_t* k, const attn_bf
   // loads in flight: 1560 GB/s against 2260 as two CTAs of 4 (B64 Hq32
   // Hkv4 N_kv 8192 d128).
   const int grp = H / Hkv;
+  if (d == 128 && grp > 1) {
+    // tensor-core kernel: up to 8 query heads of a group per CTA (the largest
+    // divisor of the group that is <= 8)
+    int G = 8;
+    while (grp % G) --G;
+    int rc = launch_decode_tc(q, k, v, o_part, l_part, B, H, Hkv, Nkv, G, num_splits, chunk, sl2, grp, seqlens, st);
+    if (rc != ATTN_OK) return rc;
+    ta::decode_combine_kernel<128><<<(unsigned)BH, 128, 0, st>>>(o_part, l_part, o, lse, num_splits);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
   const int G = (grp % 4 == 0) ? 4 : (grp % 2 == 0) ? 2 : 1;
   const unsigned grid = (unsigned)(BH / G * num_splits);
   if (G == 1) {
