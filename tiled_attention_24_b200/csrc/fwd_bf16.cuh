@@ -58,6 +58,11 @@
 #ifndef TA_POLY_PAIRS
 #define TA_POLY_PAIRS 0
 #endif
+// P handed to the P V MMA in TA_P_SPLIT parts (1, 2 or 4) at d = 128
+#ifndef TA_P_SPLIT
+#define TA_P_SPLIT 2
+#endif
+#define TA_P_HALVES (TA_P_SPLIT > 1)
 #ifndef TA_POLY_PAIRS_D64
 #define TA_POLY_PAIRS_D64 TA_POLY_PAIRS
 #endif
@@ -112,6 +117,7 @@ struct FwdBars {
   uint64_t kv_empty[5];
   uint64_t s_full[2];
   uint64_t p_full[2];
+  uint64_t p_part[2][3];  // d = 128: P of the first k + 1 of TA_P_SPLIT key parts stored
   uint64_t o_full[2];
   uint64_t epi[2];
   uint64_t s_free[2];   // d = 64: scores of tile t are in registers
@@ -191,6 +197,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars->s_full[t]), 1);
       mbar_init(smem_u32(&bars->p_full[t]), 128);
+      for (int k = 0; k < 3; ++k) mbar_init(smem_u32(&bars->p_part[t][k]), 128);
       mbar_init(smem_u32(&bars->o_full[t]), 1);
       mbar_init(smem_u32(&bars->epi[t]), 128);
       mbar_init(smem_u32(&bars->s_free[t]), 128);
@@ -315,6 +322,23 @@ __global__ void __launch_bounds__(384, 1)
       auto need_tma = [&](bool seen, uint32_t bar, uint32_t par) -> bool {
         return seen || spin_bar(bar, par, abort_flag, p.timeout_ns);
       };
+      // d = 128 with P in TA_P_SPLIT parts: the MMAs of part k once the
+      // softmax has stored it, so the first parts run while it computes the rest
+      auto issue_PV_halves = [&](int t, int st, int j) -> bool {
+        const uint64_t dv = dV0 + (uint64_t)(st * (C::STAGE >> 4));
+        const uint32_t dO = tbase + C::T_O + t * D, aP = tbase + 128 * t;
+        const uint32_t acc0 = (j > 0) ? 1u : 0u;
+        constexpr int PER = 8 / TA_P_SPLIT;
+#pragma unroll
+        for (int k = 0; k < TA_P_SPLIT; ++k) {
+          const uint32_t bar = (k < TA_P_SPLIT - 1) ? smem_u32(&bars->p_part[t][k]) : smem_u32(&bars->p_full[t]);
+          if (!need(false, bar, j & 1)) return false;
+#pragma unroll
+          for (int kk = k * PER; kk < (k + 1) * PER; ++kk)
+            mma_f16_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), C::ID_PV, kk > 0 ? 1u : acc0);
+        }
+        return true;
+      };
       const uint32_t pf0 = smem_u32(&bars->p_full[0]), pf1 = smem_u32(&bars->p_full[1]);
       int st = 0;        // stage of the current step (slot), its phase
       uint32_t sp = 0;
@@ -377,15 +401,23 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t nbar = (j + 1 < nmax) ? smem_u32(&bars->kv_full[st1]) : 0u;
           bool seenP1 = false;
           if (j < n[0]) {
-            if (!(ok = need(false, pf0, j & 1))) break;
-            seenP1 = issue_PV(0, st, j, (j < n[1]) ? pf1 : 0u, j & 1);
+            if (TA_P_HALVES) {
+              if (!(ok = issue_PV_halves(0, st, j))) break;
+            } else {
+              if (!(ok = need(false, pf0, j & 1))) break;
+              seenP1 = issue_PV(0, st, j, (j < n[1]) ? pf1 : 0u, j & 1);
+            }
             if (j == n[0] - 1) tc_commit(smem_u32(&bars->o_full[0]));
           }
           if (j + 1 < n[0]) seenP1 = issue_S(0, st, (!seenP1 && j < n[1]) ? pf1 : 0u, j & 1) || seenP1;
           seenSt = false;
           if (j < n[1]) {
-            if (!(ok = need(seenP1, pf1, j & 1))) break;
-            seenSt = issue_PV(1, st, j, nbar, sp1);
+            if (TA_P_HALVES) {
+              if (!(ok = issue_PV_halves(1, st, j))) break;
+            } else {
+              if (!(ok = need(seenP1, pf1, j & 1))) break;
+              seenSt = issue_PV(1, st, j, nbar, sp1);
+            }
             if (j == n[1] - 1) tc_commit(smem_u32(&bars->o_full[1]));
           }
           if (j + 1 < n[1]) seenSt = issue_S(1, st, seenSt ? 0u : nbar, sp1) || seenSt;
@@ -500,6 +532,23 @@ __global__ void __launch_bounds__(384, 1)
             else lsA = fadd2(lsA, f2(p0, p1));
             pk[c >> 1][(c & 1) * 16 + i] = pack_bf16(p0, p1);
           }
+          if (TA_P_HALVES && !C::SEP_P && c < 3 && ((c + 1) % (4 / TA_P_SPLIT)) == 0) {
+            // keys up to 32 (c + 1): the MMA thread may start P V on this part
+            // now (its TMEM columns held scores already in registers)
+            constexpr int W = 64 / TA_P_SPLIT;  // TMEM columns (bf16 pairs) per part
+            const int k = (c + 1) / (4 / TA_P_SPLIT) - 1;
+            if (W == 32) {
+              tmem_st32(tP + 32 * k, pk[k]);
+            } else {
+              uint32_t q16[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) q16[i] = pk[c >> 1][(c & 1) * 16 + i];
+              tmem_st16(tP + 16 * c, q16);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_part[t][k]));
+          }
         }
       } else {
         // split the exponentials between the MUFU unit and the FMA pipes
@@ -530,8 +579,24 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
         }
       }
-      tmem_st32(tP, pk[0]);
-      tmem_st32(tP + 32, pk[1]);
+      if (TA_P_HALVES && !C::SEP_P && C::POLY_PAIRS != 0 && !(tail || diag)) {
+        // the split-exponent path stores all of P and releases its parts only here
+        tmem_st32(tP, pk[0]);
+        tmem_st32(tP + 32, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        for (int k = 0; k < TA_P_SPLIT - 1; ++k) mbar_arrive(smem_u32(&bars->p_part[t][k]));
+      } else if (!TA_P_HALVES || C::SEP_P) {
+        tmem_st32(tP, pk[0]);
+        tmem_st32(tP + 32, pk[1]);
+      } else if (TA_P_SPLIT == 2) {
+        tmem_st32(tP + 32, pk[1]);
+      } else {
+        uint32_t q16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q16[i] = pk[1][16 + i];
+        tmem_st16(tP + 48, q16);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full[t]));

@@ -75,21 +75,34 @@ __global__ void __launch_bounds__(256) quant_int8_rows_kernel(const uint16_t* __
 
 // Per-(batch, head) amax, accumulated with an integer atomicMax on the bit
 // pattern (valid for non-negative floats) into amax_bits[bh] (zeroed first).
+// Each thread keeps HEAD_UNROLL 16-byte loads in flight.
+constexpr int HEAD_UNROLL = 4;
+__device__ __forceinline__ float amax_bf16x8(const uint4& w, float m) {
+  m = fmaxf(m, fabsf(__uint_as_float(w.x << 16)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.x & 0xFFFF0000u)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.y << 16)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.y & 0xFFFF0000u)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.z << 16)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.z & 0xFFFF0000u)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.w << 16)));
+  m = fmaxf(m, fabsf(__uint_as_float(w.w & 0xFFFF0000u)));
+  return m;
+}
 __global__ void __launch_bounds__(256) head_amax_kernel(const uint16_t* __restrict__ x, unsigned* __restrict__ amax_bits,
                                                         long long per_head) {
   const int bh = blockIdx.y;
   const uint16_t* src = x + (long long)bh * per_head;
+  const long long stride = (long long)gridDim.x * 256 * 8;
   float m = 0.f;
-  for (long long i = ((long long)blockIdx.x * 256 + threadIdx.x) * 8; i < per_head; i += (long long)gridDim.x * 256 * 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(src + i);
-    m = fmaxf(m, fabsf(__uint_as_float(w.x << 16)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.x & 0xFFFF0000u)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.y << 16)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.y & 0xFFFF0000u)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.z << 16)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.z & 0xFFFF0000u)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.w << 16)));
-    m = fmaxf(m, fabsf(__uint_as_float(w.w & 0xFFFF0000u)));
+  for (long long i0 = ((long long)blockIdx.x * 256 + threadIdx.x) * 8; i0 < per_head; i0 += HEAD_UNROLL * stride) {
+    uint4 w[HEAD_UNROLL];
+#pragma unroll
+    for (int u = 0; u < HEAD_UNROLL; ++u) {
+      const long long i = i0 + u * stride;
+      w[u] = (i < per_head) ? *reinterpret_cast<const uint4*>(src + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < HEAD_UNROLL; ++u) m = amax_bf16x8(w[u], m);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -111,16 +124,26 @@ __global__ void __launch_bounds__(256) quant_int8_heads_kernel(const uint16_t* _
   const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 127.f);
   const uint16_t* src = x + (long long)bh * per_head;
   int8_t* dst = xq + (long long)bh * per_head;
-  for (long long i = ((long long)blockIdx.x * 256 + threadIdx.x) * 8; i < per_head; i += (long long)gridDim.x * 256 * 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(src + i);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    uint32_t out[2] = {0, 0};
+  const long long stride = (long long)gridDim.x * 256 * 8;
+  for (long long i0 = ((long long)blockIdx.x * 256 + threadIdx.x) * 8; i0 < per_head; i0 += HEAD_UNROLL * stride) {
+    uint4 w[HEAD_UNROLL];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t bits = (e & 1) ? (ws[e >> 1] & 0xFFFF0000u) : (ws[e >> 1] << 16);
-      out[e >> 2] |= (uint32_t)(uint8_t)q8(__uint_as_float(bits), s) << (8 * (e & 3));
+    for (int u = 0; u < HEAD_UNROLL; ++u) {
+      const long long i = i0 + u * stride;
+      w[u] = (i < per_head) ? *reinterpret_cast<const uint4*>(src + i) : make_uint4(0, 0, 0, 0);
     }
-    *reinterpret_cast<uint2*>(dst + i) = make_uint2(out[0], out[1]);
+#pragma unroll
+    for (int u = 0; u < HEAD_UNROLL; ++u) {
+      const long long i = i0 + u * stride;
+      const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+      uint32_t out[2] = {0, 0};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t bits = (e & 1) ? (ws[e >> 1] & 0xFFFF0000u) : (ws[e >> 1] << 16);
+        out[e >> 2] |= (uint32_t)(uint8_t)q8(__uint_as_float(bits), s) << (8 * (e & 3));
+      }
+      if (i < per_head) *reinterpret_cast<uint2*>(dst + i) = make_uint2(out[0], out[1]);
+    }
   }
 }
 
@@ -334,14 +357,20 @@ __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const uint16_t* __r
 template <int D>
 __global__ void __launch_bounds__(256) channel_amax_kernel(const uint16_t* __restrict__ x,
                                                            unsigned* __restrict__ amax_bits, int N) {
-  constexpr int G = D / 8, R = 256 / G;  // channel groups, token rows per pass
+  constexpr int G = D / 8, R = 256 / G, PASSES = 128 / R;  // channel groups, token rows per pass
   const int bh = blockIdx.y, g = threadIdx.x % G, r = threadIdx.x / G;
   const int n0 = blockIdx.x * 128, n1 = min(N, n0 + 128);
   const uint16_t* src = x + ((size_t)bh * N) * D + g * 8;
+  uint4 w[PASSES];  // every load of the thread in flight at once
+#pragma unroll
+  for (int k = 0; k < PASSES; ++k) {
+    const int n = n0 + r + k * R;
+    w[k] = (n < n1) ? *reinterpret_cast<const uint4*>(src + (size_t)n * D) : make_uint4(0, 0, 0, 0);
+  }
   float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int n = n0 + r; n < n1; n += R) {
-    const uint4 w = *reinterpret_cast<const uint4*>(src + (size_t)n * D);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < PASSES; ++k) {
+    const uint32_t u[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(u[i] << 16)));
@@ -363,20 +392,27 @@ template <int D>
 __global__ void __launch_bounds__(256) channel_codes_kernel(const uint16_t* __restrict__ x,
                                                             const unsigned* __restrict__ amax_bits,
                                                             uint8_t* __restrict__ codes, int N) {
-  constexpr int G = D / 8, R = 256 / G;
+  constexpr int G = D / 8, R = 256 / G, PASSES = 128 / R;
   const int bh = blockIdx.y, g = threadIdx.x % G, r = threadIdx.x / G;
   const int n0 = blockIdx.x * 128, n1 = min(N, n0 + 128);
+  const uint16_t* src = x + ((size_t)bh * N) * D + g * 8;
+  uint8_t* dst = codes + ((size_t)bh * N) * D + g * 8;
+  uint4 w[PASSES];
+#pragma unroll
+  for (int k = 0; k < PASSES; ++k) {
+    const int n = n0 + r + k * R;
+    w[k] = (n < n1) ? *reinterpret_cast<const uint4*>(src + (size_t)n * D) : make_uint4(0, 0, 0, 0);
+  }
   float sc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float a = __uint_as_float(amax_bits[(size_t)bh * D + g * 8 + i]);
     sc[i] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
   }
-  const uint16_t* src = x + ((size_t)bh * N) * D + g * 8;
-  uint8_t* dst = codes + ((size_t)bh * N) * D + g * 8;
-  for (int n = n0 + r; n < n1; n += R) {
-    const uint4 w = *reinterpret_cast<const uint4*>(src + (size_t)n * D);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < PASSES; ++k) {
+    const int n = n0 + r + k * R;
+    const uint32_t u[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
     uint32_t out[2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -387,7 +423,7 @@ __global__ void __launch_bounds__(256) channel_codes_kernel(const uint16_t* __re
       else
         out[i >> 1] = pr;
     }
-    *reinterpret_cast<uint2*>(dst + (size_t)n * D) = make_uint2(out[0], out[1]);
+    if (n < n1) *reinterpret_cast<uint2*>(dst + (size_t)n * D) = make_uint2(out[0], out[1]);
   }
 }
 
