@@ -43,9 +43,16 @@ def test_fwd_gqa_equals_expanded_heads(cuda_lib):
     assert bool((o1 == o2).all()) and bool((l1 == l2).all())
 
 
-# (query heads per cache head -> heads per CTA): 4 -> 4, 8 -> 8, 3 -> 1 (plain kernel), 2 -> 2
+# (B, Hq, Hkv, Nkv, d, splits).  d = 128 runs the tensor-core kernel with G
+# query heads per work item, G the largest divisor of the group <= 8: groups
+# 4, 8, 3, 16 (two items per cache head), 5 and 7; chunks shorter than a 64-key
+# tile, chunks with no key at all (splits > Nkv), one exact tile, and more
+# items than CTAs (persistent CTAs take several).  d = 64 runs the CUDA-core
+# kernel (groups of 8 -> CTAs of 4, 2 -> 2).
 @pytest.mark.parametrize("shape", [(4, 32, 8, 3000, 128, 16), (2, 8, 1, 8192, 64, 7), (3, 6, 2, 100, 128, 16),
-                                   (2, 6, 3, 2000, 64, 5), (1, 16, 2, 700, 128, 1)],
+                                   (2, 6, 3, 2000, 64, 5), (1, 16, 2, 700, 128, 1), (1, 16, 1, 1000, 128, 4),
+                                   (2, 10, 2, 513, 128, 3), (1, 7, 1, 64, 128, 2), (2, 8, 2, 5, 128, 16),
+                                   (8, 32, 4, 4096, 128, 32)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_decode_gqa(cuda_lib, shape):
     B, Hq, Hkv, Nkv, d, splits = shape

@@ -665,7 +665,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int h = 0; h < D / 64; ++h)
             tma_store_3d(&tmO, sbase + C::Q_OFF + t * C::TILE + h * C::HALF, h * 64, r0[t], bh);
           bulk_commit();
-          bulk_wait_all();
+          bulk_wait_read();  // the CTA may exit once the tile has left shared memory
         }
       }
       __syncwarp();
