@@ -18,17 +18,18 @@
 // O = (OF + ACC * s_V / 127) / l (fp32 output) and LSE = ln2 * (m + log2 l).
 //
 // CTA = one (batch, head) x one 128-row query tile.  Warps: 0 TMA producer,
-// 1 MMA issuer, 2-9 softmax/fold/epilogue: TMEM lane quarter q is read by two
-// warps, one taking key columns [0, 64) of every block (warps 2-5), the other
-// [64, 128) (warps 6-9); the two threads of a row exchange their partial row
-// max once per block through a tagged shared-memory slot (xchg_put/get).
-// Two softmax warps per SM sub-partition give the scheduler a second
-// instruction stream while one waits on a dependency.
+// 1 MMA issuer, then NPART groups of four softmax/fold/epilogue warps: TMEM
+// lane quarter q is read by NPART warps, group g taking key columns
+// [CW g, CW g + CW) of every block (CW = 128 / NPART) and output columns
+// [CW g, CW g + CW) of O; the NPART threads of a row exchange their partial
+// row max once per block through tagged shared-memory slots (xchg_put/get).
+// NPART softmax warps per SM sub-partition give the scheduler NPART
+// instruction streams while each waits on its dependency chain.
 // TMEM: S_0 cols [0,128), S_1 [128,256) (double-buffered scores, so S_{j+1}
 // is computed while block j is in the softmax), ACC [256,384) int32,
-// OF [384,512) fp32.  P8_j lives inside S_{j%2}: keys [0, 64) in columns
-// [0, 16) and keys [64, 128) in columns [64, 80), so each half writes only
-// columns it has itself read.
+// OF [384,512) fp32.  P8_j lives inside S_{j%2}: keys [CW g, CW g + CW) in
+// columns [CW g, CW g + CW / 4), so each group writes only columns it has
+// itself read.
 // Shared memory: Q tile (128 x 128 int8 = 16 KB) and a ring of K/V tiles,
 // 128-byte swizzled.  d = 128 only.
 #pragma once
@@ -58,17 +59,25 @@ __host__ __device__ constexpr uint32_t idesc_i8(int N, bool b_mn) {
          ((uint32_t)(128 >> 4) << 24);
 }
 
+// softmax warps per TMEM lane quarter: each takes CW = 128 / I8_PARTS key
+// columns of a block (and the same number of output columns of O)
+#ifndef TA_I8_PARTS
+#define TA_I8_PARTS 2
+#endif
 struct FwdI8Cfg {
   static constexpr int D = 128;
   static constexpr int TILE = 128 * 128;  // bytes of a 128 x 128 int8 tile
   static constexpr int NSLOT = 8;
+  static constexpr int NPART = TA_I8_PARTS, CW = 128 / NPART, NCH = CW / 32;  // parts, columns, 32-col chunks
+  static constexpr int NSW = 4 * NPART;                                     // softmax warps
   static constexpr int Q_OFF = 0;
   static constexpr int SLOT_OFF = TILE;
-  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;  // [8 warps][2 bufs][64] floats
-  static constexpr int XCH_OFF = KC_OFF + 8 * 2 * 64 * 4;  // [3 slots][2 halves][128 rows] u64
-  static constexpr int BAR_OFF = XCH_OFF + 3 * 2 * 128 * 8;
+  static constexpr int KC_OFF = SLOT_OFF + NSLOT * TILE;                    // [NSW warps][2 bufs][CW] floats
+  static constexpr int XCH_OFF = KC_OFF + NSW * 2 * CW * 4;                 // [3 slots][NPART][128 rows] u64
+  static constexpr int BAR_OFF = XCH_OFF + 3 * NPART * 128 * 8;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 64 + 32 * NSW;
+  static_assert(NPART == 2 || NPART == 4, "two or four softmax warps per lane quarter");
   static constexpr uint32_t ID_S = idesc_i8(128, false);
   static constexpr uint32_t ID_PV = idesc_i8(128, true);  // V is MN-major
 };
@@ -110,7 +119,7 @@ __device__ __forceinline__ float i2f_small(uint32_t v) {
 }
 
 template <bool SCORES_ONLY>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FwdI8Cfg::THREADS, 1)
     fwd_int8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdI8Params p) {
   using C = FwdI8Cfg;
@@ -135,8 +144,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(smem_u32(&bars->s_full[0]), 1);
     mbar_init(smem_u32(&bars->s_full[1]), 1);
-    mbar_init(smem_u32(&bars->p_full[0]), 256);
-    mbar_init(smem_u32(&bars->p_full[1]), 256);
+    mbar_init(smem_u32(&bars->p_full[0]), 32 * C::NSW);
+    mbar_init(smem_u32(&bars->p_full[1]), 32 * C::NSW);
     mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(320, 1)
   {
     // exchange slots start with tag 0 (no block uses it), whatever a previous CTA left
     unsigned long long* xz = reinterpret_cast<unsigned long long*>(smem + C::XCH_OFF);
-    for (int i = threadIdx.x; i < 3 * 2 * 128; i += C::THREADS) xz[i] = 0ull;
+    for (int i = threadIdx.x; i < 3 * C::NPART * 128; i += C::THREADS) xz[i] = 0ull;
   }
   tc_fence_before();
   __syncthreads();
@@ -224,9 +233,12 @@ __global__ void __launch_bounds__(320, 1)
         const uint64_t dv = dV0 + (uint64_t)(s * (C::TILE >> 4));
         const uint32_t acc0 = (j > 0) ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // 32 keys per MMA: 32 rows x 128 B of V
-          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + (kk >> 1) * 64 + (kk & 1) * 8,
-                    dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV, kk > 0 ? 1u : acc0);
+        for (int kk = 0; kk < 4; ++kk) {  // 32 keys per MMA: 32 rows x 128 B of V
+          // keys [32 kk, 32 kk + 32): part 32 kk / CW, P8 at its first columns
+          const uint32_t col = (32 * kk / C::CW) * C::CW + (32 * kk % C::CW) / 4;
+          mma_i8_ts(tbase + 256, tbase + (j & 1) * 128 + col, dv + (uint64_t)(kk * (4096 >> 4)), C::ID_PV,
+                    kk > 0 ? 1u : acc0);
+        }
         tc_commit(smem_u32(&bars->pv_done));
         tc_commit(smem_u32(&bars->kv_empty[s]));
         if (j == n - 1) tc_commit(smem_u32(&bars->o_full));
@@ -247,15 +259,17 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ================================================================ softmax
-    const int half = (warp - 2) >> 2;  // key columns [64 half, 64 half + 64) of every block
+    constexpr int NCH = C::NCH, CW = C::CW, KPL = CW / 32;  // 32-column chunks, columns, keys per lane
+    const int part = (warp - 2) >> 2;  // key columns [CW part, CW part + CW) of every block
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;
     const int row = r0 + rr;
-    const int cb = half * 64;
+    const int cb = part * CW;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tACC = tbase + lane_off + 256 + cb;
     const uint32_t tOF = tbase + lane_off + 384 + cb;
-    // exchange slots: [0], [1] row max of even / odd blocks, [2] final l share
+    // exchange slots: [0], [1] row max of even / odd blocks, [2] final l share;
+    // each [NPART][128 rows]
     unsigned long long* xch = reinterpret_cast<unsigned long long*>(smem + C::XCH_OFF);
     const int off = p.Nkv - p.Nq;
     const float qs_row = (!SCORES_ONLY && row < p.Nq) ? p.q_scale[(size_t)bh * p.Nq + row] : 0.f;
@@ -263,21 +277,23 @@ __global__ void __launch_bounds__(320, 1)
     const float* ksrow = p.k_scale + (size_t)bh * p.Nkv;
     // Per-column constants of a key block, kc = s_K * scale * log2(e), kept in
     // this warp's own shared buffer (x / s_Q = S * kc).  Lane l owns columns
-    // cb + [2l, 2l + 2); the next block's scales are loaded one block ahead.
-    float* kcbuf = reinterpret_cast<float*>(smem + C::KC_OFF) + (warp - 2) * (2 * 64);
-    float2 ks_next = make_float2(0.f, 0.f);
+    // cb + [KPL l, KPL l + KPL); the next block's scales are loaded one block ahead.
+    float* kcbuf = reinterpret_cast<float*>(smem + C::KC_OFF) + (warp - 2) * (2 * CW);
+    float ks_next[KPL];
     auto load_ks = [&](int jj) {
-      const int c0 = jj * 128 + cb + lane * 2;
-      if (p.ks_vec && c0 + 1 < p.Nkv) {
-        ks_next = __ldg(reinterpret_cast<const float2*>(ksrow + c0));
+      const int c0 = jj * 128 + cb + lane * KPL;
+      if (KPL == 2 && p.ks_vec && c0 + 1 < p.Nkv) {
+        const float2 v2 = __ldg(reinterpret_cast<const float2*>(ksrow + c0));
+        ks_next[0] = v2.x;
+        ks_next[KPL - 1] = v2.y;
       } else {
-        ks_next.x = (c0 + 0 < p.Nkv) ? ksrow[c0 + 0] : 0.f;
-        ks_next.y = (c0 + 1 < p.Nkv) ? ksrow[c0 + 1] : 0.f;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) ks_next[k] = (c0 + k < p.Nkv) ? ksrow[c0 + k] : 0.f;
       }
     };
     auto stage_ks = [&](int jj) {
-      *reinterpret_cast<float2*>(kcbuf + (jj & 1) * 64 + lane * 2) =
-          make_float2(ks_next.x * p.sl2, ks_next.y * p.sl2);
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) kcbuf[(jj & 1) * CW + lane * KPL + k] = ks_next[k] * p.sl2;
     };
     if (!SCORES_ONLY && n > 0) {
       load_ks(0);
@@ -285,14 +301,14 @@ __global__ void __launch_bounds__(320, 1)
       if (n > 1) load_ks(1);
       __syncwarp();
     }
-    float m_ref = -INFINITY, l = 0.f;  // l: this thread's share (its 64 columns)
+    float m_ref = -INFINITY, l = 0.f;  // l: this thread's share (its CW columns)
     bool ok = true;
     if (!SCORES_ONLY) {
       uint32_t z[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) z[i] = 0u;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) tmem_st32(tOF + cc * 32, z);
+      for (int cc = 0; cc < NCH; ++cc) tmem_st32(tOF + cc * 32, z);
       tmem_st_wait();
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -302,16 +318,16 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tS = tbase + lane_off + (j & 1) * 128 + cb;
-      uint32_t s[2][32];
-      tmem_ld32(tS, s[0]);
-      tmem_ld32(tS + 32, s[1]);
-      tmem_ld_wait(s[0]);
-      tmem_ld_wait(s[1]);
+      uint32_t s[NCH][32];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) tmem_ld32(tS + c * 32, s[c]);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) tmem_ld_wait(s[c]);
       if (SCORES_ONLY) {
         if (row < p.Nq) {
           int* dst = p.s_out + ((size_t)bh * p.Nq + row) * p.Nkv + kb + cb;
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < NCH; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               if (kb + cb + c * 32 + i < p.Nkv) dst[c * 32 + i] = (int)s[c][i];
@@ -329,11 +345,11 @@ __global__ void __launch_bounds__(320, 1)
         if (p.causal) lim = min(lim, row + off - kb);
       }
       lim -= cb;
-      const float* kcb = kcbuf + (j & 1) * 64;
-      float x[2][32];
+      const float* kcb = kcbuf + (j & 1) * CW;
+      float x[NCH][32];
       const uint64_t negM2 = f2(-12582912.f, -12582912.f);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < NCH; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 kc = *reinterpret_cast<const float4*>(kcb + c * 32 + i);
@@ -348,7 +364,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (tail || diag) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < NCH; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > lim) x[c][i] = -INFINITY;
@@ -358,24 +374,32 @@ __global__ void __launch_bounds__(320, 1)
         stage_ks(j + 1);
         if (j + 2 < n) load_ks(j + 2);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        mx0 = fmax3(mx0, x[0][i], x[0][i + 1]);
-        mx1 = fmax3(mx1, x[1][i], x[1][i + 1]);
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          mxa = fmax3(mxa, x[c][i], x[c][i + 1]);
+          mxb = fmax3(mxb, x[c][i + 2], x[c][i + 3]);
+        }
+      // row max over the NPART parts.  Slot j % 2 is rewritten for block j + 2
+      // only after this thread read every partner's block j + 1 value, which
+      // each partner writes after reading ours for block j.
+      const float my_max = fmaxf(mxa, mxb);
+      float row_max = my_max;
+      unsigned long long* xj = xch + (j & 1) * (C::NPART * 128);
+      xchg_put(xj + part * 128 + rr, (uint32_t)j + 1u, my_max);
+#pragma unroll
+      for (int q = 1; q < C::NPART; ++q) {
+        float other;
+        const int pq = (part + q) % C::NPART;
+        ok = ok && xchg_get(xj + pq * 128 + rr, (uint32_t)j + 1u, other, abort_flag, p.timeout_ns);
+        row_max = fmaxf(row_max, ok ? other : row_max);
       }
-      // row max over both halves.  Slot j % 2 is rewritten for block j + 2
-      // only after this thread read the partner's block j + 1 value, which the
-      // partner writes after reading ours for block j.
-      const float my_max = fmaxf(mx0, mx1);
-      float other_max;
-      xchg_put(xch + (j & 1) * 256 + half * 128 + rr, (uint32_t)j + 1u, my_max);
-      ok = xchg_get(xch + (j & 1) * 256 + (half ^ 1) * 128 + rr, (uint32_t)j + 1u, other_max, abort_flag,
-                    p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       // s_Q > 0, so max(y) * s_Q is the row max of x
-      const float m_blk = fmaxf(my_max, other_max) * qs_row;
+      const float m_blk = row_max * qs_row;
       // tau = 0: move the reference on every increase
       const bool grow = m_blk > m_ref;
       const bool had = m_ref != -INFINITY;  // rows with earlier content need a fold
@@ -391,9 +415,9 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t qs2 = f2(qs_row, qs_row), nm2 = f2(negm, negm);
       const uint64_t mg2 = f2(12582912.f, 12582912.f);
       uint32_t isum = 0;
-      uint32_t pk[16];
+      uint32_t pk[CW / 4];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < NCH; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           float a0, a1, a2, a3;
@@ -410,8 +434,15 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       l += (float)isum * (1.f / 127.f);
-      // P8 of keys [cb, cb + 64) -> columns [cb, cb + 16) of this block's score buffer
-      tmem_st16(tS, pk);
+      // P8 of keys [cb, cb + CW) -> columns [cb, cb + CW / 4) of this block's score buffer
+      if (CW == 32) {
+        tmem_st8(tS, pk);
+      } else {
+        uint32_t p16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p16[i] = pk[i % (CW / 4)];
+        tmem_st16(tS, p16);
+      }
       if (j > 0 && __any_sync(0xffffffffu, grow && had)) {
         // fold ACC (P V of blocks < j, reference m_old) into OF
         ok = wait_bar(smem_u32(&bars->pv_done), (j - 1) & 1, abort_flag, p.timeout_ns);
@@ -420,7 +451,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const float f = (grow && had) ? factor : 1.f;
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < NCH; ++cc) {
           uint32_t a[32], o[32];
           tmem_ld32(tACC + cc * 32, a);
           tmem_ld32(tOF + cc * 32, o);
@@ -446,18 +477,25 @@ __global__ void __launch_bounds__(320, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (!SCORES_ONLY && ok) {
-      float l_other;
-      xchg_put(xch + 2 * 256 + half * 128 + rr, 1u, l);
-      ok = xchg_get(xch + 2 * 256 + (half ^ 1) * 128 + rr, 1u, l_other, abort_flag, p.timeout_ns);
+      unsigned long long* xl = xch + 2 * (C::NPART * 128);
+      xchg_put(xl + part * 128 + rr, 1u, l);
+      float lt = l;
+#pragma unroll
+      for (int q = 1; q < C::NPART; ++q) {
+        float other;
+        const int pq = (part + q) % C::NPART;
+        ok = ok && xchg_get(xl + pq * 128 + rr, 1u, other, abort_flag, p.timeout_ns);
+        lt += ok ? other : 0.f;
+      }
       ok = __all_sync(0xffffffffu, ok);
-      l += l_other;
+      l = lt;
     }
     if (!SCORES_ONLY && ok) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       float* orow = p.o + ((size_t)bh * p.Nq + row) * C::D + cb;
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < NCH; ++cc) {
         uint32_t a[32], o[32];
         tmem_ld32(tACC + cc * 32, a);
         tmem_ld32(tOF + cc * 32, o);
@@ -475,7 +513,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      if (half == 0 && row < p.Nq)
+      if (part == 0 && row < p.Nq)
         p.lse[(size_t)bh * p.Nq + row] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
