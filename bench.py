@@ -714,7 +714,8 @@ def run_ours(args):
                 "frac": pn["rate"] / peak_tc, "traffic": traffic.get("fwd_bf16_prefill_noncausal"),
                 "kernel": "fwd_bf16_kernel<128>, prefill B4 H16 N4096 d128 non-causal",
                 "peak_source": f"{peak_src} bf16 burst"}
-    for part, key in (("decode", "decode_split"), ("longseq_noncausal", "fwd_bf16_longseq_noncausal"),
+    for part, key in (("decode", "decode_split"), ("decode_gqa", "decode_gqa_tc"), ("lowp_bf16", "fwd_bf16_lowp"),
+                      ("longseq_noncausal", "fwd_bf16_longseq_noncausal"),
                       ("longseq_causal", "fwd_bf16_longseq_causal"), ("prefill_varlen_causal", "fwd_bf16_varlen_causal"),
                       ("prefill_noncausal", "fwd_bf16_prefill_noncausal"),
                       ("prefill_causal", "fwd_bf16_prefill_causal"), ("lowp_int8", "fwd_int8_lowp"),
@@ -771,7 +772,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="reference arm: oracle seconds per step cap")
-    ap.add_argument("--cpu-rows", type=int, default=48, help="query rows per (batch, head) in the oracle leg")
+    ap.add_argument("--cpu-rows", type=int, default=160, help="query rows per (batch, head) in the oracle leg")
     ap.add_argument("--no-probe", action="store_true", help="skip the tensor-peak microbenchmarks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="prefill,decode,longseq,lowp",
