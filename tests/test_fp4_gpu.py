@@ -168,3 +168,32 @@ def test_fp4_full_lowp_workload_sampled_rows(cuda_lib, mode):
         O, L, R = Q.attention_fp4(qd[:, :, rows], kd, vd, mode, False, w.scale, outcomes=True)
         assert_within_outcomes(og[b:b + 1, h:h + 1, rows], lg[b:b + 1, h:h + 1, rows], O, L, R,
                                f"fp4 mode {mode} lowp full b={b} h={h}", rows.size * w.Nkv)
+
+
+def test_nvfp4_quantiser_exact_on_rounding_ties(cuda_lib):
+    """Blocks whose quotients land exactly on e2m1 rounding midpoints (block
+    amax 6 * 2^k, so the e4m3 scale is 2^k, and x = midpoint * 2^k), the case
+    where a divide-free quotient could round the other way; rows (Q/K) and
+    token blocks (V), codes and scales bit-exact against the oracle."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    N = 128
+    x64 = np.zeros((2, N, 128))
+    for h in range(2):
+        for n in range(N):
+            k = (n % 7) - 3
+            r = np.resize(np.concatenate([[6.0], mids, -mids]), 128) * 2.0 ** k * (1 if h == 0 else -1)
+            r[::16] = 6.0 * 2.0 ** k                            # every 16-block holds its amax
+            x64[h, n] = np.roll(r, n % 16)
+    x = torch.tensor(x64, dtype=torch.float32).reshape(1, 2, N, 128).to(torch.bfloat16)
+    assert (x.float().numpy().reshape(2, N, 128) == x64).all()
+    codes, sf = G.quantize_nvfp4(cuda_lib, x.cuda(), 0)
+    assert cuda_lib.attn_check_status() == 0
+    rc, rs = Q.quantize_nvfp4(x, axis=-1)
+    assert np.array_equal(unpack_codes(codes, (2, N, 128)).reshape(1, 2, N, 128), rc)
+    assert np.array_equal(untile_sf(sf, 2, 1)[:, :N].reshape(1, 2, N, 8), rs)
+    xt = x.transpose(-1, -2).contiguous()                       # V: the same values along tokens
+    vc, vs = G.quantize_nvfp4(cuda_lib, xt.cuda(), 1)
+    assert cuda_lib.attn_check_status() == 0
+    rvc, _ = Q.quantize_nvfp4(xt, axis=-2)
+    got_vc = unpack_codes(vc, (2, 128, N)).reshape(1, 2, 128, N)
+    assert np.array_equal(np.swapaxes(got_vc, -1, -2), rvc)

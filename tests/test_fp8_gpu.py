@@ -128,3 +128,42 @@ def test_fp8_package_forward(cuda_lib):
     Oe, Le = A.attention(q, k, v, True, 128 ** -0.5)
     assert np.abs(_np(o) - Oe).max() < 0.1
     assert np.isfinite(_np(lse)).all()
+
+
+def test_fp8_quantisers_exact_on_rounding_ties(cuda_lib):
+    """Rows and channels whose quotients land exactly on e4m3 rounding
+    midpoints (amax = 448 * 2^k, so s = 2^k, and x = midpoint * 2^k), the case
+    where a divide-free quotient could round the other way: codes and scales
+    bit-exact against the oracle."""
+    from oracle.lowp import UE4M3_VALUES
+    grid = np.asarray(UE4M3_VALUES, dtype=np.float64)
+    mids = (grid[1:] + grid[:-1]) / 2
+    mids = mids[(mids > 2.0 ** -6) & (mids < 448)]
+    rows = []
+    for k in (-4, 0, 3):
+        for sign in (1.0, -1.0):
+            r = np.zeros(128)
+            r[0] = 448.0 * 2.0 ** k
+            sel = mids[np.linspace(0, mids.size - 1, 127).astype(int)]
+            r[1:] = sign * sel * 2.0 ** k
+            rows.append(r)
+    x64 = np.stack(rows)
+    x = torch.tensor(x64, dtype=torch.float32).reshape(1, 2, -1, 128).to(torch.bfloat16)
+    assert (x.float().numpy().reshape(-1, 128) == x64).all()    # midpoints are exact in bf16
+    codes, sc = G.quantize_fp8(cuda_lib, x.cuda(), 0)
+    assert cuda_lib.attn_check_status() == 0
+    rv, rs = F.quantize_fp8_rows(x, None)
+    assert np.array_equal(_np(sc), rs)
+    assert np.array_equal(_values(codes), rv)
+    # channels: token n of channel c holds pattern[n] * 2^k(c), pattern[0] = 448
+    pat = np.concatenate([[448.0], mids[np.linspace(0, mids.size - 1, 127).astype(int)]])
+    kc = np.array([(-4, 0, 3)[c % 3] for c in range(128)])
+    sgn = np.where(np.arange(128) % 2, -1.0, 1.0)
+    v64 = pat[:, None] * (2.0 ** kc)[None, :] * sgn[None, :]
+    v = torch.tensor(np.stack([v64, -v64]), dtype=torch.float32).reshape(1, 2, 128, 128).to(torch.bfloat16)
+    assert (v.float().numpy().reshape(2, 128, 128) == np.stack([v64, -v64])).all()
+    codes, sc = G.quantize_fp8(cuda_lib, v.cuda(), 1)
+    assert cuda_lib.attn_check_status() == 0
+    rv, rs = F.quantize_fp8_channels(v)
+    assert np.array_equal(_np(sc), rs)
+    assert np.array_equal(_values(codes), rv)

@@ -134,3 +134,27 @@ def test_int4_full_lowp_workload_sampled_rows(cuda_lib):
     rows = np.array(sorted({0, 1, 127, 128, 8191} | set(np.random.default_rng(2).choice(8192, 11).tolist())))
     _, flips, cos = _check_int8(cuda_lib, q, k, v, False, w.scale, rows=rows, what="int4 lowp full", int4=True)
     print(f"int4 lowp: cosine vs fp64 {cos:.4f}, boundary elements {flips}")
+
+
+def test_quantisers_exact_on_rounding_ties(cuda_lib):
+    """Rows whose quotients x / s land exactly on half-integers (amax = 127 *
+    2^k, so s = 2^k, and x = (j + 1/2) 2^k): every element is a rounding tie
+    (round half to even), the case where a divide-free quotient could round
+    the other way.  Codes and scales bit-exact against the oracle."""
+    rows = []
+    for k in range(-6, 7, 3):
+        for sign in (1.0, -1.0):
+            r = np.empty(128, dtype=np.float32)
+            r[0] = 127.0 * 2.0 ** k
+            j = np.arange(127)
+            r[1:] = sign * (j + 0.5) * 2.0 ** k * np.where(j % 2, -1.0, 1.0)
+            rows.append(r)
+    x = torch.tensor(np.stack(rows)).reshape(1, 2, -1, 128).to(torch.bfloat16)
+    assert torch.equal(x.float(), torch.tensor(np.stack(rows)).reshape(1, 2, -1, 128))  # exact in bf16
+    xq, xs = G.quantize_int8(cuda_lib, x.cuda(), per_head=False)
+    rq, rs = Q.quantize_int8_rows(x)
+    assert np.array_equal(_np(xq), rq) and np.array_equal(_np(xs), rs)
+    # per head: one scale 127 * 2^6 for each head, so ties only where x = (j + 1/2) 2^6
+    vq, vsc = G.quantize_int8(cuda_lib, x.cuda(), per_head=True)
+    rvq, rvs = Q.quantize_int8_heads(x)
+    assert np.array_equal(_np(vq), rvq) and np.array_equal(_np(vsc), rvs)
