@@ -85,6 +85,13 @@ int tap_mma_rate(int kind, int n, int iters, int grid, int flags, unsigned long 
  *   tcgen05.st (64 columns) over tensor-memory columns [384, 512) of their
  *   lane quarters while the MMAs run, as the attention softmax does. */
 #define TAP_TMEM_TRAFFIC 256
+/* With TAP_ATTN only: TAP_FLAGPOLL loads a shared-memory word (already set)
+ *   with ld.acquire before the last MMA of every S group; TAP_FLAGFENCE does
+ *   that load and a tcgen05.fence::after_thread_sync before every pair of
+ *   groups -- the same synchronisation points as TAP_TESTWAIT /
+ *   TAP_WAITFENCE, through a plain flag instead of an mbarrier. */
+#define TAP_FLAGPOLL 512
+#define TAP_FLAGFENCE 1024
 /* TAP_TWO_ISSUERS is accepted here together with TAP_ATTN (and optionally
  *   TAP_TESTWAIT | TAP_WAITFENCE): two warps each issue the attention pattern
  *   into their own accumulators (both groups with A from shared memory);

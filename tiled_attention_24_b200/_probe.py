@@ -14,6 +14,7 @@ PROBE_PATH = os.path.join(_PKG, "libtiledattn_probe.so")
 
 KINDS = {"bf16": 0, "int8": 1, "fp8": 2, "fp4": 3}
 A_TMEM, TWO_ACC, TWO_ISSUERS, COMMIT, B_MN, ATTN, TESTWAIT, WAITFENCE, TMEM_TRAFFIC = 1, 2, 4, 8, 16, 32, 64, 128, 256
+FLAGPOLL, FLAGFENCE = 512, 1024
 K_PER_MMA = {"bf16": 16, "int8": 32, "fp8": 32, "fp4": 64}
 
 _lib = None

@@ -251,6 +251,7 @@ __global__ void __launch_bounds__(128, 1) mma_tight_kernel(int iters, unsigned l
     fence_mbar_init();
     mbar_arrive(smem_u32(&bar[2]));  // phase 0 of bar[2] completes at once
     abort_flag[1] = 0;
+    abort_flag[2] = 1;  // the flag the FLAGPOLL / FLAGFENCE variants load
   }
   fence_proxy_async_smem();
   if (threadIdx.x < 32) {
@@ -327,14 +328,25 @@ __global__ void __launch_bounds__(128, 1) mma_tight_kernel(int iters, unsigned l
     const uint32_t done_bar = smem_u32(&bar[2]);
     bool seen = true;
     const long long t0 = clock64();
+    const uint32_t flag_addr = smem_u32(abort_flag + 2);  // a word set to 1 before the loop
+    auto flag_acquire = [&]() -> uint32_t {
+      uint32_t v;
+      asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(flag_addr) : "memory");
+      return v;
+    };
     for (int it = 0; it < iters; ++it) {
       if (SYNC & 2) {  // between groups: a wait on a completed barrier, then the tcgen05 fence
         seen = seen && wait_bar(done_bar, 0, abort_flag, 1000000000ull);
         tc_fence_after();
       }
+      if (SYNC & 32) {  // between groups: an acquire load of a set flag, then the tcgen05 fence
+        seen = (flag_acquire() != 0u) && seen;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         if ((SYNC & 1) && kk == 7) seen = mbar_test_wait(done_bar, 0) && seen;
+        if ((SYNC & 16) && kk == 7) seen = (flag_acquire() != 0u) && seen;
         // 32 bytes of K per MMA: step kk & 3 inside a 128-byte atom, atom kk >> 2
         const uint64_t ao = (uint64_t)(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4);
         const uint64_t bo = (uint64_t)(((kk >> 2) * N * 128 + (kk & 3) * 32) >> 4);
@@ -481,7 +493,8 @@ static int tight_dispatch(int n, int flags, int iters, int grid, unsigned long l
   if (flags & TAP_ATTN) {
     if (n != 128) return -1;
     const int sy = ((flags & TAP_TESTWAIT) ? 1 : 0) | ((flags & TAP_WAITFENCE) ? 2 : 0) |
-                   ((flags & TAP_TMEM_TRAFFIC) ? 4 : 0) | ((flags & TAP_TWO_ISSUERS) ? 8 : 0);
+                   ((flags & TAP_TMEM_TRAFFIC) ? 4 : 0) | ((flags & TAP_TWO_ISSUERS) ? 8 : 0) |
+                   ((flags & TAP_FLAGPOLL) ? 16 : 0) | ((flags & TAP_FLAGFENCE) ? 32 : 0);
     switch (sy) {  // TMEM A initialised
       case 0: return launch_tight<KIND, 128, true, true, 2, 0>(iters, grid, cycles, st);
       case 1: return launch_tight<KIND, 128, true, true, 2, 1>(iters, grid, cycles, st);
@@ -491,10 +504,13 @@ static int tight_dispatch(int n, int flags, int iters, int grid, unsigned long l
       case 7: return launch_tight<KIND, 128, true, true, 2, 7>(iters, grid, cycles, st);
       case 8: return launch_tight<KIND, 128, true, true, 2, 8>(iters, grid, cycles, st);
       case 11: return launch_tight<KIND, 128, true, true, 2, 11>(iters, grid, cycles, st);
+      case 16: return launch_tight<KIND, 128, true, true, 2, 16>(iters, grid, cycles, st);
+      case 32: return launch_tight<KIND, 128, true, true, 2, 32>(iters, grid, cycles, st);
+      case 48: return launch_tight<KIND, 128, true, true, 2, 48>(iters, grid, cycles, st);
       default: return -1;
     }
   }
-  if (flags & (TAP_TESTWAIT | TAP_WAITFENCE | TAP_TMEM_TRAFFIC)) return -1;
+  if (flags & (TAP_TESTWAIT | TAP_WAITFENCE | TAP_TMEM_TRAFFIC | TAP_FLAGPOLL | TAP_FLAGFENCE)) return -1;
   if (n == 128) {
     if (at) return cm ? launch_tight<KIND, 128, true, true>(iters, grid, cycles, st)
                       : launch_tight<KIND, 128, true, false>(iters, grid, cycles, st);
@@ -511,7 +527,7 @@ TAP_API int tap_mma_tight_rate(int kind, int n, int iters, int grid, int flags, 
                                void* stream) {
   if (iters < 1 || grid < 1 || !cycles || (n != 128 && n != 256)) return -1;
   if (flags & ~(TAP_A_TMEM | TAP_COMMIT | TAP_B_MN | TAP_ATTN | TAP_TESTWAIT | TAP_WAITFENCE | TAP_TMEM_TRAFFIC |
-                TAP_TWO_ISSUERS))
+                TAP_TWO_ISSUERS | TAP_FLAGPOLL | TAP_FLAGFENCE))
     return -1;
   if ((flags & TAP_TWO_ISSUERS) && !(flags & TAP_ATTN)) return -1;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
