@@ -16,7 +16,6 @@ plus its mean; the error relative to the bound is reported.  For N(0,1)
 inputs the bound is below 1e-2 and the plain 2e-2 applies.
 """
 import numpy as np
-import torch
 
 O_MAX_ABS = 2e-2
 O_MEAN_ABS = 2e-3

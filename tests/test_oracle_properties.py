@@ -4,7 +4,6 @@ tests.  Sizes stay small so the whole file runs in seconds."""
 import math
 
 import numpy as np
-import pytest
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 

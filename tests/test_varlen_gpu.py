@@ -4,7 +4,6 @@ tolerances as the bf16 path (max-abs 2e-2, mean-abs 2e-3 on O, 1e-3 on LSE).
 Outputs and workspaces sit between guard bands (tests._guard): the varlen
 epilogue stores rows directly, so a row past its sequence would land in the
 next sequence's rows or past the packed tensor."""
-import numpy as np
 import pytest
 import torch
 
