@@ -19,10 +19,13 @@ if ROOT not in sys.path:
 from workloads import make_qkv, make_varlen  # noqa: E402
 
 # lazy rescale: key blocks scaled by `gains` (block j by gains[min(j, -1)])
-LAZY = [(pattern, causal, d) for pattern in ("steps", "mixed") for causal in (False, True) for d in (64, 128)]
+# (N = 768 at d = 128: whole query tile pairs; 700: a ragged last pair)
+LAZY = [(pattern, causal, d, N) for pattern in ("steps", "mixed") for causal in (False, True) for d in (64, 128)
+        for N in ((700, 768) if d == 128 else (700,))]
 GAINS = {"steps": [1, 4, 8, 16, 32], "mixed": [1, 3]}
 # causal skipping: (B, H, Nq, Nkv, d)
-CAUSAL = [(1, 3, 1000, 1000, 128), (2, 2, 300, 1000, 64), (1, 2, 1000, 300, 128), (1, 1, 129, 4000, 64)]
+CAUSAL = [(1, 3, 1000, 1000, 128), (2, 2, 300, 1000, 64), (1, 2, 1000, 300, 128), (1, 1, 129, 4000, 64),
+          (1, 3, 1024, 1024, 128), (1, 2, 512, 1000, 128)]
 
 
 def lazy_inputs(pattern, d, N=700):
@@ -78,9 +81,9 @@ def main():
         status = ta.attn_check_status()
         out[group][name] = {"counters": ta.attn_debug_counters(reset=True), "status": status}
 
-    for pattern, causal, d in LAZY:
-        q, k, v = (t.to(dev) for t in lazy_inputs(pattern, d))
-        record("lazy", f"{pattern}-{int(causal)}-{d}", lambda: ta.forward(q, k, v, causal, d ** -0.5))
+    for pattern, causal, d, N in LAZY:
+        q, k, v = (t.to(dev) for t in lazy_inputs(pattern, d, N))
+        record("lazy", f"{pattern}-{int(causal)}-{d}-{N}", lambda: ta.forward(q, k, v, causal, d ** -0.5))
     for B, H, Nq, Nkv, d in CAUSAL:
         q, k, v = (t.to(dev) for t in causal_inputs(B, H, Nq, Nkv, d))
         record("causal", f"{B}-{H}-{Nq}-{Nkv}-{d}", lambda: ta.forward(q, k, v, True, d ** -0.5))

@@ -83,3 +83,21 @@ def test_traffic_record_is_dropped_when_the_sources_change(tmp_path, monkeypatch
     data["sources"] = "0" * 16
     out.write_text(json.dumps(data))
     assert traffic.load(str(out)) == {}
+
+
+def test_traffic_digest_covers_every_kernel_source():
+    """Every source file libtiledattn.so is compiled from (api.cu and the
+    headers it includes) is part of the digest, so that no kernel can change
+    under a stale traffic record."""
+    import re
+    from tiled_attention_24_b200 import traffic
+    csrc = os.path.join(traffic.PKG, traffic._LIB_SOURCES[0])
+    seen, todo = set(), ["api.cu"]
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        with open(os.path.join(csrc, f)) as fh:
+            todo += [m for m in re.findall(r'#include "([^"]+)"', fh.read()) if os.path.exists(os.path.join(csrc, m))]
+    assert seen <= set(traffic._LIB_SOURCES[1]), sorted(seen - set(traffic._LIB_SOURCES[1]))

@@ -73,14 +73,14 @@ def _all_masked_tiles(B, H, Nq, Nkv):
     return B * H * n
 
 
-@pytest.mark.parametrize("case", C.LAZY, ids=lambda c: f"{c[0]}-causal{int(c[1])}-d{c[2]}")
+@pytest.mark.parametrize("case", C.LAZY, ids=lambda c: f"{c[0]}-causal{int(c[1])}-d{c[2]}-N{c[3]}")
 def test_rescale_count_matches_oracle(child, case):
-    pattern, causal, d = case
-    got = child["lazy"][f"{pattern}-{int(causal)}-{d}"]
+    pattern, causal, d, N = case
+    got = child["lazy"][f"{pattern}-{int(causal)}-{d}-{N}"]
     assert got["status"] == 0 and got["counters"][2] == 0
-    q, k, v = C.lazy_inputs(pattern, d)
+    q, k, v = C.lazy_inputs(pattern, d, N)
     total, slack, near = _expected_moves(q, k, v, causal, d)
-    print(f"{pattern} causal={causal} d={d}: device {got['counters'][0]}, oracle {total} "
+    print(f"{pattern} causal={causal} d={d} N={N}: device {got['counters'][0]}, oracle {total} "
           f"({near} rows within {BAND} of the threshold, slack {slack})")
     assert total > 0
     assert abs(got["counters"][0] - total) <= slack

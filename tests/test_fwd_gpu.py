@@ -68,6 +68,35 @@ def test_ragged_shapes(cuda_lib, shape, causal):
     assert_bf16_close(o, lse, O, L, f"{shape} causal={causal}")
 
 
+# Many (head, query-pair) CTAs at d = 128: more CTAs than SMs, so that every
+# SM runs several in turn; N_kv <= 128 gives CTAs of a single key block (one
+# step, whose stage carries only V_0); ragged key tails and N_kv > N_q move
+# the diagonal and tail masks off the tile grid.
+MANY_CTAS = [
+    # B, H, Nq, Nkv
+    (1, 1, 256, 256),
+    (1, 2, 512, 300),
+    (2, 3, 768, 1000),
+    (1, 2, 256, 1),
+    (1, 160, 256, 128),
+    (1, 170, 256, 100),
+    (1, 160, 256, 300),
+    (2, 90, 512, 700),
+    (1, 40, 1024, 1024),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", MANY_CTAS, ids=lambda s: "x".join(map(str, s)))
+def test_many_ctas_and_short_key_ranges(cuda_lib, shape, causal):
+    B, H, Nq, Nkv = shape
+    q, k, v = make_qkv("prefill", seed=Nq + Nkv + H, B=B, H=H, Nq=Nq, Nkv=Nkv, d=128)
+    scale = 128 ** -0.5
+    o, lse = run(cuda_lib, q, k, v, causal, scale)
+    O, L = A.attention(q, k, v, causal, scale)
+    assert_bf16_close(o, lse, O, L, f"{shape} causal={causal}")
+
+
 def test_causal_future_keys_do_not_matter(cuda_lib):
     q, k, v = make_qkv("prefill", seed=3, B=1, H=2, Nq=384, Nkv=384, d=128)
     o1, l1 = run(cuda_lib, q, k, v, True, 128 ** -0.5)
@@ -145,24 +174,26 @@ def _growing_keys(q_seed, B, H, N, d, gains):
     return q, k.to(torch.bfloat16), v
 
 
+@pytest.mark.parametrize("N", [700, 768])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("pattern", ["steps", "mixed"])
-def test_lazy_rescale_correction(cuda_lib, pattern, causal, d):
+def test_lazy_rescale_correction(cuda_lib, pattern, causal, d, N):
     """'steps': block gains 1, 4, 8, 16, 32 -- every row's max rises by far
     more than 8 at each of the first blocks, so every warp corrects O
     repeatedly.  'mixed': gains 1, 3, 3, ... -- the rise at block 1 is close
     to the threshold, so within one warp some rows rescale and others keep a
-    stale reference (the correction factor is then 1 for them)."""
+    stale reference (the correction factor is then 1 for them).  N = 768
+    fills every query tile pair; N = 700 leaves a ragged last pair."""
     gains = [1, 4, 8, 16, 32] if pattern == "steps" else [1, 3]
-    q, k, v = _growing_keys(17 + d, 1, 2, 700, d, gains)
+    q, k, v = _growing_keys(17 + d, 1, 2, N, d, gains)
     scale = d ** -0.5
     o, lse = run(cuda_lib, q, k, v, causal, scale)
     O, L, n_resc = A.attention_lazy_rescale(q, k, v, causal, scale, tau=8.0, count_rescales=True)
     Od, Ld = A.attention(q, k, v, causal, scale)
     assert np.abs(O - Od).max() < 1e-9                     # the lazy form is the definition
-    rows = 2 * 700
-    print(f"lazy rescale {pattern} d={d} causal={causal}: {n_resc} rescales over {rows} rows")
+    rows = 2 * N
+    print(f"lazy rescale {pattern} d={d} N={N} causal={causal}: {n_resc} rescales over {rows} rows")
     assert n_resc >= (rows // 2 if pattern == "steps" else 50)
     if pattern == "mixed":
         _, _, n_moved_any = A.attention_lazy_rescale(q, k, v, causal, scale, tau=0.0, count_rescales=True)

@@ -96,9 +96,10 @@ struct FwdCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
-  // register split (launch: 384 threads x 168): warpgroup 0 drops to 80,
-  // the two softmax warpgroups rise to 208: 128*80 + 256*208 = 63488 <= 384*168
-  static constexpr int REG_LOW = 80, REG_HIGH = 208;
+  // register split (launch: 384 threads x 168): warpgroup 0 drops to 80 (72
+  // at d = 64), the two softmax warpgroups rise to 208 (216):
+  // 128*80 + 256*208 = 63488 and 128*72 + 256*216 = 64512 <= 384*168
+  static constexpr int REG_LOW = (D == 64) ? 72 : 80, REG_HIGH = (D == 64) ? 216 : 208;
   // d = 64: P gets its own TMEM columns (S_0, S_1 [0,256), P_0, P_1 [256,384),
   // O_0, O_1 [384,512)), so a tile's next S is issued as soon as its softmax
   // holds the current scores, not after its P V.  d = 128: no room; P aliases S.

@@ -77,7 +77,8 @@ struct FwdF4Cfg {
   static constexpr int PSF_OFF = P_OFF + 4 * TILE;        // [tile][buffer] P scales
   static constexpr int ONES_OFF = PSF_OFF + 4 * SF;      // 16 x 128 e2m1 ones (0x22 bytes)
   static constexpr int SF1_OFF = ONES_OFF + 1024;        // 512 bytes of scale 1.0 (0x38)
-  static constexpr int BAR_OFF = SF1_OFF + 512;
+  static constexpr int RCP_OFF = SF1_OFF + 512;          // 128 floats: 1 / value of each e4m3 code
+  static constexpr int BAR_OFF = RCP_OFF + 512;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;
   static constexpr int THREADS = 384;
   // register split (launch: 384 threads x 168): warpgroup 0 drops to 72, the
@@ -218,6 +219,12 @@ __global__ void __launch_bounds__(384, 1)
   // constant operands of the row-sum MMA: e2m1 ones (code 2) and their scales (1.0)
   for (int i = threadIdx.x; i < (1024 + 512) / 4; i += C::THREADS)
     *reinterpret_cast<uint32_t*>(smem + C::ONES_OFF + i * 4) = (i < 256) ? 0x22222222u : 0x38383838u;
+  // reciprocals of the e4m3 block scales of P (quantise-after-exp), correctly
+  // rounded once here instead of once per 16 keys in the softmax (0 for code 0)
+  if (threadIdx.x < 128) {
+    const float v = e4m3_value(threadIdx.x);
+    reinterpret_cast<float*>(smem + C::RCP_OFF)[threadIdx.x] = (v > 0.f) ? __frcp_rn(v) : 0.f;
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -389,6 +396,7 @@ __global__ void __launch_bounds__(384, 1)
     const int off = p.Nkv - p.Nq;
     const float sl2 = p.sl2;
     const bool direct = p.p_mode == 0;
+    const float* rcp_tab = reinterpret_cast<const float*>(smem + C::RCP_OFF);
     float m_ref = -INFINITY;  // l lives in TMEM (column tL), summed by the tensor core
     bool ok = present[t];
     if (!SCORES_ONLY && direct) {
@@ -482,9 +490,8 @@ __global__ void __launch_bounds__(384, 1)
           const float a4 = fmax3(__uint_as_float(v[12]), __uint_as_float(v[13]), __uint_as_float(v[14]));
           const float amax = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, __uint_as_float(v[15])), 0.f);
           const uint32_t sfc = (amax > 0.f) ? e4m3_rne(__fdiv_rn(fmaxf(amax, 1e-30f), 6.f)) : 0u;
-          const float sc = e4m3_value(sfc);
           psf[sf_offset(rr, blk)] = (uint8_t)sfc;
-          rs[blk] = (sc > 0.f) ? __frcp_rn(sc) : 0.f;
+          rs[blk] = rcp_tab[sfc];  // p <= 1, so amax / 6 <= 1/6 and sfc < 128
         }
       }
 #pragma unroll

@@ -450,20 +450,28 @@ __global__ void __launch_bounds__(FwdI8Cfg::THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const float f = (grow && had) ? factor : 1.f;
-#pragma unroll 1
+        // every chunk of ACC and OF requested before the first wait (one
+        // tensor-memory round trip instead of one per chunk)
+        uint32_t a[NCH][32], o[NCH][32];
+#pragma unroll
         for (int cc = 0; cc < NCH; ++cc) {
-          uint32_t a[32], o[32];
-          tmem_ld32(tACC + cc * 32, a);
-          tmem_ld32(tOF + cc * 32, o);
-          tmem_ld_wait(a);
-          tmem_ld_wait(o);
+          tmem_ld32(tACC + cc * 32, a[cc]);
+          tmem_ld32(tOF + cc * 32, o[cc]);
+        }
+#pragma unroll
+        for (int cc = 0; cc < NCH; ++cc) {
+          tmem_ld_wait(a[cc]);
+          tmem_ld_wait(o[cc]);
+        }
+#pragma unroll
+        for (int cc = 0; cc < NCH; ++cc) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            o[i] = __float_as_uint((__uint_as_float(o[i]) + (float)(int)a[i] * sv127) * f);
-            a[i] = 0u;
+            o[cc][i] = __float_as_uint((__uint_as_float(o[cc][i]) + (float)(int)a[cc][i] * sv127) * f);
+            a[cc][i] = 0u;
           }
-          tmem_st32(tOF + cc * 32, o);
-          tmem_st32(tACC + cc * 32, a);
+          tmem_st32(tOF + cc * 32, o[cc]);
+          tmem_st32(tACC + cc * 32, a[cc]);
         }
       }
       tmem_st_wait();

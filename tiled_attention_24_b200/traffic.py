@@ -27,8 +27,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 PATH = os.path.join(ROOT, "profiles", "traffic.json")
-_LIB_SOURCES = ("csrc", ("api.cu", "bwd_bf16.cuh", "decode.cuh", "exp2_poly.cuh", "fwd_bf16.cuh", "fwd_fp4.cuh",
-                         "fwd_fp8.cuh", "fwd_int8.cuh", "ptx.cuh", "quant.cuh"))
+_LIB_SOURCES = ("csrc", ("api.cu", "bwd_bf16.cuh", "decode.cuh", "decode_tc.cuh", "exp2_poly.cuh", "fwd_bf16.cuh",
+                         "fwd_fp4.cuh", "fwd_fp8.cuh", "fwd_int8.cuh", "ptx.cuh", "quant.cuh"))
 
 
 def library_digest() -> str:
