@@ -213,7 +213,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = make_tmap_bf16(&tv, v, D, Nkv, B * Hkv)) != ATTN_OK) return rc;
   if ((rc = make_tmap_bf16(&to, o, D, Nq, BH)) != ATTN_OK) return rc;
   if ((rc = set_smem_attr(ta::fwd_bf16_kernel<D>, C::SMEM)) != ATTN_OK) return rc;
-  ta::FwdParams p;
+  ta::FwdParams p{};
   p.lse = lse;
   p.Nq = Nq;
   p.Nkv = Nkv;
@@ -223,6 +223,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal = causal ? 1 : 0;
   p.sl2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_ns;
+  {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    p.wave = sms;  // one CTA per SM (shared memory)
+  }
   const long long grid = (long long)BH * p.n_qp;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   ta::fwd_bf16_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, to, p);
@@ -240,7 +246,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   if ((rc = make_tmap_tok(&tk, k, D, Hkv, total_k)) != ATTN_OK) return rc;
   if ((rc = make_tmap_tok(&tv, v, D, Hkv, total_k)) != ATTN_OK) return rc;
   if ((rc = set_smem_attr(ta::fwd_bf16_kernel<D, true>, C::SMEM)) != ATTN_OK) return rc;
-  ta::FwdParams p;
+  ta::FwdParams p{};
   p.lse = lse;
   p.Nq = 0;
   p.Nkv = 0;

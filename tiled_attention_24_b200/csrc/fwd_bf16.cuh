@@ -11,6 +11,9 @@
 // CTA = one (batch, head) and TWO query tiles of 128 rows (256 rows).  Roles
 // (warp specialisation, "FlashAttention 4" section "What is new"):
 //   warp 0      TMA producer: Q tiles once, then K_j, V_j into a smem ring
+//               (Q and K_0 issued before the CTA-wide barrier; near its end
+//               it prefetches into L2 the first tiles of the CTA one wave
+//               later, the likely next occupant of the SM)
 //   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
 //   warps 2-3   idle (they complete warpgroup 0, whose registers are handed
 //               to the softmax warpgroups with setmaxnreg)
@@ -81,6 +84,7 @@ struct FwdParams {
   const int* cu_k;  // [nb + 1] key offsets in the packed K / V
   uint16_t* o;      // packed O [total_q][H][D]
   int nb, H, total_q, total_k;
+  int wave;  // CTAs resident at once (one per SM): CTA b prefetches CTA b + wave's first tiles into L2
 };
 
 template <int D>
@@ -207,6 +211,35 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
+    // the producer thread starts the Q and K_0 copies before the CTA-wide
+    // barrier, so that their latency overlaps the TMEM allocation (the barrier
+    // words it just wrote are made visible to the async proxy first)
+    fence_proxy_async_smem();
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    const uint32_t qbar = smem_u32(&bars->q_full);
+    mbar_arrive_expect_tx(qbar, (present[0] + present[1]) * C::TILE);
+    for (int t = 0; t < 2; ++t) {
+      if (!present[t]) continue;
+      for (int h = 0; h < D / 64; ++h) {
+        if constexpr (VARLEN)
+          tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, head, qstart + r0[t]);
+        else
+          tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
+      }
+    }
+    if (nmax > 0) {  // stage 0: K_0 only (its slot has never been used: no empty wait)
+      const uint32_t fb = smem_u32(&bars->kv_full[0]);
+      mbar_arrive_expect_tx(fb, C::TILE);
+      const int kvh0 = head / p.group;
+      for (int h = 0; h < D / 64; ++h) {
+        if constexpr (VARLEN)
+          tma_load_3d(sbase + C::SLOT_OFF + C::TILE + h * C::HALF, &tmK, fb, h * 64, kvh0, kstart);
+        else
+          tma_load_3d(sbase + C::SLOT_OFF + C::TILE + h * C::HALF, &tmK, fb, h * 64, 0, kvh0);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
@@ -222,28 +255,27 @@ __global__ void __launch_bounds__(384, 1)
    if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       const uint32_t qbar = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qbar, (present[0] + present[1]) * C::TILE);
-      for (int t = 0; t < 2; ++t) {
-        if (!present[t]) continue;
-        for (int h = 0; h < D / 64; ++h) {
-          if constexpr (VARLEN)
-            tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, head, qstart + r0[t]);
-          else
-            tma_load_3d(sbase + C::Q_OFF + t * C::TILE + h * C::HALF, &tmQ, qbar, h * 64, r0[t], bh);
-        }
-      }
       const int kvh = head / p.group;  // key/value head of this query head
-      // stage i (0..nmax): V_{i-1} at +0 (none for i = 0), K_i at +TILE (none for i = nmax)
-      int it = 0, slot = 0;
-      uint32_t ph = 0;
+      // stage i (0..nmax): V_{i-1} at +0 (none for i = 0), K_i at +TILE (none
+      // for i = nmax); stage 0 was issued before the CTA-wide barrier
+      int it = 1, slot = 1 % C::NSTAGE;
+      uint32_t ph = (C::NSTAGE == 1) ? 1u : 0u;
       bool ok = true;
-      for (int i = 0; nmax > 0 && i <= nmax && ok; ++i, ++it, (++slot == C::NSTAGE) ? (slot = 0, ph ^= 1u) : 0u) {
+      for (int i = 1; nmax > 0 && i <= nmax && ok; ++i, ++it, (++slot == C::NSTAGE) ? (slot = 0, ph ^= 1u) : 0u) {
         ok = wait_bar(smem_u32(&bars->kv_empty[slot]), ph ^ 1, abort_flag, p.timeout_ns);
         if (!ok) break;
+        if (!VARLEN && p.wave > 0 && i == max(1, nmax - 4) && blockIdx.x + p.wave < gridDim.x) {
+          // the CTA that will most likely take this SM next (one wave later):
+          // its Q tiles and first K tile into L2 now
+          const int nb2 = blockIdx.x + p.wave;
+          const int bh2 = p.causal ? (int)(nb2 % BH) : (int)(nb2 / p.n_qp);
+          const int qp2 = p.causal ? p.n_qp - 1 - (int)(nb2 / BH) : (int)(nb2 % p.n_qp);
+          for (int t = 0; t < 2; ++t)
+            if (qp2 * 256 + t * 128 < Nq)
+              for (int h = 0; h < D / 64; ++h) tma_prefetch_3d(&tmQ, h * 64, qp2 * 256 + t * 128, bh2);
+          for (int h = 0; h < D / 64; ++h) tma_prefetch_3d(&tmK, h * 64, 0, bh2 / p.group);
+        }
         const uint32_t fb = smem_u32(&bars->kv_full[slot]);
         mbar_arrive_expect_tx(fb, ((i > 0) + (i < nmax)) * C::TILE);
         const uint32_t dst = sbase + C::SLOT_OFF + slot * C::STAGE;
