@@ -669,11 +669,8 @@ __global__ void __launch_bounds__(384, 1)
               (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       } else {
       uint8_t* stage = smem + C::Q_OFF + t * C::TILE;  // Q_t is no longer read
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait(o);
+      // columns [32 cc, 32 cc + 32) of O_t / l -> bf16 -> the swizzled staging tile
+      auto emit = [&](int cc, const uint32_t (&o)[32]) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           uint32_t w[4];
@@ -687,6 +684,25 @@ __global__ void __launch_bounds__(384, 1)
           const int h = c16 >> 3, ch = c16 & 7;
           uint8_t* dst = stage + h * C::HALF + rr * 128 + ((ch ^ (rr & 7)) << 4);
           *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      };
+      if constexpr (D == 128) {
+        // every column requested before one wait (the scores' registers are
+        // free by now): one tensor-memory round trip instead of four
+        uint32_t oall[D / 32][32];
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tO + cc * 32, oall[cc]);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(oall[cc]);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) emit(cc, oall[cc]);
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+          emit(cc, o);
         }
       }
       if (row < Nq)
