@@ -5,8 +5,8 @@ built from, so that a kernel change turns every recorded figure stale.
 Record (after captures of the launch list with those two metrics, one pass):
 
     python -m tiled_attention_24_b200.traffic \\
-        fwd_bf16_prefill_noncausal=gpurun_out/fwd_traffic.csv:0 \\
-        decode_split=gpurun_out/decode_traffic.csv:0:8 ...
+        fwd_bf16_prefill_noncausal=fwd_traffic.csv:0 \\
+        decode_split=decode_traffic.csv:0:8 ...
 
 Each argument is KEY=CSV:ID[:SCALE]: the launch with that ID in an ncu
 `--csv` log, its read + write bytes times SCALE (a smaller capture scaled to
